@@ -1,0 +1,284 @@
+"""Plain fp64 CPU oracle for Monarch-factorised video attention (forward).
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path may import, call or
+execute this module: only the tests, ``__graft_entry__.smoke()`` and the
+benchmark's CPU-baseline leg use it.  It shares no code with the CUDA library
+and imports nothing from the product package.
+
+What it computes
+----------------
+MonarchRT (arXiv 2602.12271, "MonarchRT: Efficient Attention for Real-Time
+Video Generation") replaces dense 3D self-attention softmax(S)V over a
+T x H x W token grid by an attention matrix constrained to Monarch form,
+M = P blockdiag(L) P^T blockdiag(R) (abstract; gist.science explainer §2
+"Methodology: MonarchRT"), with blocks aligned to the video grid (§2.A
+"Block Alignment") and tiled inside a frame (§2.B "Tiled Monarch
+Parameterization").  L and R come from the alternating refinement of the
+original MonarchAttention algorithm (§2.C "Finetuning and Efficient
+Implementation": "iterative refinement", one step after finetuning).  The
+pages give no equations; the reading implemented here is:
+
+  grid -> blocks  token (t, y, x) of a frame grid with tiles th x tw maps to
+                  tile  c1 = (t*(H/th) + y//th)*(W/tw) + x//tw   (block axis 1)
+                  pos   c2 = (y % th)*tw + x % tw                (block axis 2)
+  D1  M[(a1,a2),(c1,c2)] = L_{a2}[a1,c1] * R_{c1}[a2,c2]
+  D2  scores S = s * q.k, s = 1/sqrt(d)
+  D3  initial L: block identity (self-attention); for a KV cache with
+      key frames Tk > query frames T, the eps -> 0 limit of
+      (1-eps)[c1 == a1 + (Tk-T)P] + eps/|visible(a1)|
+  D4  R step:  beta = sum_a1 L,  q~ = (sum_a1 L q)/beta,
+               R_{c1}[a2,:] = softmax_c2(s q~[c1,a2].k[c1,c2])
+  D5  h[c1,a2] = -sum_c2 R log R
+  D6  L step:  k~ = sum_c2 R k,
+               L_{a2}[a1,:] = softmax_c1(s q[a1,a2].k~[c1,a2] + h[c1,a2])
+  D7  one iteration = one R step then one L step
+  D8  output:  z = sum_c2 R v,  y = sum_c1 L z,  out = y scattered back to
+               the grid order
+
+D4 and D6 are the exact block maximisers of the variational softmax
+objective F(M) = sum_rows <M_row, S_row> + H(M_row) (whose unconstrained
+maximiser over row-stochastic M is softmax(S)); this is what the tests pin.
+
+Everything here is fp64 numpy; ``np.matmul`` is the only library primitive
+used as a step.  Loops run over (batch, head) so memory stays one head deep.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class Grid:
+    """Token grid and tiling.  T query frames, Tk key frames (Tk == T is
+    self-attention), frame H x W, spatial tile th x tw."""
+
+    T: int
+    H: int
+    W: int
+    th: int
+    tw: int
+    Tk: int | None = None
+
+    @property
+    def Tkey(self) -> int:
+        return self.T if self.Tk is None else self.Tk
+
+    @property
+    def tiles_per_frame(self) -> int:
+        return (self.H // self.th) * (self.W // self.tw)
+
+    @property
+    def b2(self) -> int:
+        return self.th * self.tw
+
+    @property
+    def b1q(self) -> int:
+        return self.T * self.tiles_per_frame
+
+    @property
+    def b1k(self) -> int:
+        return self.Tkey * self.tiles_per_frame
+
+    @property
+    def Nq(self) -> int:
+        return self.T * self.H * self.W
+
+    @property
+    def Nk(self) -> int:
+        return self.Tkey * self.H * self.W
+
+    def check(self) -> None:
+        if self.H % self.th or self.W % self.tw:
+            raise ValueError("tile must divide the frame")
+        if self.Tkey < self.T:
+            raise ValueError("key frames must include the query chunk")
+
+
+def block_index(frames: int, H: int, W: int, th: int, tw: int) -> np.ndarray:
+    """idx[c1, c2] = grid token index n = (t*H + y)*W + x of tile c1,
+    position c2 (block alignment, gist.science explainer §2.A; tiling §2.B).
+
+    Written as an explicit loop over grid tokens so it reads like the
+    definition of the map."""
+    nty, ntx = H // th, W // tw
+    P = nty * ntx
+    idx = np.empty((frames * P, th * tw), dtype=np.int64)
+    for t in range(frames):
+        for y in range(H):
+            for x in range(W):
+                c1 = (t * nty + y // th) * ntx + x // tw
+                c2 = (y % th) * tw + x % tw
+                idx[c1, c2] = (t * H + y) * W + x
+    return idx
+
+
+def _softmax_last(x: np.ndarray) -> np.ndarray:
+    m = x.max(axis=-1, keepdims=True)
+    e = np.exp(x - m)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+def _logsumexp_last(x: np.ndarray) -> np.ndarray:
+    m = x.max(axis=-1)
+    return m + np.log(np.exp(x - m[..., None]).sum(axis=-1))
+
+
+def initial_qtilde(qb: np.ndarray, grid: Grid) -> np.ndarray:
+    """q~ of the first R step (D3 + D4) for one head.
+
+    qb: [b1q, b2, d] queries in block order.  Returns [b1k, b2, d].
+
+    Self-attention: L0 is the block identity, so beta = 1 and q~[c1] = q[c1].
+    KV cache (Tk > T): the query chunk is the last T frames of the key
+    sequence, so query tile a1 is aligned with key tile a1 + (Tk-T)P.  With
+    L0 = (1-eps)*aligned + eps*uniform-over-visible, an aligned key tile gets
+    its own query tile as eps -> 0, and an earlier (cached) key tile gets the
+    mean of q over the query tiles that see it, weighted by 1/|visible(a1)|.
+    Every cached frame precedes the query chunk, so every query tile sees
+    every key tile and the weights are uniform.  (The pages describe the
+    KV-cache regime -- autoregressive chunks attending to cached frames,
+    gist.science explainer §1 and §4 -- but not this initialisation.)
+    """
+    b1q, b2, d = qb.shape
+    if grid.Tkey == grid.T:
+        return qb.copy()
+    off = (grid.Tkey - grid.T) * grid.tiles_per_frame
+    b1k = grid.b1k
+    visible = np.ones((b1q, b1k), dtype=bool)  # the query chunk sees all keys
+    w = 1.0 / visible.sum(axis=1)  # 1/|visible(a1)|
+    qt = np.empty((b1k, b2, d))
+    for c1 in range(b1k):
+        if c1 >= off:
+            qt[c1] = qb[c1 - off]
+        else:
+            wa = w * visible[:, c1]
+            qt[c1] = np.einsum("a,apd->pd", wa, qb) / wa.sum()
+    return qt
+
+
+@dataclass
+class HeadState:
+    """Factors and intermediates of one head after the last iteration."""
+
+    qt: np.ndarray  # [b1k, b2, d]   q~ used by the last R step
+    R: np.ndarray  # [b1k, b2, b2]  R_{c1}[a2, c2]
+    h: np.ndarray  # [b1k, b2]      entropy of R_{c1}[a2, :]
+    kt: np.ndarray  # [b1k, b2, d]   k~[c1, a2]
+    L: np.ndarray  # [b2, b1q, b1k] L_{a2}[a1, c1]
+    lse: np.ndarray  # [b2, b1q]     log-sum-exp of the last L step's rows
+    z: np.ndarray  # [b1k, b2, d]   z[c1, a2] = sum_c2 R v
+    y: np.ndarray  # [b1q, b2, d]   output in block order
+    objective: list  # F(M) after every iteration
+
+
+def _r_step(qt: np.ndarray, kb: np.ndarray, scale: float):
+    """D4 + D5 for one head: qt, kb [b1k, b2, d] -> R [b1k, b2, b2], h [b1k, b2]."""
+    s_r = scale * np.matmul(qt, np.swapaxes(kb, 1, 2))  # [c1, a2, c2]
+    R = _softmax_last(s_r)
+    h = -(R * np.log(R)).sum(axis=-1)
+    return R, h
+
+
+def _l_step(qb: np.ndarray, kt: np.ndarray, h: np.ndarray, scale: float):
+    """D6 for one head: qb [b1q,b2,d], kt [b1k,b2,d], h [b1k,b2] ->
+    L [b2, b1q, b1k], lse [b2, b1q]."""
+    qp = np.swapaxes(qb, 0, 1)  # [a2, a1, d]
+    kp = np.swapaxes(kt, 0, 1)  # [a2, c1, d]
+    s_l = scale * np.matmul(qp, np.swapaxes(kp, 1, 2)) + h.T[:, None, :]
+    return _softmax_last(s_l), _logsumexp_last(s_l)
+
+
+def _column_qtilde(L: np.ndarray, qb: np.ndarray) -> np.ndarray:
+    """D4's aggregation for one head: q~[c1,a2] = sum_a1 L q / sum_a1 L."""
+    beta = L.sum(axis=1)  # [a2, c1]
+    num = np.matmul(np.swapaxes(L, 1, 2), np.swapaxes(qb, 0, 1))  # [a2, c1, d]
+    return np.swapaxes(num / beta[:, :, None], 0, 1)  # [c1, a2, d]
+
+
+def head_objective(L, R, qb, kb, scale) -> float:
+    """F(M) = sum_rows <M, S> + H(M) for the Monarch M of one head, written
+    through the factors: M[(a1,a2),(c1,c2)] = L_{a2}[a1,c1] R_{c1}[a2,c2]."""
+    S = scale * np.einsum("apd,cjd->apcj", qb, kb)
+    M = np.einsum("pac,cpj->apcj", L, R)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ent = np.where(M > 0, -M * np.log(M), 0.0)
+    return float((M * S).sum() + ent.sum())
+
+
+def monarch_head(qb, kb, vb, grid: Grid, iters: int, scale: float,
+                 track_objective: bool = False) -> HeadState:
+    """One (batch, head): qb [b1q,b2,d], kb/vb [b1k,b2,d] in block order."""
+    if iters < 1:
+        raise ValueError("iters must be >= 1")
+    qt = initial_qtilde(qb, grid)
+    obj = []
+    L = None
+    for it in range(iters):
+        if it > 0:
+            qt = _column_qtilde(L, qb)  # L of the previous iteration
+        R, h = _r_step(qt, kb, scale)
+        kt = np.matmul(R, kb)  # k~[c1, a2] = sum_c2 R k
+        L, lse = _l_step(qb, kt, h, scale)
+        if track_objective:
+            obj.append(head_objective(L, R, qb, kb, scale))
+    z = np.matmul(R, vb)  # [c1, a2, d]
+    y = np.swapaxes(np.matmul(L, np.swapaxes(z, 0, 1)), 0, 1)  # [a1, a2, d]
+    return HeadState(qt=qt, R=R, h=h, kt=kt, L=L, lse=lse, z=z, y=y,
+                     objective=obj)
+
+
+def monarch_attention(q, k, v, grid: Grid, iters: int, scale: float | None = None,
+                      heads=None, return_states: bool = False):
+    """Monarch attention forward.
+
+    q: [B, Hh, Nq, d]; k, v: [B, Hh, Nk, d], tokens in grid order (t, y, x).
+    Returns out [B, Hh, Nq, d] (fp64).  ``heads`` optionally restricts the
+    computation to a list of (b, h) pairs (other rows of ``out`` stay NaN);
+    heads are independent, so a subset is an exact sample.
+    """
+    grid.check()
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Hh, Nq, d = q.shape
+    assert Nq == grid.Nq and k.shape[2] == grid.Nk and v.shape[2] == grid.Nk
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    iq = block_index(grid.T, grid.H, grid.W, grid.th, grid.tw)
+    ik = block_index(grid.Tkey, grid.H, grid.W, grid.th, grid.tw)
+    out = np.full(q.shape, np.nan)
+    states = {}
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(Hh)]
+    for b, h in todo:
+        st = monarch_head(q[b, h][iq], k[b, h][ik], v[b, h][ik], grid, iters, scale)
+        out[b, h][iq] = st.y
+        if return_states:
+            states[(b, h)] = st
+    return (out, states) if return_states else out
+
+
+def dense_attention(q, k, v, scale: float | None = None):
+    """Textbook softmax(s q k^T) v per (batch, head), fp64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    if scale is None:
+        scale = 1.0 / np.sqrt(q.shape[-1])
+    s = scale * np.matmul(q, np.swapaxes(k, -1, -2))
+    return np.matmul(_softmax_last(s), v)
+
+
+def monarch_flops(grid: Grid, d: int, iters: int, B: int = 1, heads: int = 1) -> float:
+    """Algorithmic FLOPs of one forward: 2*iters*F_L + (2*iters+1)*F_R per head,
+    F_L = 2*b2*b1q*b1k*d (one L-sized contraction), F_R = 2*b1k*b2^2*d."""
+    FL = 2.0 * grid.b2 * grid.b1q * grid.b1k * d
+    FR = 2.0 * grid.b1k * grid.b2 * grid.b2 * d
+    return B * heads * (2 * iters * FL + (2 * iters + 1) * FR)
+
+
+def dense_flops(grid: Grid, d: int, B: int = 1, heads: int = 1) -> float:
+    """FLOPs of dense attention on the same shape: 4*Nq*Nk*d per head."""
+    return 4.0 * B * heads * grid.Nq * grid.Nk * d
