@@ -1,0 +1,409 @@
+"""Benchmark of the Monarch video-attention forward on B200.
+
+One step = one full forward call (every refinement iteration, every kernel)
+over one batch of seeded synthetic input.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--impl ours|reference]
+
+--impl reference times the fp64 CPU oracle (the only reference that exists
+for this method here) on a bounded sample of the same workload.
+
+Multi-GPU: one process per GPU (torchrun); (batch, head) units are
+independent, so every rank runs its own full copy of the workload with no
+collective on the data path (weak scaling); the timed region is bracketed by
+barriers and the max over ranks is reported.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from structured_sparse_attention_grid_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+
+METRIC = "Monarch-attn ms/call & effective TFLOP/s, bf16, N=4680–32760; % roofline"
+DEFAULT_WORKLOAD = "chunk_4680_bf16"
+L2_BYTES = 126 * 2**20
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        j = json.load(open(p))
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------------------
+# Algorithmic work of one call (no recompute counted).
+def geometry(w):
+    P = (w.H // w.th) * (w.W // w.tw)
+    return dict(P=P, b2=w.th * w.tw, b1q=w.T * P, b1k=w.Tkey * P)
+
+
+def work_model(w):
+    g = geometry(w)
+    BH = w.B * w.heads
+    FL = 2.0 * g["b2"] * g["b1q"] * g["b1k"] * w.d  # one L-sized contraction, per head
+    FR = 2.0 * g["b1k"] * g["b2"] ** 2 * w.d        # one R-sized contraction, per head
+    es = 4 if w.dtype == "f32" else 2
+    nq, nk = w.Nq * w.d * es * BH, w.Nk * w.d * es * BH  # bytes of q (= out) and of k (= v)
+    flops_total = BH * (2 * w.iters * FL + (2 * w.iters + 1) * FR)
+    # per-phase algorithmic FLOPs and compulsory bytes of ONE launch
+    lse = BH * g["b2"] * g["b1q"] * 4
+    hb = BH * g["b2"] * g["b1k"] * 4
+    phases = {
+        "l_out": dict(flops=BH * 2 * FL, bytes=nq + 2 * nk + hb + nq),   # q, k~, z, h -> out
+        "l_row": dict(flops=BH * FL, bytes=nq + nk + hb + lse),          # q, k~, h -> lse
+        "l_col": dict(flops=BH * FL, bytes=nq + nk + hb + lse + nk),     # q, k~, h, lse -> q~
+        "r_step": dict(flops=BH * 2 * FR, bytes=3 * nk),                 # q~, k -> k~ (final: +v, z)
+        "qbar": dict(flops=0.0, bytes=nq),
+    }
+    return dict(flops=flops_total, io_bytes=2 * nq + 2 * nk, dense_flops=4.0 * BH * w.Nq * w.Nk * w.d,
+                phases=phases, FL=FL, FR=FR)
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons in the background."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.mark = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def begin(self):
+        self.mark = time.time()
+
+    def end(self):
+        self.stop_t = time.time()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = [r for t, r in self.rows if self.mark and self.mark - 0.15 <= t <= self.stop_t + 0.15]
+        if not rows:
+            rows = [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, device):
+    import structured_sparse_attention_grid_b200 as m
+    w = WORKLOADS[args.workload]
+    model = work_model(w)
+    peaks = load_peaks()
+    q, k, v = make_inputs(w)
+    qd, kd, vd = (t.to(device) for t in (q, k, v))
+    out = torch.empty_like(qd)
+    stream = torch.cuda.current_stream(device)
+    io_bytes = model["io_bytes"]
+    flush = torch.empty(int(2 * L2_BYTES), dtype=torch.uint8, device=device)
+    flush_l2 = io_bytes < 4 * L2_BYTES  # inputs smaller than ~4x L2: flush between steps
+
+    def step():
+        m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters, stream=stream)
+
+    for _ in range(args.warmup):
+        if flush_l2:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+
+    clocks = ClockSampler(torch.cuda.current_device() if device.index is None else device.index)
+    clocks.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    launches0 = m.launch_count()
+    clocks.begin()
+    for i in range(args.steps):
+        if flush_l2:
+            flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    clocks.end()
+    launches = m.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = sum(per_step) / len(per_step)
+    # If the timed steps were short, keep sampling clocks for a moment under load.
+    if sum(per_step) < 1000.0:
+        t_end = time.time() + 1.0
+        while time.time() < t_end:
+            step()
+        torch.cuda.synchronize(device)
+        clocks.end()
+    clocks.stop()
+
+    if world > 1:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # Per-kernel times: the same step, with CUDA events around every launch.
+    m.profile_enable(True)
+    m.profile_read(reset=True)
+    nprof = max(3, min(args.steps, 20))
+    for _ in range(nprof):
+        if flush_l2:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize(device)
+    prof = m.profile_read(reset=True)
+    m.profile_enable(False)
+    dom = max((p for p in prof if prof[p][1] > 0), key=lambda p: prof[p][0])
+    dom_ms = prof[dom][0] / prof[dom][1]
+    ph = model["phases"][dom]
+    t_flop = ph["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = ph["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    if t_flop >= t_hbm and w.dtype != "f32":
+        roof = {"bound": "tensor", "achieved": ph["flops"] / (dom_ms * 1e-3) / 1e12,
+                "peak": peaks["bf16_tflops"], "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": ph["bytes"] / (dom_ms * 1e-3) / 1e9,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = dom
+    roof["launch_ms"] = dom_ms
+    roof["peak_source"] = peaks["source"]
+
+    call_roof_ms = 1e3 * max(model["flops"] / (peaks["bf16_tflops"] * 1e12), io_bytes / (peaks["hbm_gbs"] * 1e9))
+
+    # End to end through the host-buffer entry point (copies inside the timed region).
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(q).pin_memory()
+    for _ in range(2):
+        m.monarch_attn_fwd_host(qh, kh, vh, oh, w.T, w.H, w.W, w.th, w.tw, w.iters, stream=stream)
+    e2e_n = max(3, min(args.steps, 10))
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(device)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_n):
+        m.monarch_attn_fwd_host(qh, kh, vh, oh, w.T, w.H, w.W, w.th, w.tw, w.iters, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1) / e2e_n
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    es = q.element_size()
+    rec = {
+        "metric": METRIC,
+        "value": world * model["flops"] / (ms * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded; positional + planted-pair structure, see workloads.py)",
+        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.T, w.H, w.W],
+                   "kv_frames": w.Tkey, "head_dim": w.d, "tile": [w.th, w.tw], "iters": w.iters,
+                   "Nq": w.Nq, "Nk": w.Nk, "parallelism": f"replicas{world}",
+                   "l2": "flushed between steps" if flush_l2 else "inputs larger than L2"},
+        "monarch_gflop_per_call": model["flops"] / 1e9,
+        "dense_gflop_per_call": model["dense_flops"] / 1e9,
+        "call_roofline": {"roofline_ms": call_roof_ms, "frac": call_roof_ms / ms,
+                          "bound": "tensor" if model["flops"] / (peaks["bf16_tflops"] * 1e12)
+                          >= io_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"},
+        "roofline": roof,
+        "kernels": {p: {"ms_per_launch": prof[p][0] / prof[p][1], "launches_per_step": prof[p][1] / nprof}
+                    for p in prof if prof[p][1] > 0},
+        "e2e": {"value": world * model["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_call": e2e_ms,
+                "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
+                "d2h_bytes_per_step": q.numel() * es},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    return rec, (q, k, v, w)
+
+
+def cpu_baseline(w, q, k, v, budget_s: float):
+    """Times the fp64 oracle on the host on whole (batch, head) units until
+    about budget_s seconds of CPU work; returns the record and the throughput
+    in the metric's unit."""
+    from oracle import monarch as om
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        blas = 1
+    g = om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None)
+    model = work_model(w)
+    per_head = model["flops"] / (w.B * w.heads)
+    done, t0 = 0, time.perf_counter()
+    units = [(b, h) for b in range(w.B) for h in range(w.heads)]
+    while True:
+        b, h = units[done % len(units)]
+        qn, kn, vn = (t[b:b + 1, h:h + 1].double().numpy() for t in (q, k, v))
+        om.monarch_attention(qn, kn, vn, g, w.iters)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or done >= len(units):
+            break
+    value = done * per_head / el / 1e12
+    return {"value": value, "unit": "TFLOP/s", "cores": blas, "host_cpus": os.cpu_count(),
+            "kind": "oracle", "sample": f"{done} of {len(units)} (batch, head) units of {w.name}, "
+                                        f"{el:.1f} s fp64 numpy"}, el / done
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores: a bounded sample of the
+    workload per step (whole (batch, head) units)."""
+    w = WORKLOADS[args.workload]
+    q, k, v = make_inputs(w)
+    from oracle import monarch as om
+    g = om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None)
+    model = work_model(w)
+    per_head = model["flops"] / (w.B * w.heads)
+    units = [(b, h) for b in range(w.B) for h in range(w.heads)]
+    # size the per-step sample so warm-up + steps stay within ~2 minutes
+    t0 = time.perf_counter()
+    qn, kn, vn = (t[0:1, 0:1].double().numpy() for t in (q, k, v))
+    om.monarch_attention(qn, kn, vn, g, w.iters)
+    t_unit = time.perf_counter() - t0
+    per_step = max(1, min(len(units), int(120.0 / max(1e-3, t_unit) / max(1, args.steps + args.warmup))))
+    times = []
+    for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
+        for j in range(per_step):
+            b, h = units[(s * per_step + j) % len(units)]
+            qn, kn, vn = (t[b:b + 1, h:h + 1].double().numpy() for t in (q, k, v))
+            om.monarch_attention(qn, kn, vn, g, w.iters)
+        if s >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    sec = sum(times) / len(times)
+    value = per_step * per_head / sec / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        blas = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:  # noqa: BLE001
+        blas = 1
+    sample = f"{per_step} of {len(units)} (batch, head) units of {w.name} per step, fp64 numpy"
+    return {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": sec * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "heads": w.heads, "grid": [w.T, w.H, w.W],
+                   "kv_frames": w.Tkey, "head_dim": w.d, "tile": [w.th, w.tw], "iters": w.iters,
+                   "parallelism": "host"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "kind": "oracle", "cores": blas, "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, rank, world)), flush=True)
+        return
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    rec, (q, k, v, w) = run_ours(args, rank, world, device)
+    if rank == 0:
+        if world == 1:
+            cb, _ = cpu_baseline(w, q, k, v, args.cpu_budget)
+            rec["cpu_baseline"] = cb
+        print(json.dumps(rec), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

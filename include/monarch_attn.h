@@ -1,0 +1,144 @@
+/*
+ * monarch_attn.h -- C ABI of the B200 (sm_100a) Monarch video-attention forward.
+ *
+ * Operation (MonarchRT: Efficient Attention for Real-Time Video Generation;
+ * gist.science explainer §2 "Methodology", §2.A "Block Alignment", §2.B "Tiled
+ * Monarch Parameterization", §2.C "Finetuning and Efficient Implementation"):
+ * per (batch, head) the attention matrix over a T x H x W token grid is
+ * constrained to Monarch form M = P blockdiag(L) P^T blockdiag(R), with
+ *   tile     c1 = (t*(H/tile_h) + y/tile_h)*(W/tile_w) + x/tile_w
+ *   position c2 = (y % tile_h)*tile_w + x % tile_w,
+ *   M[(a1,a2),(c1,c2)] = L_{a2}[a1,c1] * R_{c1}[a2,c2],
+ * where L and R come from `iters` rounds of alternating refinement (each an
+ * R step then an L step):
+ *   R step: q~[c1,a2] = sum_a1 L q / sum_a1 L;  R_{c1}[a2,:] = softmax_c2(s q~.k)
+ *           h[c1,a2] = entropy of R_{c1}[a2,:]
+ *   L step: k~[c1,a2] = sum_c2 R k;  L_{a2}[a1,:] = softmax_c1(s q.k~ + h)
+ *   output: z = sum_c2 R v;  y[a1,a2] = sum_c1 L z;  out = y in grid order,
+ * s = 1/sqrt(d).  The first R step starts from L = block identity; with a KV
+ * cache (kv_len > T*H*W) the query tiles align with the last T key frames and
+ * cached key tiles start from the mean query of their position.  The query
+ * chunk is the newest chunk, so chunk-causal attention masks no key.  M is
+ * never materialised.
+ *
+ * Layouts: q and out are contiguous [B, heads, T*H*W, d]; k and v are
+ * contiguous [B, heads, kv_len, d]; tokens in grid order n = (t*H + y)*W + x.
+ * kv_len == T*H*W is self-attention; kv_len = Tk*H*W with Tk > T is a KV-cache
+ * step whose queries are the last T of the Tk key frames.
+ *
+ * dtype: MONARCH_F32, MONARCH_BF16 or MONARCH_F16 for all four tensors.
+ * Arithmetic: fp32 accumulation; bf16/f16 tensor-core operands for the bf16
+ * and f16 types; fp32 CUDA-core arithmetic for f32.
+ *
+ * Ownership: the caller owns q, k, v, out (device memory, 16-byte aligned).
+ * The library never keeps a pointer past the call's stream work.
+ * monarch_attn_fwd allocates its workspace stream-ordered on `stream`
+ * (cudaMallocAsync / cudaFreeAsync); monarch_attn_fwd_ws uses a caller buffer
+ * of at least monarch_attn_workspace_bytes(...) bytes instead.
+ *
+ * Behaviour: asynchronous on `stream` (no host synchronisation, except in
+ * monarch_attn_fwd_host); returns MONARCH_OK or a negative status, with a
+ * message in monarch_attn_last_error() (thread-local).  Arguments are
+ * validated on the host before any launch; kernels never trap.
+ */
+#ifndef MONARCH_ATTN_H
+#define MONARCH_ATTN_H
+
+#include <stddef.h>
+#include <cuda_runtime.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum {
+  MONARCH_OK = 0,
+  MONARCH_EINVAL = -1,      /* bad shape, null or misaligned pointer, bad dtype */
+  MONARCH_ENOMEM = -2,      /* workspace allocation failed or buffer too small */
+  MONARCH_ECUDA = -3,       /* a CUDA runtime call or launch failed */
+  MONARCH_EUNSUPPORTED = -4 /* valid but outside the built kernels' limits */
+};
+
+enum { MONARCH_F32 = 0, MONARCH_BF16 = 1, MONARCH_F16 = 2 };
+
+/* Forward.  q, k, v, out: device pointers (layouts above).  B, heads >= 1;
+ * T, H, W >= 1; d in {64, 128}; tile_h | H, tile_w | W, tile_h*tile_w <= 64;
+ * iters >= 1; kv_len a multiple of H*W and >= T*H*W.  stream may be 0. */
+int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                     int B, int heads, int T, int H, int W, int d,
+                     int tile_h, int tile_w, int iters, long kv_len,
+                     int dtype, cudaStream_t stream);
+
+/* Bytes of workspace the forward needs for these arguments (0 on invalid
+ * arguments, with the reason in monarch_attn_last_error()). */
+size_t monarch_attn_workspace_bytes(int B, int heads, int T, int H, int W, int d,
+                                    int tile_h, int tile_w, int iters, long kv_len,
+                                    int dtype);
+
+/* Same as monarch_attn_fwd with a caller-owned device workspace of
+ * workspace_bytes >= monarch_attn_workspace_bytes(...); nothing is allocated.
+ * The workspace must not be used by other work while the call's stream work
+ * runs. */
+int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
+                        int B, int heads, int T, int H, int W, int d,
+                        int tile_h, int tile_w, int iters, long kv_len,
+                        int dtype, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream);
+
+/* End-to-end variant on HOST buffers: copies q, k, v host->device, runs the
+ * forward and copies out device->host, all on `stream`, then synchronises
+ * `stream` before returning (so `out` is ready).  Device buffers are
+ * allocated stream-ordered and freed before return.  Pinned host memory gives
+ * asynchronous copies; pageable memory works but is slower. */
+int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                          void* out_host, int B, int heads, int T, int H, int W, int d,
+                          int tile_h, int tile_w, int iters, long kv_len,
+                          int dtype, cudaStream_t stream);
+
+/* Byte offsets, inside a workspace, of the intermediates left by the last
+ * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (dtype),
+ * [1] z (dtype, same shape), [2] q~ of the last R step with iters >= 2
+ * (dtype, same shape), [3] h [B*heads][b2][b1k] (f32), [4] row log2-sum-exp of
+ * the last non-final L step [B*heads][b2][b1q] (f32, base-2 logits s*log2(e)*
+ * q.k~ + log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32).  Returns
+ * the total bytes, 0 on invalid arguments. */
+size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int d,
+                                     int tile_h, int tile_w, int iters, long kv_len,
+                                     int dtype, size_t offsets[6]);
+
+/* Instrumentation.  Kernel phases of one forward: */
+enum {
+  MONARCH_PHASE_QBAR = 0,   /* mean query per position (KV-cache init)        */
+  MONARCH_PHASE_R_STEP = 1, /* R step: per-tile softmax, entropy, k~ (and z)  */
+  MONARCH_PHASE_L_ROW = 2,  /* L step row pass of a non-final iteration (LSE) */
+  MONARCH_PHASE_L_OUT = 3,  /* final L step fused with y = L z and the store  */
+  MONARCH_PHASE_L_COL = 4,  /* column pass q~ = L^T q / L^T 1                 */
+  MONARCH_NUM_PHASES = 5
+};
+
+/* Number of kernels this process has launched through the library (host
+ * counter, always on). */
+unsigned long long monarch_attn_launch_count(void);
+
+/* on != 0: record a CUDA event pair on the launching stream around every
+ * kernel launch from now on (adds a few microseconds per launch); 0: stop.
+ * Returns MONARCH_OK. */
+int monarch_attn_profile_enable(int on);
+
+/* Waits for the recorded events and adds, per phase p < n, the total kernel
+ * milliseconds to ms[p] and the launch count to launches[p] (either pointer
+ * may be null), accumulated since the last reset; reset != 0 clears the
+ * totals afterwards.  Returns MONARCH_OK or MONARCH_ECUDA. */
+int monarch_attn_profile_read(double* ms, unsigned long long* launches, int n, int reset);
+
+/* Thread-local message of the last failing call ("" if none). */
+const char* monarch_attn_last_error(void);
+
+/* ABI version (major*100 + minor). */
+int monarch_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MONARCH_ATTN_H */

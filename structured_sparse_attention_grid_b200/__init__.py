@@ -1,0 +1,160 @@
+"""Python binding of the B200 Monarch video-attention library (C ABI).
+
+Argument marshalling only: every step of the forward runs in the CUDA
+kernels of ``libmonarch_attn.so``.  PyTorch provides device memory and
+streams.  There is no fallback: if the library is missing, calls fail.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmonarch_attn.so")
+
+MONARCH_F32, MONARCH_BF16, MONARCH_F16 = 0, 1, 2
+PHASES = ("qbar", "r_step", "l_row", "l_out", "l_col")
+
+# Every symbol the header declares, with its ctypes signature.
+_SIGS = {
+    "monarch_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                         + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p]),
+    "monarch_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_int]),
+    "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                            + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
+                               ctypes.c_void_p]),
+    "monarch_attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                              + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p]),
+    "monarch_attn_workspace_layout": (ctypes.c_size_t, [ctypes.c_int] * 9
+                                      + [ctypes.c_long, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]),
+    "monarch_attn_launch_count": (ctypes.c_ulonglong, []),
+    "monarch_attn_profile_enable": (ctypes.c_int, [ctypes.c_int]),
+    "monarch_attn_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
+                                                 ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int,
+                                                 ctypes.c_int]),
+    "monarch_attn_last_error": (ctypes.c_char_p, []),
+    "monarch_attn_version": (ctypes.c_int, []),
+}
+
+_lib = None
+
+
+class MonarchError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"monarch_attn error {code}: {msg}")
+        self.code = code
+
+
+def load_library(path: str = LIB_PATH):
+    """Loads the C-ABI library (once) and declares its signatures."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with "
+                           "`python -m structured_sparse_attention_grid_b200.build`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _dtype_code(t) -> int:
+    import torch
+    codes = {torch.float32: MONARCH_F32, torch.bfloat16: MONARCH_BF16, torch.float16: MONARCH_F16}
+    if t.dtype not in codes:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return codes[t.dtype]
+
+
+def _stream_ptr(stream) -> int:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream)
+
+
+def _check(rc: int):
+    if rc != 0:
+        raise MonarchError(rc, _lib.monarch_attn_last_error().decode())
+
+
+def _shape_args(q, k, T, H, W, tile_h, tile_w, iters):
+    B, heads, nq, d = q.shape
+    if nq != T * H * W:
+        raise ValueError(f"q has {nq} tokens, grid {T}x{H}x{W} has {T * H * W}")
+    return [B, heads, T, H, W, d, tile_h, tile_w, iters, int(k.shape[2])]
+
+
+def _check_tensors(*ts):
+    for t in ts:
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous [B, heads, N, d]")
+
+
+def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
+    """out <- Monarch attention of (q, k, v); CUDA tensors, contiguous
+    [B, heads, N, d]; kv length = k.shape[2].  Asynchronous on ``stream``."""
+    lib = load_library()
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
+    _check(lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                *args, _dtype_code(q), _stream_ptr(stream)))
+    return out
+
+
+def workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype_code):
+    lib = load_library()
+    offs = (ctypes.c_size_t * 6)()
+    total = lib.monarch_attn_workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters,
+                                              kv_len, dtype_code, offs)
+    if total == 0:
+        raise MonarchError(-1, lib.monarch_attn_last_error().decode())
+    return int(total), [int(o) for o in offs]
+
+
+def monarch_attn_fwd_ws(q, k, v, out, workspace, T, H, W, tile_h, tile_w, iters, stream=None):
+    """As monarch_attn_fwd with a caller-owned device workspace (uint8 tensor)."""
+    lib = load_library()
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
+    _check(lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                   *args, _dtype_code(q), workspace.data_ptr(),
+                                   workspace.numel() * workspace.element_size(),
+                                   _stream_ptr(stream)))
+    return out
+
+
+def monarch_attn_fwd_host(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
+    """End-to-end call on HOST tensors (pinned for asynchronous copies): the
+    library copies in, computes, copies out and synchronises the stream."""
+    lib = load_library()
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
+    _check(lib.monarch_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     *args, _dtype_code(q), _stream_ptr(stream)))
+    return out
+
+
+def launch_count() -> int:
+    """Kernels launched so far by this process through the library."""
+    return int(load_library().monarch_attn_launch_count())
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library kernel with CUDA events on its stream."""
+    load_library().monarch_attn_profile_enable(1 if on else 0)
+
+
+def profile_read(reset: bool = True) -> dict:
+    """{phase: (total_ms, launches)} accumulated since the last reset."""
+    lib = load_library()
+    n = len(PHASES)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_ulonglong * n)()
+    _check(lib.monarch_attn_profile_read(ms, cnt, n, 1 if reset else 0))
+    return {p: (float(ms[i]), int(cnt[i])) for i, p in enumerate(PHASES)}

@@ -1,0 +1,342 @@
+// Host side of the Monarch video-attention forward: argument validation,
+// geometry, workspace layout and the launch sequence of one call.  Every
+// step of the computation runs in this library's kernels.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <cmath>
+#include <mutex>
+#include <atomic>
+#include <string>
+#include <vector>
+
+#include "monarch_attn.h"
+#include "common.cuh"
+#include "kernels_simt.cuh"
+
+using namespace monarch;
+
+namespace {
+
+thread_local std::string g_err;
+
+int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(MONARCH_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+// ---- instrumentation: launch counter and optional per-phase event timing ----
+std::atomic<unsigned long long> g_launches{0};
+
+struct Profiler {
+  std::mutex mu;
+  bool on = false;
+  struct Rec { int phase; cudaEvent_t a, b; };
+  std::vector<Rec> pending;
+  std::vector<cudaEvent_t> pool;
+  double ms[MONARCH_NUM_PHASES] = {};
+  unsigned long long n[MONARCH_NUM_PHASES] = {};
+  cudaEvent_t get() {
+    if (!pool.empty()) {
+      cudaEvent_t e = pool.back();
+      pool.pop_back();
+      return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+  }
+};
+Profiler g_prof;
+
+// Launches one kernel through `f`, counting it and, when profiling is on,
+// bracketing it with events on its stream.
+template <typename F>
+void launch(int phase, cudaStream_t st, F&& f) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (!g_prof.on) {
+    f();
+    return;
+  }
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  cudaEvent_t a = g_prof.get(), b = g_prof.get();
+  cudaEventRecord(a, st);
+  f();
+  cudaEventRecord(b, st);
+  g_prof.pending.push_back({phase, a, b});
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t elem_size(int dtype) { return dtype == MONARCH_F32 ? 4 : 2; }
+
+struct Plan {
+  Geo g;
+  int dtype;
+  int iters;
+  bool kv;
+  size_t off[6];
+  size_t total;
+};
+
+constexpr int kMaxB2 = 64;
+
+int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int iters,
+              long kv_len, int dtype, Plan* p) {
+  if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1)
+    return fail(MONARCH_EINVAL, "B, heads, T, H, W must be >= 1 (got %d %d %d %d %d)", B, heads, T, H, W);
+  if (d != 64 && d != 128) return fail(MONARCH_EINVAL, "head_dim d must be 64 or 128 (got %d)", d);
+  if (th < 1 || tw < 1 || H % th || W % tw)
+    return fail(MONARCH_EINVAL, "tile %dx%d must divide the %dx%d frame", th, tw, H, W);
+  if (iters < 1) return fail(MONARCH_EINVAL, "iters must be >= 1 (got %d)", iters);
+  if (dtype != MONARCH_F32 && dtype != MONARCH_BF16 && dtype != MONARCH_F16)
+    return fail(MONARCH_EINVAL, "unknown dtype %d", dtype);
+  const long long hw = (long long)H * W;
+  const long long nq = (long long)T * hw;
+  if (kv_len < nq || kv_len % hw)
+    return fail(MONARCH_EINVAL, "kv_len %ld must be a multiple of H*W=%lld and >= T*H*W=%lld", kv_len, hw, nq);
+  if (th * tw > kMaxB2)
+    return fail(MONARCH_EUNSUPPORTED, "tile_h*tile_w = %d exceeds the supported %d positions per tile", th * tw, kMaxB2);
+  const long long Tk = kv_len / hw;
+  const long long BH = (long long)B * heads;
+  if (BH * (long long)kv_len * d >= (1LL << 40) || Tk * (H / th) * (W / tw) >= (1LL << 30))
+    return fail(MONARCH_EUNSUPPORTED, "problem too large");
+  Geo& g = p->g;
+  g.BH = (int)BH;
+  g.T = T;
+  g.Tk = (int)Tk;
+  g.H = H;
+  g.W = W;
+  g.d = d;
+  g.th = th;
+  g.tw = tw;
+  g.ntx = W / tw;
+  g.P = (H / th) * (W / tw);
+  g.b2 = th * tw;
+  g.b1q = T * g.P;
+  g.b1k = g.Tk * g.P;
+  g.off = (g.Tk - T) * g.P;
+  g.Nq = nq;
+  g.Nk = kv_len;
+  g.sl2 = (float)(1.0 / std::sqrt((double)d) * 1.4426950408889634);
+  p->dtype = dtype;
+  p->iters = iters;
+  p->kv = g.Tk != T;
+  const size_t es = elem_size(dtype);
+  const size_t big = (size_t)BH * g.b2 * g.b1k * d * es;
+  size_t sizes[6] = {big, big, big, (size_t)BH * g.b2 * g.b1k * 4, (size_t)BH * g.b2 * g.b1q * 4,
+                     (size_t)BH * g.b2 * d * 4};
+  size_t o = 0;
+  for (int i = 0; i < 6; ++i) {
+    p->off[i] = o;
+    o += align256(sizes[i]);
+  }
+  p->total = o;
+  return MONARCH_OK;
+}
+
+int check_ptr(const void* ptr, const char* name) {
+  if (!ptr) return fail(MONARCH_EINVAL, "%s is null", name);
+  if (reinterpret_cast<uintptr_t>(ptr) & 15) return fail(MONARCH_EINVAL, "%s is not 16-byte aligned", name);
+  return MONARCH_OK;
+}
+
+template <typename T>
+int run(const Plan& p, const T* q, const T* k, const T* v, T* out, char* ws, cudaStream_t st) {
+  const Geo& g = p.g;
+  Work<T> w;
+  w.kt = reinterpret_cast<T*>(ws + p.off[0]);
+  w.z = reinterpret_cast<T*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<T*>(ws + p.off[2]);
+  w.h = reinterpret_cast<float*>(ws + p.off[3]);
+  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
+  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+
+  const size_t r_smem = (size_t)(3 * g.b2 * g.d + g.b2 * (g.b2 + 1)) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(r_step_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r_smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(r_step)");
+  constexpr int kRows = 16;
+  for (int it = 0; it < p.iters; ++it) {
+    const int final_step = it == p.iters - 1;
+    int mode = QT_BUFFER;
+    if (it == 0) {
+      mode = p.kv ? QT_KVINIT : QT_IDENTITY;
+      if (p.kv)
+        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<T><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
+    } else {
+      dim3 grid((g.b1k + kRows - 1) / kRows, g.b2, g.BH);
+      launch(MONARCH_PHASE_L_COL, st, [&] {
+        if (g.d == 128) l_col_simt<T, 128><<<grid, 32 * kRows, 0, st>>>(q, w, g);
+        else l_col_simt<T, 64><<<grid, 32 * kRows, 0, st>>>(q, w, g);
+      });
+    }
+    launch(MONARCH_PHASE_R_STEP, st, [&] {
+      r_step_simt<T><<<dim3(g.b1k, g.BH), 128, r_smem, st>>>(q, k, v, w, g, mode, final_step);
+    });
+    dim3 grid((g.b1q + kRows - 1) / kRows, g.b2, g.BH);
+    launch(final_step ? MONARCH_PHASE_L_OUT : MONARCH_PHASE_L_ROW, st, [&] {
+      if (g.d == 128) l_row_simt<T, 128><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
+      else l_row_simt<T, 64><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
+    });
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return MONARCH_OK;
+}
+
+int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* out, void* ws,
+             cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  switch (p.dtype) {
+    case MONARCH_F32:
+      return run<float>(p, (const float*)q, (const float*)k, (const float*)v, (float*)out, w, st);
+    case MONARCH_BF16:
+      return run<__nv_bfloat16>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                (const __nv_bfloat16*)v, (__nv_bfloat16*)out, w, st);
+    default:
+      return run<__half>(p, (const __half*)q, (const __half*)k, (const __half*)v, (__half*)out, w, st);
+  }
+}
+
+int check_io(const void* q, const void* k, const void* v, const void* out) {
+  int rc;
+  if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v")) ||
+      (rc = check_ptr(out, "out")))
+    return rc;
+  return MONARCH_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int monarch_attn_version(void) { return 100; }
+
+unsigned long long monarch_attn_launch_count(void) { return g_launches.load(); }
+
+int monarch_attn_profile_enable(int on) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  g_prof.on = on != 0;
+  return MONARCH_OK;
+}
+
+int monarch_attn_profile_read(double* ms, unsigned long long* launches, int n, int reset) {
+  std::lock_guard<std::mutex> lk(g_prof.mu);
+  int rc = MONARCH_OK;
+  for (auto& r : g_prof.pending) {
+    float t = 0.f;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&t, r.a, r.b);
+    if (e != cudaSuccess && rc == MONARCH_OK) rc = cuda_fail(e, "profile events");
+    g_prof.ms[r.phase] += t;
+    g_prof.n[r.phase] += 1;
+    g_prof.pool.push_back(r.a);
+    g_prof.pool.push_back(r.b);
+  }
+  g_prof.pending.clear();
+  for (int p = 0; p < n && p < MONARCH_NUM_PHASES; ++p) {
+    if (ms) ms[p] = g_prof.ms[p];
+    if (launches) launches[p] = g_prof.n[p];
+  }
+  if (reset)
+    for (int p = 0; p < MONARCH_NUM_PHASES; ++p) g_prof.ms[p] = 0, g_prof.n[p] = 0;
+  return rc;
+}
+
+const char* monarch_attn_last_error(void) { return g_err.c_str(); }
+
+size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int d, int tile_h,
+                                     int tile_w, int iters, long kv_len, int dtype,
+                                     size_t offsets[6]) {
+  Plan p;
+  if (make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p) != MONARCH_OK) return 0;
+  if (offsets)
+    for (int i = 0; i < 6; ++i) offsets[i] = p.off[i];
+  return p.total;
+}
+
+size_t monarch_attn_workspace_bytes(int B, int heads, int T, int H, int W, int d, int tile_h,
+                                    int tile_w, int iters, long kv_len, int dtype) {
+  return monarch_attn_workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype,
+                                       nullptr);
+}
+
+int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out, int B, int heads,
+                        int T, int H, int W, int d, int tile_h, int tile_w, int iters, long kv_len,
+                        int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  if (rc) return rc;
+  if ((rc = check_io(q, k, v, out))) return rc;
+  if ((rc = check_ptr(workspace, "workspace"))) return rc;
+  if (workspace_bytes < p.total)
+    return fail(MONARCH_ENOMEM, "workspace of %zu bytes is smaller than the %zu needed", workspace_bytes, p.total);
+  return dispatch(p, q, k, v, out, workspace, stream);
+}
+
+int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int heads,
+                     int T, int H, int W, int d, int tile_h, int tile_w, int iters, long kv_len,
+                     int dtype, cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  if (rc) return rc;
+  if ((rc = check_io(q, k, v, out))) return rc;
+  void* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocAsync(%zu): %s", p.total, cudaGetErrorString(e));
+  }
+  rc = dispatch(p, q, k, v, out, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                          void* out_host, int B, int heads, int T, int H, int W, int d,
+                          int tile_h, int tile_w, int iters, long kv_len, int dtype,
+                          cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  if (rc) return rc;
+  if (!q_host || !k_host || !v_host || !out_host) return fail(MONARCH_EINVAL, "null host pointer");
+  const size_t es = elem_size(dtype);
+  const size_t qb = (size_t)p.g.BH * p.g.Nq * d * es;
+  const size_t kb = (size_t)p.g.BH * p.g.Nk * d * es;
+  const size_t oq = 0, ok = align256(qb), ov = ok + align256(kb), oo = ov + align256(kb);
+  const size_t ow = oo + align256(qb);
+  char* buf = nullptr;
+  cudaError_t e = cudaMallocAsync((void**)&buf, ow + p.total, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocAsync(%zu): %s", ow + p.total, cudaGetErrorString(e));
+  }
+  if ((e = cudaMemcpyAsync(buf + oq, q_host, qb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(buf + ok, k_host, kb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
+      (e = cudaMemcpyAsync(buf + ov, v_host, kb, cudaMemcpyHostToDevice, stream)) != cudaSuccess) {
+    rc = cuda_fail(e, "cudaMemcpyAsync(host->device)");
+  }
+  if (rc == MONARCH_OK) rc = dispatch(p, buf + oq, buf + ok, buf + ov, buf + oo, buf + ow, stream);
+  if (rc == MONARCH_OK && (e = cudaMemcpyAsync(out_host, buf + oo, qb, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+    rc = cuda_fail(e, "cudaMemcpyAsync(device->host)");
+  cudaFreeAsync(buf, stream);
+  e = cudaStreamSynchronize(stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) rc = cuda_fail(e, "cudaStreamSynchronize");
+  return rc;
+}
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+"""CPU checks of the C-ABI library: it loads without a GPU, exports every
+symbol the header declares, and validates arguments on the host (no compute
+call is made here)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import structured_sparse_attention_grid_b200 as m
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \t\*]*?\b(monarch_\w+)\s*\(", src, flags=re.M)
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from structured_sparse_attention_grid_b200 import build
+    build.build()
+    return m.load_library()
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    assert "monarch_attn_fwd" in names and "monarch_attn_last_error" in names
+    assert len(names) == len(set(names))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_declared_functions()) == set(m._SIGS)
+
+
+def test_version(lib):
+    assert lib.monarch_attn_version() >= 100
+
+
+CFG1 = dict(B=1, heads=12, T=3, H=30, W=52, d=128, th=6, tw=4, iters=2, kv=4680, dt=1)
+
+
+def _ws(c, **kw):
+    c = {**c, **kw}
+    return m.load_library().monarch_attn_workspace_bytes(c["B"], c["heads"], c["T"], c["H"], c["W"], c["d"],
+                                                         c["th"], c["tw"], c["iters"], c["kv"], c["dt"])
+
+
+def test_workspace_bytes_counts_the_intermediates(lib):
+    total, offs = m.workspace_layout(1, 12, 3, 30, 52, 128, 6, 4, 2, 4680, 1)
+    big = 12 * 24 * 195 * 128 * 2  # k~, z, q~ in bf16
+    assert offs[0] == 0 and offs[1] >= big and offs[2] - offs[1] >= big
+    assert total >= 3 * big + 12 * 24 * 195 * 4 * 2
+    assert total == _ws(CFG1)
+
+
+@pytest.mark.parametrize("bad,needle", [
+    (dict(H=31), "tile"),
+    (dict(tw=5), "tile"),
+    (dict(d=96), "head_dim"),
+    (dict(iters=0), "iters"),
+    (dict(kv=4681), "kv_len"),
+    (dict(kv=3000), "kv_len"),
+    (dict(dt=7), "dtype"),
+    (dict(B=0), ">= 1"),
+])
+def test_invalid_arguments_are_rejected_on_the_host(lib, bad, needle):
+    assert _ws(CFG1, **bad) == 0
+    assert needle in lib.monarch_attn_last_error().decode()
+
+
+def test_oversized_tile_is_unsupported(lib):
+    assert _ws(CFG1, th=30, tw=52) == 0
+    assert "exceeds" in lib.monarch_attn_last_error().decode()
+
+
+def test_null_pointer_is_rejected_before_any_launch(lib):
+    c = CFG1
+    rc = lib.monarch_attn_fwd(None, None, None, None, c["B"], c["heads"], c["T"], c["H"], c["W"], c["d"],
+                              c["th"], c["tw"], c["iters"], c["kv"], c["dt"], None)
+    assert rc == -1
+    assert "null" in lib.monarch_attn_last_error().decode()
+
+
+def test_misaligned_pointer_is_rejected(lib):
+    c = CFG1
+    rc = lib.monarch_attn_fwd(0x1008, 0x2000, 0x3000, 0x4000, c["B"], c["heads"], c["T"], c["H"], c["W"],
+                              c["d"], c["th"], c["tw"], c["iters"], c["kv"], c["dt"], None)
+    assert rc == -1
+    assert "aligned" in lib.monarch_attn_last_error().decode()
+
+
+def test_product_path_does_not_import_the_oracle():
+    pkg = os.path.join(ROOT, "structured_sparse_attention_grid_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), f
+                assert not any("oracle" in inc for inc in re.findall(r"#include.*", src)), f

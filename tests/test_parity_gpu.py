@@ -1,0 +1,206 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs.
+
+Tolerances: fp32 max|err| <= 1e-4; bf16/f16 max|err| <= 2e-2 * RMS(oracle
+output).  Full-size workloads compare every output of a sample of heads
+(heads are independent, so a head is an exact sample) plus all-head
+properties (finite output, every row a convex combination of v rows)."""
+
+import numpy as np
+import pytest
+import torch
+
+import structured_sparse_attention_grid_b200 as m
+from oracle import monarch as om
+from structured_sparse_attention_grid_b200.workloads import WORKLOADS, Workload, make_inputs
+
+pytestmark = pytest.mark.gpu
+
+TOL_F32 = 1e-4
+TOL_LOWP = 2e-2
+
+
+def _grid(w):
+    return om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None)
+
+
+def _run_gpu(w, q, k, v):
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    return out
+
+
+def _compare(w, out_gpu, q, k, v, heads=None):
+    qn, kn, vn = (t.double().numpy() for t in (q, k, v))
+    ref = om.monarch_attention(qn, kn, vn, _grid(w), w.iters, heads=heads)
+    got = out_gpu.double().cpu().numpy()
+    hs = heads or [(b, h) for b in range(w.B) for h in range(w.heads)]
+    err, rms = 0.0, 0.0
+    for b, h in hs:
+        err = max(err, float(np.abs(got[b, h] - ref[b, h]).max()))
+        rms = max(rms, float(np.sqrt((ref[b, h] ** 2).mean())))
+    if w.dtype == "f32":
+        assert err <= TOL_F32, f"{w.name}: max|err| {err:.3e} > {TOL_F32}"
+    else:
+        assert err <= TOL_LOWP * rms, f"{w.name}: max|err| {err:.3e} > {TOL_LOWP} * rms {rms:.3e}"
+    return err, rms
+
+
+def _all_head_properties(out, v):
+    o = out.float()
+    assert torch.isfinite(o).all()
+    vd = v.cuda().float()
+    lo = vd.amin(dim=2, keepdim=True)
+    hi = vd.amax(dim=2, keepdim=True)
+    slack = 1e-2 * (hi - lo) + 1e-3
+    assert (o >= lo - slack).all() and (o <= hi + slack).all()
+
+
+@pytest.mark.parametrize("name", ["toy_256_f32", "toy_256_f32_separable"])
+def test_toy_fp32(name, cuda_lib):
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _compare(w, out, q, k, v)
+
+
+def test_toy_separable_matches_dense_attention(cuda_lib):
+    w = WORKLOADS["toy_256_f32_separable"]
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v).double().cpu().numpy()
+    ref = om.dense_attention(q.double().numpy(), k.double().numpy(), v.double().numpy())
+    assert np.abs(out - ref).max() <= TOL_F32
+
+
+@pytest.mark.parametrize("name", ["chunk_4680_bf16", "kvcache_4680x32760_bf16", "sweep_2048_f16",
+                                  "sweep_8192_f16"])
+def test_workload_all_heads(name, cuda_lib):
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _all_head_properties(out, v)
+    _compare(w, out, q, k, v)
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("full_32760_bf16", [(0, 0), (1, 11)]),
+    ("sweep_32768_f16", [(0, 0), (0, 13), (0, 23)]),
+])
+def test_workload_sampled_heads(name, heads, cuda_lib):
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _all_head_properties(out, v)
+    _compare(w, out, q, k, v, heads=heads)
+
+
+def _custom(dtype, T, H, W, d, th, tw, iters, Tk=0, B=2, heads=3, kind="pos_planted", seed=7):
+    return Workload(f"custom_{dtype}_{T}x{H}x{W}_d{d}_{th}x{tw}_it{iters}_Tk{Tk}", B, heads, T, H, W, d,
+                    th, tw, iters, dtype, seed, kind, Tk=Tk, planted=8)
+
+
+EDGE = [
+    # ragged tiles (b1 = 75 not a multiple of any tile), every iteration count
+    _custom("bf16", 5, 12, 20, 128, 4, 4, 1),
+    _custom("bf16", 5, 12, 20, 128, 4, 4, 2),
+    _custom("f16", 5, 12, 20, 64, 4, 4, 3),
+    _custom("f32", 3, 8, 12, 128, 2, 4, 2),
+    # KV cache with b1q != b1k and a ragged tail
+    _custom("bf16", 2, 12, 20, 128, 4, 4, 2, Tk=7),
+    _custom("f16", 1, 8, 8, 64, 4, 2, 3, Tk=5),
+    _custom("f32", 2, 8, 8, 64, 4, 4, 2, Tk=3),
+    # degenerate: one position per tile (b2 = 1) and one tile per sequence (b1 = 1)
+    _custom("bf16", 2, 6, 8, 128, 1, 1, 2),
+    _custom("bf16", 1, 6, 8, 128, 6, 8, 2),
+    _custom("f32", 1, 6, 8, 64, 6, 8, 1),
+    # largest supported tile (64 positions) and b1 exactly one 128-row block
+    _custom("f16", 2, 32, 32, 64, 8, 8, 2),
+    _custom("bf16", 8, 16, 16, 128, 4, 2, 2, B=1, heads=2),
+]
+
+
+@pytest.mark.parametrize("w", EDGE, ids=[w.name for w in EDGE])
+def test_edge_cases(w, cuda_lib):
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _compare(w, out, q, k, v)
+
+
+def test_degenerate_grids_reduce_to_dense_attention(cuda_lib):
+    for w in (_custom("f32", 2, 6, 8, 64, 1, 1, 2, kind="iid"), _custom("f32", 1, 6, 8, 64, 6, 8, 2, kind="iid")):
+        q, k, v = make_inputs(w)
+        out = _run_gpu(w, q, k, v).double().cpu().numpy()
+        ref = om.dense_attention(q.double().numpy(), k.double().numpy(), v.double().numpy())
+        assert np.abs(out - ref).max() <= TOL_F32
+
+
+def test_intermediates_match_the_oracle_on_the_toy(cuda_lib):
+    w = _custom("f32", 4, 8, 8, 64, 4, 4, 2, B=1, heads=2, kind="iid")
+    q, k, v = make_inputs(w)
+    total, offs = m.workspace_layout(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw, w.iters, w.Nk, m.MONARCH_F32)
+    ws = torch.zeros(total, dtype=torch.uint8, device="cuda")
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    m.monarch_attn_fwd_ws(qd, kd, vd, out, ws, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    g = _grid(w)
+    _, states = om.monarch_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(), g,
+                                     w.iters, return_states=True)
+    b2, b1, d = g.b2, g.b1k, w.d
+
+    def view(i, n, dt=torch.float32):
+        return ws[offs[i]:offs[i] + n * 4].view(dt)
+
+    kt = view(0, 2 * b2 * b1 * d).view(2, b2, b1, d).cpu().double().numpy()
+    qt = view(2, 2 * b2 * b1 * d).view(2, b2, b1, d).cpu().double().numpy()
+    hh = view(3, 2 * b2 * b1).view(2, b2, b1).cpu().double().numpy()
+    for h in range(2):
+        st = states[(0, h)]
+        np.testing.assert_allclose(kt[h], np.swapaxes(st.kt, 0, 1), atol=1e-4)
+        np.testing.assert_allclose(qt[h], np.swapaxes(st.qt, 0, 1), atol=1e-4)
+        np.testing.assert_allclose(hh[h], st.h.T, atol=1e-4)
+
+
+def test_host_buffer_entry_point(cuda_lib):
+    w = WORKLOADS["toy_256_f32"]
+    q, k, v = make_inputs(w)
+    out = torch.empty_like(q).pin_memory()
+    m.monarch_attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), out, w.T, w.H, w.W, w.th,
+                            w.tw, w.iters)
+    _compare(w, out, q, k, v)
+
+
+def test_workspace_entry_point_matches_allocating_call(cuda_lib):
+    w = WORKLOADS["chunk_4680_bf16"]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    total, _ = m.workspace_layout(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw, w.iters, w.Nk, m.MONARCH_BF16)
+    ws = torch.empty(total, dtype=torch.uint8, device="cuda")
+    a, b = torch.empty_like(q), torch.empty_like(q)
+    m.monarch_attn_fwd(q, k, v, a, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    m.monarch_attn_fwd_ws(q, k, v, b, ws, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_repeated_calls_are_deterministic(cuda_lib):
+    w = WORKLOADS["sweep_2048_f16"]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    a, b = torch.empty_like(q), torch.empty_like(q)
+    m.monarch_attn_fwd(q, k, v, a, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    m.monarch_attn_fwd(q, k, v, b, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_invalid_call_returns_an_error_and_leaves_the_context_usable(cuda_lib):
+    w = WORKLOADS["toy_256_f32"]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    out = torch.empty_like(q)
+    with pytest.raises(m.MonarchError) as e:
+        m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, 3, w.tw, w.iters)  # 3 does not divide H
+    assert e.value.code == -1
+    m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
