@@ -26,9 +26,14 @@
  * kv_len == T*H*W is self-attention; kv_len = Tk*H*W with Tk > T is a KV-cache
  * step whose queries are the last T of the Tk key frames.
  *
- * dtype: MONARCH_F32, MONARCH_BF16 or MONARCH_F16 for all four tensors.
- * Arithmetic: fp32 accumulation; bf16/f16 tensor-core operands for the bf16
- * and f16 types; fp32 CUDA-core arithmetic for f32.
+ * dtype: MONARCH_F32, MONARCH_BF16 or MONARCH_F16 for q, k, v.  out_dtype:
+ * MONARCH_F32 or dtype.  With bf16/f16 inputs an f32 output keeps the result
+ * within 2e-2 of the output RMS of the exact (fp64) answer on peaked video
+ * attention, which rounding the output to bf16 alone can exceed.
+ * Arithmetic: fp32 accumulation and fp32 softmax statistics; tensor-core
+ * contractions take f16 operands, with computed operands split into an f16
+ * high part and an f16 low part (two products) where one rounding would cost
+ * accuracy; f32 inputs use fp32 CUDA-core arithmetic throughout.
  *
  * Ownership: the caller owns q, k, v, out (device memory, 16-byte aligned).
  * The library never keeps a pointer past the call's stream work.
@@ -67,7 +72,7 @@ enum { MONARCH_F32 = 0, MONARCH_BF16 = 1, MONARCH_F16 = 2 };
 int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out,
                      int B, int heads, int T, int H, int W, int d,
                      int tile_h, int tile_w, int iters, long kv_len,
-                     int dtype, cudaStream_t stream);
+                     int dtype, int out_dtype, cudaStream_t stream);
 
 /* Bytes of workspace the forward needs for these arguments (0 on invalid
  * arguments, with the reason in monarch_attn_last_error()). */
@@ -82,7 +87,7 @@ size_t monarch_attn_workspace_bytes(int B, int heads, int T, int H, int W, int d
 int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
                         int B, int heads, int T, int H, int W, int d,
                         int tile_h, int tile_w, int iters, long kv_len,
-                        int dtype, void* workspace, size_t workspace_bytes,
+                        int dtype, int out_dtype, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
 /* End-to-end variant on HOST buffers: copies q, k, v host->device, runs the
@@ -93,12 +98,13 @@ int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
 int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                           void* out_host, int B, int heads, int T, int H, int W, int d,
                           int tile_h, int tile_w, int iters, long kv_len,
-                          int dtype, cudaStream_t stream);
+                          int dtype, int out_dtype, cudaStream_t stream);
 
 /* Byte offsets, inside a workspace, of the intermediates left by the last
- * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (dtype),
- * [1] z (dtype, same shape), [2] q~ of the last R step with iters >= 2
- * (dtype, same shape), [3] h [B*heads][b2][b1k] (f32), [4] row log2-sum-exp of
+ * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (f32 for
+ * f32 inputs; otherwise an f16 high plane followed by an f16 low plane),
+ * [1] z (same form), [2] q~ of the last R step with iters >= 2 (f32, same
+ * shape), [3] h [B*heads][b2][b1k] (f32), [4] row log2-sum-exp of
  * the last non-final L step [B*heads][b2][b1q] (f32, base-2 logits s*log2(e)*
  * q.k~ + log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32).  Returns
  * the total bytes, 0 on invalid arguments. */

@@ -19,13 +19,13 @@ PHASES = ("qbar", "r_step", "l_row", "l_out", "l_col")
 # Every symbol the header declares, with its ctypes signature.
 _SIGS = {
     "monarch_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
-                         + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p]),
+                         + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_int]),
     "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
-                            + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p, ctypes.c_size_t,
-                               ctypes.c_void_p]),
+                            + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                               ctypes.c_size_t, ctypes.c_void_p]),
     "monarch_attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
-                              + [ctypes.c_long, ctypes.c_int, ctypes.c_void_p]),
+                              + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_workspace_layout": (ctypes.c_size_t, [ctypes.c_int] * 9
                                       + [ctypes.c_long, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]),
     "monarch_attn_launch_count": (ctypes.c_ulonglong, []),
@@ -98,12 +98,13 @@ def _check_tensors(*ts):
 
 def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
     """out <- Monarch attention of (q, k, v); CUDA tensors, contiguous
-    [B, heads, N, d]; kv length = k.shape[2].  Asynchronous on ``stream``."""
+    [B, heads, N, d]; kv length = k.shape[2]; out is float32 or q's dtype.
+    Asynchronous on ``stream``."""
     lib = load_library()
     _check_tensors(q, k, v, out)
     args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
     _check(lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                *args, _dtype_code(q), _stream_ptr(stream)))
+                                *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
 
 
@@ -123,7 +124,7 @@ def monarch_attn_fwd_ws(q, k, v, out, workspace, T, H, W, tile_h, tile_w, iters,
     _check_tensors(q, k, v, out)
     args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
     _check(lib.monarch_attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                   *args, _dtype_code(q), workspace.data_ptr(),
+                                   *args, _dtype_code(q), _dtype_code(out), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(),
                                    _stream_ptr(stream)))
     return out
@@ -136,7 +137,7 @@ def monarch_attn_fwd_host(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=N
     _check_tensors(q, k, v, out)
     args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
     _check(lib.monarch_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                     *args, _dtype_code(q), _stream_ptr(stream)))
+                                     *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
 
 

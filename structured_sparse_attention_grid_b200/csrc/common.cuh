@@ -68,15 +68,16 @@ enum QtMode : int {
   QT_BUFFER = 2,    // later steps: q~ produced by the column pass
 };
 
-// Workspace pointers of one call (device memory).
-template <typename T>
+// Workspace of one call (device memory).  The SIMT kernels keep k~, z and q~
+// in fp32; the tensor-core kernels store k~ and z as two fp16 planes (hi, lo)
+// in the same bytes.
 struct Work {
-  T* kt;       // [BH][b2][b1k][d]  k~[c1,a2]
-  T* z;        // [BH][b2][b1k][d]  z[c1,a2]
-  T* qt;       // [BH][b2][b1k][d]  q~[c1,a2]
-  float* h;    // [BH][b2][b1k]     entropy of R_{c1}[a2,:]
-  float* lse;  // [BH][b2][b1q]     base-2 log-sum-exp of L rows
-  float* qbar; // [BH][b2][d]       mean query per position (KV init)
+  float* kt;    // [BH][b2][b1k][d]  k~[c1,a2]
+  float* z;     // [BH][b2][b1k][d]  z[c1,a2]
+  float* qt;    // [BH][b2][b1k][d]  q~[c1,a2]
+  float* h;     // [BH][b2][b1k]     entropy of R_{c1}[a2,:]
+  float* lse;   // [BH][b2][b1q]     base-2 log-sum-exp of L rows
+  float* qbar;  // [BH][b2][d]       mean query per position (KV init)
 };
 
 }  // namespace monarch

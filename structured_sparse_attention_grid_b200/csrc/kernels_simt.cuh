@@ -30,7 +30,7 @@ __global__ void qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, G
 template <typename T>
 __global__ void __launch_bounds__(128)
 r_step_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-            Work<T> w, Geo g, int mode, int final_step) {
+            Work w, Geo g, int mode, int final_step) {
   extern __shared__ float smem[];
   const int c1 = blockIdx.x, bh = blockIdx.y;
   const int d = g.d, b2 = g.b2;
@@ -54,7 +54,7 @@ r_step_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
       qv = (c1 >= g.off) ? to_f(qh[token_of(g, c1 - g.off, c2) * d + c])
                          : w.qbar[((long long)bh * b2 + c2) * d + c];
     } else {
-      qv = to_f(w.qt[(((long long)bh * b2 + c2) * g.b1k + c1) * d + c]);
+      qv = w.qt[(((long long)bh * b2 + c2) * g.b1k + c1) * d + c];
     }
     sQ[i] = qv;  // row a2 = c2 index here: q~[c1, a2]
   }
@@ -105,8 +105,8 @@ r_step_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
       if (final_step) av = fmaf(r[c2], sV[c2 * d + c], av);
     }
     const long long o = (((long long)bh * b2 + a2) * g.b1k + c1) * d + c;
-    w.kt[o] = from_f<T>(ak);
-    if (final_step) w.z[o] = from_f<T>(av);
+    w.kt[o] = ak;
+    if (final_step) w.z[o] = av;
   }
 }
 
@@ -116,9 +116,9 @@ r_step_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
 // out[token(a1,a2)] = sum_c1 L z / sum L (inverse permutation fused into the
 // store); otherwise writes the row's base-2 log-sum-exp.
 // grid (ceil(b1q/ROWS), b2, BH), block 32*ROWS.
-template <typename T, int D>
+template <typename T, typename TO, int D>
 __global__ void __launch_bounds__(512)
-l_row_simt(const T* __restrict__ q, T* __restrict__ out, Work<T> w, Geo g, int final_step) {
+l_row_simt(const T* __restrict__ q, TO* __restrict__ out, Work w, Geo g, int final_step) {
   constexpr int KC = 32;   // key tiles staged per chunk
   constexpr int PER = D / 32;
   __shared__ float sK[KC][D];
@@ -143,8 +143,8 @@ l_row_simt(const T* __restrict__ q, T* __restrict__ out, Work<T> w, Geo g, int f
     __syncthreads();
     for (int i = threadIdx.x; i < nk * D; i += blockDim.x) {
       const int j = i / D, c = i - j * D;
-      sK[j][c] = to_f(w.kt[(base + c0 + j) * D + c]);
-      if (final_step) sZ[j][c] = to_f(w.z[(base + c0 + j) * D + c]);
+      sK[j][c] = w.kt[(base + c0 + j) * D + c];
+      if (final_step) sZ[j][c] = w.z[(base + c0 + j) * D + c];
     }
     for (int j = threadIdx.x; j < nk; j += blockDim.x) sH[j] = w.h[base + c0 + j] * kLog2e;
     __syncthreads();
@@ -167,9 +167,9 @@ l_row_simt(const T* __restrict__ q, T* __restrict__ out, Work<T> w, Geo g, int f
   if (!valid) return;
   if (final_step) {
     const float inv = 1.f / l;
-    T* orow = out + (long long)bh * g.Nq * D + token_of(g, a1, a2) * D;
+    TO* orow = out + (long long)bh * g.Nq * D + token_of(g, a1, a2) * D;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = from_f<T>(acc[i] * inv);
+    for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = from_f<TO>(acc[i] * inv);
   } else if (lane == 0) {
     w.lse[((long long)bh * g.b2 + a2) * g.b1q + a1] = m + log2f(l);
   }
@@ -182,7 +182,7 @@ l_row_simt(const T* __restrict__ q, T* __restrict__ out, Work<T> w, Geo g, int f
 // grid (ceil(b1k/ROWS), b2, BH), block 32*ROWS.
 template <typename T, int D>
 __global__ void __launch_bounds__(512)
-l_col_simt(const T* __restrict__ q, Work<T> w, Geo g) {
+l_col_simt(const T* __restrict__ q, Work w, Geo g) {
   constexpr int QC = 32;
   constexpr int PER = D / 32;
   __shared__ float sQ[QC][D];
@@ -196,7 +196,7 @@ l_col_simt(const T* __restrict__ q, Work<T> w, Geo g) {
   float kv[PER], acc[PER];
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
-    kv[i] = valid ? to_f(w.kt[(kbase + c1) * D + lane + 32 * i]) * g.sl2 : 0.f;
+    kv[i] = valid ? w.kt[(kbase + c1) * D + lane + 32 * i] * g.sl2 : 0.f;
     acc[i] = 0.f;
   }
   const float hb = valid ? w.h[kbase + c1] * kLog2e : 0.f;
@@ -231,7 +231,7 @@ l_col_simt(const T* __restrict__ q, Work<T> w, Geo g) {
   if (!valid) return;
   const float inv = 1.f / beta;
 #pragma unroll
-  for (int i = 0; i < PER; ++i) w.qt[(kbase + c1) * D + lane + 32 * i] = from_f<T>(acc[i] * inv);
+  for (int i = 0; i < PER; ++i) w.qt[(kbase + c1) * D + lane + 32 * i] = acc[i] * inv;
 }
 
 }  // namespace monarch

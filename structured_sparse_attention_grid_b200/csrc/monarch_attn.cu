@@ -83,6 +83,7 @@ size_t elem_size(int dtype) { return dtype == MONARCH_F32 ? 4 : 2; }
 struct Plan {
   Geo g;
   int dtype;
+  int out_dtype;
   int iters;
   bool kv;
   size_t off[6];
@@ -92,7 +93,7 @@ struct Plan {
 constexpr int kMaxB2 = 64;
 
 int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int iters,
-              long kv_len, int dtype, Plan* p) {
+              long kv_len, int dtype, int out_dtype, Plan* p) {
   if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1)
     return fail(MONARCH_EINVAL, "B, heads, T, H, W must be >= 1 (got %d %d %d %d %d)", B, heads, T, H, W);
   if (d != 64 && d != 128) return fail(MONARCH_EINVAL, "head_dim d must be 64 or 128 (got %d)", d);
@@ -101,6 +102,8 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
   if (iters < 1) return fail(MONARCH_EINVAL, "iters must be >= 1 (got %d)", iters);
   if (dtype != MONARCH_F32 && dtype != MONARCH_BF16 && dtype != MONARCH_F16)
     return fail(MONARCH_EINVAL, "unknown dtype %d", dtype);
+  if (out_dtype != dtype && out_dtype != MONARCH_F32)
+    return fail(MONARCH_EINVAL, "out_dtype %d must be MONARCH_F32 or the input dtype %d", out_dtype, dtype);
   const long long hw = (long long)H * W;
   const long long nq = (long long)T * hw;
   if (kv_len < nq || kv_len % hw)
@@ -130,10 +133,10 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
   g.Nk = kv_len;
   g.sl2 = (float)(1.0 / std::sqrt((double)d) * 1.4426950408889634);
   p->dtype = dtype;
+  p->out_dtype = out_dtype;
   p->iters = iters;
   p->kv = g.Tk != T;
-  const size_t es = elem_size(dtype);
-  const size_t big = (size_t)BH * g.b2 * g.b1k * d * es;
+  const size_t big = (size_t)BH * g.b2 * g.b1k * d * 4;  // fp32, or two fp16 planes
   size_t sizes[6] = {big, big, big, (size_t)BH * g.b2 * g.b1k * 4, (size_t)BH * g.b2 * g.b1q * 4,
                      (size_t)BH * g.b2 * d * 4};
   size_t o = 0;
@@ -151,13 +154,13 @@ int check_ptr(const void* ptr, const char* name) {
   return MONARCH_OK;
 }
 
-template <typename T>
-int run(const Plan& p, const T* q, const T* k, const T* v, T* out, char* ws, cudaStream_t st) {
+template <typename T, typename TO>
+int run(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* ws, cudaStream_t st) {
   const Geo& g = p.g;
-  Work<T> w;
-  w.kt = reinterpret_cast<T*>(ws + p.off[0]);
-  w.z = reinterpret_cast<T*>(ws + p.off[1]);
-  w.qt = reinterpret_cast<T*>(ws + p.off[2]);
+  Work w;
+  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
+  w.z = reinterpret_cast<float*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
   w.h = reinterpret_cast<float*>(ws + p.off[3]);
   w.lse = reinterpret_cast<float*>(ws + p.off[4]);
   w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
@@ -185,8 +188,8 @@ int run(const Plan& p, const T* q, const T* k, const T* v, T* out, char* ws, cud
     });
     dim3 grid((g.b1q + kRows - 1) / kRows, g.b2, g.BH);
     launch(final_step ? MONARCH_PHASE_L_OUT : MONARCH_PHASE_L_ROW, st, [&] {
-      if (g.d == 128) l_row_simt<T, 128><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
-      else l_row_simt<T, 64><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
+      if (g.d == 128) l_row_simt<T, TO, 128><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
+      else l_row_simt<T, TO, 64><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
     });
   }
   e = cudaGetLastError();
@@ -194,17 +197,21 @@ int run(const Plan& p, const T* q, const T* k, const T* v, T* out, char* ws, cud
   return MONARCH_OK;
 }
 
+template <typename T>
+int dispatch_out(const Plan& p, const void* q, const void* k, const void* v, void* out, char* w,
+                 cudaStream_t st) {
+  if (p.out_dtype == MONARCH_F32)
+    return run<T, float>(p, (const T*)q, (const T*)k, (const T*)v, (float*)out, w, st);
+  return run<T, T>(p, (const T*)q, (const T*)k, (const T*)v, (T*)out, w, st);
+}
+
 int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* out, void* ws,
              cudaStream_t st) {
   char* w = static_cast<char*>(ws);
   switch (p.dtype) {
-    case MONARCH_F32:
-      return run<float>(p, (const float*)q, (const float*)k, (const float*)v, (float*)out, w, st);
-    case MONARCH_BF16:
-      return run<__nv_bfloat16>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
-                                (const __nv_bfloat16*)v, (__nv_bfloat16*)out, w, st);
-    default:
-      return run<__half>(p, (const __half*)q, (const __half*)k, (const __half*)v, (__half*)out, w, st);
+    case MONARCH_F32: return dispatch_out<float>(p, q, k, v, out, w, st);
+    case MONARCH_BF16: return dispatch_out<__nv_bfloat16>(p, q, k, v, out, w, st);
+    default: return dispatch_out<__half>(p, q, k, v, out, w, st);
   }
 }
 
@@ -259,7 +266,7 @@ size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int 
                                      int tile_w, int iters, long kv_len, int dtype,
                                      size_t offsets[6]) {
   Plan p;
-  if (make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p) != MONARCH_OK) return 0;
+  if (make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, dtype, &p) != MONARCH_OK) return 0;
   if (offsets)
     for (int i = 0; i < 6; ++i) offsets[i] = p.off[i];
   return p.total;
@@ -273,10 +280,11 @@ size_t monarch_attn_workspace_bytes(int B, int heads, int T, int H, int W, int d
 
 int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out, int B, int heads,
                         int T, int H, int W, int d, int tile_h, int tile_w, int iters, long kv_len,
-                        int dtype, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+                        int dtype, int out_dtype, void* workspace, size_t workspace_bytes,
+                        cudaStream_t stream) {
   g_err.clear();
   Plan p;
-  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
   if (rc) return rc;
   if ((rc = check_io(q, k, v, out))) return rc;
   if ((rc = check_ptr(workspace, "workspace"))) return rc;
@@ -287,10 +295,10 @@ int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out, 
 
 int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int heads,
                      int T, int H, int W, int d, int tile_h, int tile_w, int iters, long kv_len,
-                     int dtype, cudaStream_t stream) {
+                     int dtype, int out_dtype, cudaStream_t stream) {
   g_err.clear();
   Plan p;
-  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
   if (rc) return rc;
   if ((rc = check_io(q, k, v, out))) return rc;
   void* ws = nullptr;
@@ -308,17 +316,18 @@ int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int
 int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                           void* out_host, int B, int heads, int T, int H, int W, int d,
                           int tile_h, int tile_w, int iters, long kv_len, int dtype,
-                          cudaStream_t stream) {
+                          int out_dtype, cudaStream_t stream) {
   g_err.clear();
   Plan p;
-  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, &p);
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
   if (rc) return rc;
   if (!q_host || !k_host || !v_host || !out_host) return fail(MONARCH_EINVAL, "null host pointer");
   const size_t es = elem_size(dtype);
   const size_t qb = (size_t)p.g.BH * p.g.Nq * d * es;
   const size_t kb = (size_t)p.g.BH * p.g.Nk * d * es;
+  const size_t ob = (size_t)p.g.BH * p.g.Nq * d * elem_size(out_dtype);
   const size_t oq = 0, ok = align256(qb), ov = ok + align256(kb), oo = ov + align256(kb);
-  const size_t ow = oo + align256(qb);
+  const size_t ow = oo + align256(ob);
   char* buf = nullptr;
   cudaError_t e = cudaMallocAsync((void**)&buf, ow + p.total, stream);
   if (e != cudaSuccess) {
@@ -331,7 +340,7 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
     rc = cuda_fail(e, "cudaMemcpyAsync(host->device)");
   }
   if (rc == MONARCH_OK) rc = dispatch(p, buf + oq, buf + ok, buf + ov, buf + oo, buf + ow, stream);
-  if (rc == MONARCH_OK && (e = cudaMemcpyAsync(out_host, buf + oo, qb, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
+  if (rc == MONARCH_OK && (e = cudaMemcpyAsync(out_host, buf + oo, ob, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
     rc = cuda_fail(e, "cudaMemcpyAsync(device->host)");
   cudaFreeAsync(buf, stream);
   e = cudaStreamSynchronize(stream);

@@ -58,7 +58,7 @@ def _ws(c, **kw):
 
 def test_workspace_bytes_counts_the_intermediates(lib):
     total, offs = m.workspace_layout(1, 12, 3, 30, 52, 128, 6, 4, 2, 4680, 1)
-    big = 12 * 24 * 195 * 128 * 2  # k~, z, q~ in bf16
+    big = 12 * 24 * 195 * 128 * 4  # k~, z, q~: fp32 or two f16 planes
     assert offs[0] == 0 and offs[1] >= big and offs[2] - offs[1] >= big
     assert total >= 3 * big + 12 * 24 * 195 * 4 * 2
     assert total == _ws(CFG1)
@@ -87,15 +87,23 @@ def test_oversized_tile_is_unsupported(lib):
 def test_null_pointer_is_rejected_before_any_launch(lib):
     c = CFG1
     rc = lib.monarch_attn_fwd(None, None, None, None, c["B"], c["heads"], c["T"], c["H"], c["W"], c["d"],
-                              c["th"], c["tw"], c["iters"], c["kv"], c["dt"], None)
+                              c["th"], c["tw"], c["iters"], c["kv"], c["dt"], c["dt"], None)
     assert rc == -1
     assert "null" in lib.monarch_attn_last_error().decode()
+
+
+def test_bad_output_dtype_is_rejected(lib):
+    c = CFG1
+    rc = lib.monarch_attn_fwd(0x1000, 0x2000, 0x3000, 0x4000, c["B"], c["heads"], c["T"], c["H"], c["W"],
+                              c["d"], c["th"], c["tw"], c["iters"], c["kv"], 1, 2, None)
+    assert rc == -1
+    assert "out_dtype" in lib.monarch_attn_last_error().decode()
 
 
 def test_misaligned_pointer_is_rejected(lib):
     c = CFG1
     rc = lib.monarch_attn_fwd(0x1008, 0x2000, 0x3000, 0x4000, c["B"], c["heads"], c["T"], c["H"], c["W"],
-                              c["d"], c["th"], c["tw"], c["iters"], c["kv"], c["dt"], None)
+                              c["d"], c["th"], c["tw"], c["iters"], c["kv"], c["dt"], c["dt"], None)
     assert rc == -1
     assert "aligned" in lib.monarch_attn_last_error().decode()
 

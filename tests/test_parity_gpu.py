@@ -24,9 +24,9 @@ def _grid(w):
     return om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None)
 
 
-def _run_gpu(w, q, k, v):
+def _run_gpu(w, q, k, v, out_dtype=torch.float32):
     qd, kd, vd = (t.cuda() for t in (q, k, v))
-    out = torch.empty_like(qd)
+    out = torch.empty(qd.shape, dtype=out_dtype, device=qd.device)
     m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
     torch.cuda.synchronize()
     return out
@@ -163,6 +163,15 @@ def test_intermediates_match_the_oracle_on_the_toy(cuda_lib):
         np.testing.assert_allclose(hh[h], st.h.T, atol=1e-4)
 
 
+def test_output_in_input_dtype_is_the_rounded_f32_output(cuda_lib):
+    for name in ("chunk_4680_bf16", "sweep_2048_f16"):
+        w = WORKLOADS[name]
+        q, k, v = make_inputs(w)
+        o32 = _run_gpu(w, q, k, v)
+        olow = _run_gpu(w, q, k, v, out_dtype=q.dtype)
+        assert torch.equal(olow, o32.to(q.dtype))
+
+
 def test_host_buffer_entry_point(cuda_lib):
     w = WORKLOADS["toy_256_f32"]
     q, k, v = make_inputs(w)
@@ -177,7 +186,8 @@ def test_workspace_entry_point_matches_allocating_call(cuda_lib):
     q, k, v = (t.cuda() for t in make_inputs(w))
     total, _ = m.workspace_layout(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw, w.iters, w.Nk, m.MONARCH_BF16)
     ws = torch.empty(total, dtype=torch.uint8, device="cuda")
-    a, b = torch.empty_like(q), torch.empty_like(q)
+    a = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    b = torch.empty_like(a)
     m.monarch_attn_fwd(q, k, v, a, w.T, w.H, w.W, w.th, w.tw, w.iters)
     m.monarch_attn_fwd_ws(q, k, v, b, ws, w.T, w.H, w.W, w.th, w.tw, w.iters)
     torch.cuda.synchronize()
@@ -187,7 +197,8 @@ def test_workspace_entry_point_matches_allocating_call(cuda_lib):
 def test_repeated_calls_are_deterministic(cuda_lib):
     w = WORKLOADS["sweep_2048_f16"]
     q, k, v = (t.cuda() for t in make_inputs(w))
-    a, b = torch.empty_like(q), torch.empty_like(q)
+    a = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    b = torch.empty_like(a)
     m.monarch_attn_fwd(q, k, v, a, w.T, w.H, w.W, w.th, w.tw, w.iters)
     m.monarch_attn_fwd(q, k, v, b, w.T, w.H, w.W, w.th, w.tw, w.iters)
     torch.cuda.synchronize()
