@@ -10,9 +10,13 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "monarch_attn.h"
 #include "common.cuh"
 #include "kernels_simt.cuh"
+#include "kernels_tc.cuh"
+#include "kernels_rstep.cuh"
 
 using namespace monarch;
 
@@ -112,7 +116,7 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
     return fail(MONARCH_EUNSUPPORTED, "tile_h*tile_w = %d exceeds the supported %d positions per tile", th * tw, kMaxB2);
   const long long Tk = kv_len / hw;
   const long long BH = (long long)B * heads;
-  if (BH * (long long)kv_len * d >= (1LL << 40) || Tk * (H / th) * (W / tw) >= (1LL << 30))
+  if (BH * (long long)kv_len * d >= (1LL << 40) || Tk * (H / th) * (W / tw) >= (1LL << 30) || BH > 65535)
     return fail(MONARCH_EUNSUPPORTED, "problem too large");
   Geo& g = p->g;
   g.BH = (int)BH;
@@ -151,6 +155,111 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
 int check_ptr(const void* ptr, const char* name) {
   if (!ptr) return fail(MONARCH_EINVAL, "%s is null", name);
   if (reinterpret_cast<uintptr_t>(ptr) & 15) return fail(MONARCH_EINVAL, "%s is not 16-byte aligned", name);
+  return MONARCH_OK;
+}
+
+// ---- tensor-core path (bf16 / f16 inputs) -------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      f = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  }();
+  return fn;
+}
+
+// 3-D map over a pair of planes [2][BH*b2][rows][d] of 16-bit elements; box
+// = 64 elements of d x 128 rows x 1, 128-byte swizzle, zero fill past `rows`.
+int plane_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int d, long long rows,
+              long long planes_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled is not available");
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes_rows};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MONARCH_OK;
+}
+
+template <typename K>
+cudaError_t allow_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <typename TQ, typename TO, int D>
+int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* ws, cudaStream_t st) {
+  const Geo& g = p.g;
+  Work w;
+  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
+  w.z = reinterpret_cast<float*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
+  w.h = reinterpret_cast<float*>(ws + p.off[3]);
+  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
+  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  TcPlanes<TQ> planes;
+  planes.kt_hi = reinterpret_cast<TQ*>(w.kt);
+  planes.z_hi = reinterpret_cast<__half*>(w.z);
+  planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
+
+  const CUtensorMapDataType dq =
+      TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  CUtensorMap tm_kt, tm_z;
+  int rc;
+  if ((rc = plane_map(&tm_kt, planes.kt_hi, dq, D, g.b1k, 2LL * g.BH * g.b2))) return rc;
+  if ((rc = plane_map(&tm_z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, D, g.b1k, 2LL * g.BH * g.b2))) return rc;
+
+  constexpr size_t smem_row = l_row_tc_smem<TQ, D, false>();
+  constexpr size_t smem_out = l_row_tc_smem<TQ, D, true>();
+  constexpr size_t smem_col = l_col_tc_smem<D>();
+  const int mt = (g.b2 + 15) / 16, tpc = 4 / mt;
+  const size_t smem_r = (size_t)tpc * 2 * (16 * mt) * (D + 8) * sizeof(TQ);
+  static bool attrs_set = false;
+  if (!attrs_set) {
+    cudaError_t e;
+    if ((e = allow_smem(l_row_tc<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
+        (e = allow_smem(l_row_tc<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
+        (e = allow_smem(l_col_tc<TQ, D>, smem_col)) != cudaSuccess ||
+        (e = allow_smem(r_step_tc<TQ, D>, 4 * 2 * 64 * (D + 8) * sizeof(TQ))) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncSetAttribute");
+    attrs_set = true;
+  }
+  const dim3 grid_q((g.b1q + kTile - 1) / kTile, g.b2, g.BH);
+  const dim3 grid_k((g.b1k + kTile - 1) / kTile, g.b2, g.BH);
+  const dim3 grid_r((g.b1k + tpc - 1) / tpc, g.BH);
+  for (int it = 0; it < p.iters; ++it) {
+    const int final_step = it == p.iters - 1;
+    int mode = QT_BUFFER;
+    if (it == 0) {
+      mode = p.kv ? QT_KVINIT : QT_IDENTITY;
+      if (p.kv)
+        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
+    } else {
+      launch(MONARCH_PHASE_L_COL, st, [&] {
+        l_col_tc<TQ, D><<<grid_k, 128, smem_col, st>>>(q, tm_kt, w.h, w.lse, w.qt, g);
+      });
+    }
+    launch(MONARCH_PHASE_R_STEP, st, [&] {
+      r_step_tc<TQ, D><<<grid_r, 128, smem_r, st>>>(q, k, v, w, planes, g, mode, final_step);
+    });
+    if (final_step) {
+      launch(MONARCH_PHASE_L_OUT, st, [&] {
+        l_row_tc<TQ, TO, D, true><<<grid_q, 128, smem_out, st>>>(q, out, tm_kt, tm_z, w.h, w.lse, g);
+      });
+    } else {
+      launch(MONARCH_PHASE_L_ROW, st, [&] {
+        l_row_tc<TQ, TO, D, false><<<grid_q, 128, smem_row, st>>>(q, out, tm_kt, tm_z, w.h, w.lse, g);
+      });
+    }
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return MONARCH_OK;
 }
 
@@ -197,12 +306,22 @@ int run(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* ws, cu
   return MONARCH_OK;
 }
 
+template <typename T, typename TO>
+int run_any(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* w, cudaStream_t st) {
+  if constexpr (sizeof(T) == 4) {
+    return run<T, TO>(p, q, k, v, out, w, st);
+  } else {
+    if (p.g.d == 128) return run_tc<T, TO, 128>(p, q, k, v, out, w, st);
+    return run_tc<T, TO, 64>(p, q, k, v, out, w, st);
+  }
+}
+
 template <typename T>
 int dispatch_out(const Plan& p, const void* q, const void* k, const void* v, void* out, char* w,
                  cudaStream_t st) {
   if (p.out_dtype == MONARCH_F32)
-    return run<T, float>(p, (const T*)q, (const T*)k, (const T*)v, (float*)out, w, st);
-  return run<T, T>(p, (const T*)q, (const T*)k, (const T*)v, (T*)out, w, st);
+    return run_any<T, float>(p, (const T*)q, (const T*)k, (const T*)v, (float*)out, w, st);
+  return run_any<T, T>(p, (const T*)q, (const T*)k, (const T*)v, (T*)out, w, st);
 }
 
 int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* out, void* ws,
