@@ -137,6 +137,13 @@ int monarch_attn_profile_enable(int on);
  * totals afterwards.  Returns MONARCH_OK or MONARCH_ECUDA. */
 int monarch_attn_profile_read(double* ms, unsigned long long* launches, int n, int reset);
 
+/* Device error word of the current device: 0 when no kernel of this library
+ * has reported a problem; 1 when a bounded wait inside a kernel gave up (the
+ * kernel then skipped its remaining work and its output is invalid).
+ * Synchronous (reads device memory); reset != 0 clears the word.  Returns -1
+ * if the word cannot be read. */
+int monarch_attn_device_error(int reset);
+
 /* Thread-local message of the last failing call ("" if none). */
 const char* monarch_attn_last_error(void);
 

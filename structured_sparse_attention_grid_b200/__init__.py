@@ -33,6 +33,7 @@ _SIGS = {
     "monarch_attn_profile_read": (ctypes.c_int, [ctypes.POINTER(ctypes.c_double),
                                                  ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int,
                                                  ctypes.c_int]),
+    "monarch_attn_device_error": (ctypes.c_int, [ctypes.c_int]),
     "monarch_attn_last_error": (ctypes.c_char_p, []),
     "monarch_attn_version": (ctypes.c_int, []),
 }
@@ -159,3 +160,8 @@ def profile_read(reset: bool = True) -> dict:
     cnt = (ctypes.c_ulonglong * n)()
     _check(lib.monarch_attn_profile_read(ms, cnt, n, 1 if reset else 0))
     return {p: (float(ms[i]), int(cnt[i])) for i, p in enumerate(PHASES)}
+
+
+def device_error(reset: bool = False) -> int:
+    """0 unless a library kernel gave up a bounded wait (see the header)."""
+    return int(load_library().monarch_attn_device_error(1 if reset else 0))

@@ -41,6 +41,7 @@ template <> struct TcType<__half> {
 constexpr int kTile = 128;          // rows of every tensor-core tile
 constexpr int kHalfBytes = 16384;   // one [128 rows][128 B] swizzled half
 constexpr float kColShift = 15.f;   // L^T q: L scaled by 2^15 (the ratio is unchanged)
+constexpr float kLazyRescale = 8.f; // row pass: shift moves only when the max grows by > 2^8
 
 // Gathers the 128 query rows (a1 = blk*128 + r) of position a2 into a
 // swizzled operand tile with cp.async; thread r copies row r.  Rows past b1q
@@ -189,12 +190,15 @@ l_row_tc(const TQ* __restrict__ q, TO* __restrict__ out, const __grid_constant__
     float mb = -INFINITY;
 #pragma unroll
     for (int i = 0; i < kTile; ++i) mb = fmaxf(mb, x[i]);
-    const float mn = fmaxf(m, mb);
-    const float corr = ptx::ex2(m - mn);  // 0 on the first tile
+    // The running shift m moves only when the tile max exceeds it by more than
+    // 2^8 (P <= 256 stays exact-range in f16); the accumulator is rescaled then.
+    const bool move = mb > m + kLazyRescale;
+    const float mn = move ? mb : m;
+    const float corr = ptx::ex2(m - mn);  // 0 on the first tile, 1 when m stays
     float sum = 0.f;
     if (OUT) {
-      if (j > 0 && mn > m) {
-        // rescale the output accumulator row
+      // tcgen05.ld / st are warp-collective: rescale when any lane moved
+      if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t r[32];

@@ -5,6 +5,8 @@
 #include <cstdio>
 #include <cstring>
 #include <cmath>
+#include <chrono>
+#include <cstdlib>
 #include <mutex>
 #include <atomic>
 #include <string>
@@ -63,11 +65,34 @@ struct Profiler {
 };
 Profiler g_prof;
 
+// MONARCH_DEBUG_SYNC=1: synchronise after every launch and report the phase,
+// the time and the device error word on stderr (debugging aid).
+bool debug_sync() {
+  static const bool on = [] {
+    const char* e = getenv("MONARCH_DEBUG_SYNC");
+    return e && e[0] == '1';
+  }();
+  return on;
+}
+
+int read_device_error(int reset);
+
 // Launches one kernel through `f`, counting it and, when profiling is on,
 // bracketing it with events on its stream.
 template <typename F>
 void launch(int phase, cudaStream_t st, F&& f) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (debug_sync()) {
+    static const char* names[] = {"qbar", "r_step", "l_row", "l_out", "l_col"};
+    fprintf(stderr, "[monarch] launch %s ...\n", names[phase]);
+    auto t0 = std::chrono::steady_clock::now();
+    f();
+    cudaError_t e = cudaStreamSynchronize(st);
+    const double ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
+    fprintf(stderr, "[monarch]   %s done: %.3f ms, %s, device error word %d\n", names[phase], ms,
+            cudaGetErrorString(e), read_device_error(0));
+    return;
+  }
   if (!g_prof.on) {
     f();
     return;
@@ -78,6 +103,16 @@ void launch(int phase, cudaStream_t st, F&& f) {
   f();
   cudaEventRecord(b, st);
   g_prof.pending.push_back({phase, a, b});
+}
+
+int read_device_error(int reset) {
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, ptx::g_device_error, sizeof(int)) != cudaSuccess) return -1;
+  if (reset) {
+    const int z = 0;
+    cudaMemcpyToSymbol(ptx::g_device_error, &z, sizeof(int));
+  }
+  return v;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -349,6 +384,8 @@ extern "C" {
 int monarch_attn_version(void) { return 100; }
 
 unsigned long long monarch_attn_launch_count(void) { return g_launches.load(); }
+
+int monarch_attn_device_error(int reset) { return read_device_error(reset); }
 
 int monarch_attn_profile_enable(int on) {
   std::lock_guard<std::mutex> lk(g_prof.mu);
