@@ -100,6 +100,27 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
                           int tile_h, int tile_w, int iters, long kv_len,
                           int dtype, int out_dtype, cudaStream_t stream);
 
+/* Allocation-free forward (no counterpart in the paper: an interface for
+ * callers that cannot allocate device memory while they run, such as a
+ * real-time generation loop that must never stall or fail on an allocation,
+ * or a host application that owns all device memory).  Same arguments and
+ * result as monarch_attn_fwd, but the workspace comes from a fixed 96 MiB
+ * array in device memory that the library holds on every device it is
+ * loaded on until the process exits; no cudaMalloc / cudaMallocAsync /
+ * cudaFree is called.  Problems whose workspace
+ * (monarch_attn_workspace_bytes) exceeds 96 MiB are rejected with
+ * MONARCH_ENOMEM and a message.  The first call on a device looks up the
+ * array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture.  All calls on a device
+ * share the one array and it keeps the last call's contents (every value is
+ * written before it is read, so nothing needs clearing): calls whose GPU work
+ * overlaps (different streams, or different host threads) race on it and
+ * must be serialised by the caller. */
+int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                             int B, int heads, int T, int H, int W, int d,
+                             int tile_h, int tile_w, int iters, long kv_len,
+                             int dtype, int out_dtype, cudaStream_t stream);
+
 /* Byte offsets, inside a workspace, of the intermediates left by the last
  * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (f32 for
  * f32 inputs; otherwise an f16 high plane followed by an f16 low plane),

@@ -24,6 +24,8 @@ _SIGS = {
     "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                ctypes.c_size_t, ctypes.c_void_p]),
+    "monarch_attn_fwd_noalloc": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                                 + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                               + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_workspace_layout": (ctypes.c_size_t, [ctypes.c_int] * 9
@@ -128,6 +130,19 @@ def monarch_attn_fwd_ws(q, k, v, out, workspace, T, H, W, tile_h, tile_w, iters,
                                    *args, _dtype_code(q), _dtype_code(out), workspace.data_ptr(),
                                    workspace.numel() * workspace.element_size(),
                                    _stream_ptr(stream)))
+    return out
+
+
+def monarch_attn_fwd_noalloc(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
+    """As monarch_attn_fwd, for callers that cannot allocate device memory
+    while running: the library takes its workspace from a fixed 96 MiB array
+    it holds on each device, so no allocation happens.  Larger problems are
+    rejected; concurrent calls on one device must not overlap on the GPU."""
+    lib = load_library()
+    _check_tensors(q, k, v, out)
+    args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
+    _check(lib.monarch_attn_fwd_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                        *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
 
 

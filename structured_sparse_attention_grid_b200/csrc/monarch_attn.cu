@@ -505,3 +505,57 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free forward.  Some callers cannot allocate device memory once
+// they are running: a real-time generation loop that must not stall or fail
+// on an allocation mid-stream, or a host application that owns every byte of
+// device memory and forbids allocations from plug-ins.  This entry point takes
+// its workspace from a fixed array in device memory that exists as soon as the
+// library is loaded on a device (and stays until the process exits), so it
+// never calls cudaMalloc, cudaMallocAsync or cudaFree.
+constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;  // 96 MiB per device
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device.  The host-side
+// name of the array is only a stand-in, so the address is looked up once per
+// device, with that device current, and cached.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+    g_scratch_ptr[dev] = p;
+  }
+  *out = g_scratch_ptr[dev];
+  return MONARCH_OK;
+}
+}  // namespace
+
+extern "C" int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out, int B,
+                                        int heads, int T, int H, int W, int d, int tile_h, int tile_w,
+                                        int iters, long kv_len, int dtype, int out_dtype, cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
+  if (rc) return rc;
+  if ((rc = check_io(q, k, v, out))) return rc;
+  if (p.total > kNoAllocScratchBytes)
+    return fail(MONARCH_ENOMEM,
+                "problem needs %zu bytes of workspace; the allocation-free entry point has a fixed %zu-byte "
+                "scratch array (use monarch_attn_fwd or monarch_attn_fwd_ws)",
+                p.total, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch(&scratch))) return rc;
+  return dispatch(p, q, k, v, out, scratch, stream);
+}
