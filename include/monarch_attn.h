@@ -37,8 +37,10 @@
  *
  * Ownership: the caller owns q, k, v, out (device memory, 16-byte aligned).
  * The library never keeps a pointer past the call's stream work.
- * monarch_attn_fwd allocates its workspace stream-ordered on `stream`
- * (cudaMallocAsync / cudaFreeAsync); monarch_attn_fwd_ws uses a caller buffer
+ * monarch_attn_fwd allocates its workspace stream-ordered on `stream` from a
+ * per-device memory pool owned by the library that keeps freed memory for the
+ * next call (cudaMallocFromPoolAsync / cudaFreeAsync); monarch_attn_fwd_ws
+ * uses a caller buffer
  * of at least monarch_attn_workspace_bytes(...) bytes instead.
  *
  * Behaviour: asynchronous on `stream` (no host synchronisation, except in
@@ -104,11 +106,11 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
  * callers that cannot allocate device memory while they run, such as a
  * real-time generation loop that must never stall or fail on an allocation,
  * or a host application that owns all device memory).  Same arguments and
- * result as monarch_attn_fwd, but the workspace comes from a fixed 96 MiB
+ * result as monarch_attn_fwd, but the workspace comes from a fixed 128 MiB
  * array in device memory that the library holds on every device it is
  * loaded on until the process exits; no cudaMalloc / cudaMallocAsync /
  * cudaFree is called.  Problems whose workspace
- * (monarch_attn_workspace_bytes) exceeds 96 MiB are rejected with
+ * (monarch_attn_workspace_bytes) exceeds 128 MiB are rejected with
  * MONARCH_ENOMEM and a message.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
  * make that first call before any stream capture.  All calls on a device
@@ -123,15 +125,18 @@ int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* 
 
 /* Byte offsets, inside a workspace, of the intermediates left by the last
  * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (f32 for
- * f32 inputs; otherwise an f16 high plane followed by an f16 low plane),
- * [1] z (same form), [2] q~ of the last R step with iters >= 2 (f32, same
- * shape), [3] h [B*heads][b2][b1k] (f32), [4] row log2-sum-exp of
- * the last non-final L step [B*heads][b2][b1q] (f32, base-2 logits s*log2(e)*
- * q.k~ + log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32).  Returns
- * the total bytes, 0 on invalid arguments. */
+ * f32 inputs; otherwise a high plane of the input type followed by a low
+ * plane), [1] z (f32 for f32 inputs; otherwise f16 high and low planes),
+ * [2] q~ of the last R step with iters >= 2 (f32, same shape), [3] h
+ * [B*heads][b2][b1k_pad] (f32), [4] row log2-sum-exp of the last non-final
+ * L step [B*heads][b2][b1q_pad] (f32, base-2 logits s*log2(e)*q.k~ +
+ * log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32), [6] queries in
+ * block-major order [B*heads][b2][b1q][d] (input type; bf16/f16 only).
+ * b1k_pad and b1q_pad are b1k and b1q rounded up to a multiple of 4.
+ * Returns the total bytes, 0 on invalid arguments. */
 size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int d,
                                      int tile_h, int tile_w, int iters, long kv_len,
-                                     int dtype, size_t offsets[6]);
+                                     int dtype, size_t offsets[7]);
 
 /* Instrumentation.  Kernel phases of one forward: */
 enum {

@@ -113,7 +113,7 @@ def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
 
 def workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype_code):
     lib = load_library()
-    offs = (ctypes.c_size_t * 6)()
+    offs = (ctypes.c_size_t * 7)()
     total = lib.monarch_attn_workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters,
                                               kv_len, dtype_code, offs)
     if total == 0:
@@ -135,7 +135,7 @@ def monarch_attn_fwd_ws(q, k, v, out, workspace, T, H, W, tile_h, tile_w, iters,
 
 def monarch_attn_fwd_noalloc(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
     """As monarch_attn_fwd, for callers that cannot allocate device memory
-    while running: the library takes its workspace from a fixed 96 MiB array
+    while running: the library takes its workspace from a fixed 128 MiB array
     it holds on each device, so no allocation happens.  Larger problems are
     rejected; concurrent calls on one device must not overlap on the GPU."""
     lib = load_library()

@@ -24,6 +24,8 @@ struct Geo {
   int b2;        // positions per tile (th*tw)
   int b1q, b1k;  // query tiles, key tiles
   int off;       // key tile aligned with query tile 0: (Tk - T) * P
+  int b1k_pad;   // row stride of h (b1k rounded up to 4: 16-byte rows for TMA)
+  int b1q_pad;   // row stride of the row LSE
   long long Nq, Nk;
   float sl2;     // s * log2(e), s = 1/sqrt(d)
 };
@@ -75,9 +77,10 @@ struct Work {
   float* kt;    // [BH][b2][b1k][d]  k~[c1,a2]
   float* z;     // [BH][b2][b1k][d]  z[c1,a2]
   float* qt;    // [BH][b2][b1k][d]  q~[c1,a2]
-  float* h;     // [BH][b2][b1k]     entropy of R_{c1}[a2,:]
-  float* lse;   // [BH][b2][b1q]     base-2 log-sum-exp of L rows
+  float* h;     // [BH][b2][b1k_pad] entropy of R_{c1}[a2,:]
+  float* lse;   // [BH][b2][b1q_pad] base-2 log-sum-exp of L rows
   float* qbar;  // [BH][b2][d]       mean query per position (KV init)
+  void* qb;     // [BH][b2][b1q][d]  queries in block-major order (input type)
 };
 
 }  // namespace monarch

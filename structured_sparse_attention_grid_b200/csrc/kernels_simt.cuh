@@ -91,7 +91,7 @@ r_step_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restric
     const float inv = 1.f / l;
     for (int c2 = lane; c2 < b2; c2 += 32) row[c2] *= inv;
     // h = -sum R ln R = ln l - sum R (x ln 2)  with x in base-2 units
-    if (lane == 0) w.h[((long long)bh * b2 + a2) * g.b1k + c1] = logf(l) - (sx * inv) * 0.6931471805599453f;
+    if (lane == 0) w.h[((long long)bh * b2 + a2) * g.b1k_pad + c1] = logf(l) - (sx * inv) * 0.6931471805599453f;
   }
   __syncthreads();
 
@@ -146,7 +146,8 @@ l_row_simt(const T* __restrict__ q, TO* __restrict__ out, Work w, Geo g, int fin
       sK[j][c] = w.kt[(base + c0 + j) * D + c];
       if (final_step) sZ[j][c] = w.z[(base + c0 + j) * D + c];
     }
-    for (int j = threadIdx.x; j < nk; j += blockDim.x) sH[j] = w.h[base + c0 + j] * kLog2e;
+    const float* hrow = w.h + ((long long)bh * g.b2 + a2) * g.b1k_pad;
+    for (int j = threadIdx.x; j < nk; j += blockDim.x) sH[j] = hrow[c0 + j] * kLog2e;
     __syncthreads();
     for (int j = 0; j < nk; ++j) {
       float p = 0.f;
@@ -171,7 +172,7 @@ l_row_simt(const T* __restrict__ q, TO* __restrict__ out, Work w, Geo g, int fin
 #pragma unroll
     for (int i = 0; i < PER; ++i) orow[lane + 32 * i] = from_f<TO>(acc[i] * inv);
   } else if (lane == 0) {
-    w.lse[((long long)bh * g.b2 + a2) * g.b1q + a1] = m + log2f(l);
+    w.lse[((long long)bh * g.b2 + a2) * g.b1q_pad + a1] = m + log2f(l);
   }
 }
 
@@ -199,10 +200,10 @@ l_col_simt(const T* __restrict__ q, Work w, Geo g) {
     kv[i] = valid ? w.kt[(kbase + c1) * D + lane + 32 * i] * g.sl2 : 0.f;
     acc[i] = 0.f;
   }
-  const float hb = valid ? w.h[kbase + c1] * kLog2e : 0.f;
+  const float hb = valid ? w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] * kLog2e : 0.f;
   float beta = 0.f, mc = -INFINITY;
   const T* qh = q + (long long)bh * g.Nq * D;
-  const float* lse = w.lse + ((long long)bh * g.b2 + a2) * g.b1q;
+  const float* lse = w.lse + ((long long)bh * g.b2 + a2) * g.b1q_pad;
   for (int a0 = 0; a0 < g.b1q; a0 += QC) {
     const int nq = min(QC, g.b1q - a0);
     __syncthreads();

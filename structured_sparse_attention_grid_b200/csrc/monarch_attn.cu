@@ -19,6 +19,7 @@
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 #include "kernels_rstep.cuh"
+#include "kernels_tc2.cuh"
 
 using namespace monarch;
 
@@ -119,13 +120,15 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t elem_size(int dtype) { return dtype == MONARCH_F32 ? 4 : 2; }
 
+constexpr int kRegions = 7;  // k~, z, q~, h, lse, mean query, block-major q
+
 struct Plan {
   Geo g;
   int dtype;
   int out_dtype;
   int iters;
   bool kv;
-  size_t off[6];
+  size_t off[kRegions];
   size_t total;
 };
 
@@ -168,6 +171,8 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
   g.b1q = T * g.P;
   g.b1k = g.Tk * g.P;
   g.off = (g.Tk - T) * g.P;
+  g.b1k_pad = (g.b1k + 3) & ~3;
+  g.b1q_pad = (g.b1q + 3) & ~3;
   g.Nq = nq;
   g.Nk = kv_len;
   g.sl2 = (float)(1.0 / std::sqrt((double)d) * 1.4426950408889634);
@@ -175,11 +180,16 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
   p->out_dtype = out_dtype;
   p->iters = iters;
   p->kv = g.Tk != T;
-  const size_t big = (size_t)BH * g.b2 * g.b1k * d * 4;  // fp32, or two fp16 planes
-  size_t sizes[6] = {big, big, big, (size_t)BH * g.b2 * g.b1k * 4, (size_t)BH * g.b2 * g.b1q * 4,
-                     (size_t)BH * g.b2 * d * 4};
+  const size_t big = (size_t)BH * g.b2 * g.b1k * d * 4;  // fp32, or two 16-bit planes
+  size_t sizes[kRegions] = {big,
+                            big,
+                            big,
+                            (size_t)BH * g.b2 * g.b1k_pad * 4,
+                            (size_t)BH * g.b2 * g.b1q_pad * 4,
+                            (size_t)BH * g.b2 * d * 4,
+                            dtype == MONARCH_F32 ? 0 : (size_t)BH * g.b2 * g.b1q * d * 2};
   size_t o = 0;
-  for (int i = 0; i < 6; ++i) {
+  for (int i = 0; i < kRegions; ++i) {
     p->off[i] = o;
     o += align256(sizes[i]);
   }
@@ -206,19 +216,15 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 3-D map over a pair of planes [2][BH*b2][rows][d] of 16-bit elements; box
-// = 64 elements of d x 128 rows x 1, 128-byte swizzle, zero fill past `rows`.
-int plane_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int d, long long rows,
-              long long planes_rows) {
+// Tiled tensor map with a 128-byte swizzle (rank 2 or 3, 16-bit or 32-bit
+// elements); zero fill outside the tensor.
+int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int rank, const cuuint64_t* dims,
+             const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swz) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)rows, (cuuint64_t)planes_rows};
-  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)rows * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(map, dt, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MONARCH_OK;
 }
@@ -238,6 +244,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   w.h = reinterpret_cast<float*>(ws + p.off[3]);
   w.lse = reinterpret_cast<float*>(ws + p.off[4]);
   w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  w.qb = ws + p.off[6];
   TcPlanes<TQ> planes;
   planes.kt_hi = reinterpret_cast<TQ*>(w.kt);
   planes.z_hi = reinterpret_cast<__half*>(w.z);
@@ -245,23 +252,42 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
 
   const CUtensorMapDataType dq =
       TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  CUtensorMap tm_kt, tm_z;
+  v2::Maps maps;
   int rc;
-  if ((rc = plane_map(&tm_kt, planes.kt_hi, dq, D, g.b1k, 2LL * g.BH * g.b2))) return rc;
-  if ((rc = plane_map(&tm_z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, D, g.b1k, 2LL * g.BH * g.b2))) return rc;
+  {
+    const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
+    cuuint32_t box3[3] = {64, (cuuint32_t)v2::kBlk, 1};
+    cuuint64_t dq3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, rows};
+    cuuint64_t sq3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1q * D * 2};
+    cuuint64_t dk3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, 2 * rows};
+    cuuint64_t sk3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1k * D * 2};
+    cuuint32_t box2[2] = {(cuuint32_t)v2::kBlk, 1};
+    cuuint64_t dh2[2] = {(cuuint64_t)g.b1k_pad, rows};
+    cuuint64_t sh2[1] = {(cuuint64_t)g.b1k_pad * 4};
+    cuuint64_t dl2[2] = {(cuuint64_t)g.b1q_pad, rows};
+    cuuint64_t sl2[1] = {(cuuint64_t)g.b1q_pad * 4};
+    if ((rc = make_map(&maps.qb, w.qb, dq, 3, dq3, sq3, box3, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&maps.kt, planes.kt_hi, dq, 3, dk3, sk3, box3, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&maps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&maps.h, w.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dh2, sh2, box2, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+        (rc = make_map(&maps.lse, w.lse, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dl2, sl2, box2,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)))
+      return rc;
+  }
 
-  constexpr size_t smem_row = l_row_tc_smem<TQ, D, false>();
-  constexpr size_t smem_out = l_row_tc_smem<TQ, D, true>();
-  constexpr size_t smem_col = l_col_tc_smem<D>();
+  constexpr size_t smem_row = v2::l_row_smem<D, false>();
+  constexpr size_t smem_out = v2::l_row_smem<D, true>();
+  constexpr size_t smem_col = v2::l_col_smem<D>();
   const int mt = (g.b2 + 15) / 16, tpc = 4 / mt;
-  const size_t smem_r = (size_t)tpc * 2 * (16 * mt) * (D + 8) * sizeof(TQ);
+
   static bool attrs_set = false;
   if (!attrs_set) {
     cudaError_t e;
-    if ((e = allow_smem(l_row_tc<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
-        (e = allow_smem(l_row_tc<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
-        (e = allow_smem(l_col_tc<TQ, D>, smem_col)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc<TQ, D>, 4 * 2 * 64 * (D + 8) * sizeof(TQ))) != cudaSuccess)
+    if ((e = allow_smem(v2::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
+        (e = allow_smem(v2::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
+        (e = allow_smem(v2::l_col<TQ, D>, smem_col)) != cudaSuccess ||
+        (e = allow_smem(r_step_tc<TQ, D>, r_step_tc_smem<D>(64, 3))) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
     attrs_set = true;
   }
@@ -277,19 +303,20 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
     } else {
       launch(MONARCH_PHASE_L_COL, st, [&] {
-        l_col_tc<TQ, D><<<grid_k, 128, smem_col, st>>>(q, tm_kt, w.h, w.lse, w.qt, g);
+        v2::l_col<TQ, D><<<grid_k, v2::kThreads, smem_col, st>>>(maps, w.h, w.qt, g);
       });
     }
+    const size_t smem_r = r_step_tc_smem<D>(g.b2, r_step_slots(mode, final_step));
     launch(MONARCH_PHASE_R_STEP, st, [&] {
       r_step_tc<TQ, D><<<grid_r, 128, smem_r, st>>>(q, k, v, w, planes, g, mode, final_step);
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
-        l_row_tc<TQ, TO, D, true><<<grid_q, 128, smem_out, st>>>(q, out, tm_kt, tm_z, w.h, w.lse, g);
+        v2::l_row<TQ, TO, D, true><<<grid_q, v2::kThreads, smem_out, st>>>(out, maps, w.lse, g);
       });
     } else {
       launch(MONARCH_PHASE_L_ROW, st, [&] {
-        l_row_tc<TQ, TO, D, false><<<grid_q, 128, smem_row, st>>>(q, out, tm_kt, tm_z, w.h, w.lse, g);
+        v2::l_row<TQ, TO, D, false><<<grid_q, v2::kThreads, smem_row, st>>>(out, maps, w.lse, g);
       });
     }
   }
@@ -308,6 +335,7 @@ int run(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* ws, cu
   w.h = reinterpret_cast<float*>(ws + p.off[3]);
   w.lse = reinterpret_cast<float*>(ws + p.off[4]);
   w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  w.qb = ws + p.off[6];
 
   const size_t r_smem = (size_t)(3 * g.b2 * g.d + g.b2 * (g.b2 + 1)) * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(r_step_simt<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)r_smem);
@@ -369,6 +397,33 @@ int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* o
   }
 }
 
+// Stream-ordered workspace comes from a per-device pool owned by the library
+// that keeps freed memory (release threshold = max), so repeated calls reuse
+// it without returning memory to the driver between calls.
+int workspace_pool(cudaMemPool_t* out) {
+  static std::mutex mu;
+  static cudaMemPool_t pools[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool;
+    if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return cuda_fail(e, "cudaMemPoolCreate");
+    uint64_t keep = ~0ull;
+    if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemPoolSetAttribute");
+    pools[dev] = pool;
+  }
+  *out = pools[dev];
+  return MONARCH_OK;
+}
+
 int check_io(const void* q, const void* k, const void* v, const void* out) {
   int rc;
   if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v")) ||
@@ -420,11 +475,11 @@ const char* monarch_attn_last_error(void) { return g_err.c_str(); }
 
 size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int d, int tile_h,
                                      int tile_w, int iters, long kv_len, int dtype,
-                                     size_t offsets[6]) {
+                                     size_t offsets[7]) {
   Plan p;
   if (make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, dtype, &p) != MONARCH_OK) return 0;
   if (offsets)
-    for (int i = 0; i < 6; ++i) offsets[i] = p.off[i];
+    for (int i = 0; i < kRegions; ++i) offsets[i] = p.off[i];
   return p.total;
 }
 
@@ -458,10 +513,12 @@ int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int
   if (rc) return rc;
   if ((rc = check_io(q, k, v, out))) return rc;
   void* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(&ws, p.total, stream);
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, p.total, pool, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(MONARCH_ENOMEM, "cudaMallocAsync(%zu): %s", p.total, cudaGetErrorString(e));
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", p.total, cudaGetErrorString(e));
   }
   rc = dispatch(p, q, k, v, out, ws, stream);
   e = cudaFreeAsync(ws, stream);
@@ -485,10 +542,12 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
   const size_t oq = 0, ok = align256(qb), ov = ok + align256(kb), oo = ov + align256(kb);
   const size_t ow = oo + align256(ob);
   char* buf = nullptr;
-  cudaError_t e = cudaMallocAsync((void**)&buf, ow + p.total, stream);
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync((void**)&buf, ow + p.total, pool, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(MONARCH_ENOMEM, "cudaMallocAsync(%zu): %s", ow + p.total, cudaGetErrorString(e));
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", ow + p.total, cudaGetErrorString(e));
   }
   if ((e = cudaMemcpyAsync(buf + oq, q_host, qb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
       (e = cudaMemcpyAsync(buf + ok, k_host, kb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
@@ -514,7 +573,7 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
 // its workspace from a fixed array in device memory that exists as soon as the
 // library is loaded on a device (and stays until the process exits), so it
 // never calls cudaMalloc, cudaMallocAsync or cudaFree.
-constexpr size_t kNoAllocScratchBytes = size_t(96) << 20;  // 96 MiB per device
+constexpr size_t kNoAllocScratchBytes = size_t(128) << 20;  // 128 MiB per device
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
