@@ -128,7 +128,8 @@ int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* 
  * f32 inputs; otherwise a high plane of the input type followed by a low
  * plane), [1] z (f32 for f32 inputs; otherwise f16 high and low planes),
  * [2] q~ of the last R step with iters >= 2 (f32, same shape), [3] h
- * [B*heads][b2][b1k_pad] (f32), [4] row log2-sum-exp of the last non-final
+ * [B*heads][b2][b1k_pad] (f32; in nats for f32 inputs, in bits, i.e. base-2
+ * entropy, for bf16/f16 inputs), [4] row log2-sum-exp of the last non-final
  * L step [B*heads][b2][b1q_pad] (f32, base-2 logits s*log2(e)*q.k~ +
  * log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32), [6] queries in
  * block-major order [B*heads][b2][b1q][d] (input type; bf16/f16 only).

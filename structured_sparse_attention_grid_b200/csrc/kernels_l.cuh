@@ -1,0 +1,578 @@
+// tcgen05 kernels of the L step for bf16 / f16 inputs (row pass, output pass,
+// column pass).
+//
+// A CTA owns two 128-row tiles (A and B) of one (head, position a2) problem.
+// Warps 0-3 run the softmax of tile A and warps 4-7 that of tile B (thread r
+// of a warpgroup owns row r of its tile = TMEM lane r); warp 8 issues the
+// MMAs and warp 9 the TMA loads, each from one lane.  The issuer alternates
+// between the tiles, so one tile's MMAs run while the other's softmax works.
+//
+// Every MMA is N >= 128 wide: a single thread issues about one tcgen05.mma per
+// 60 cycles, so an N = 64 instruction (32 cycles of math) would leave the
+// tensor pipe half idle.
+//   row pass     S = q [k~_hi ; k~_lo]^T   (N = 128: the two planes of a
+//                64-key block side by side; the softmax adds the halves)
+//   output pass  O += P z_hi + P z_lo      (A = P in TMEM over S, N = d)
+//   column pass  S^T = k~_hi q^T + k~_lo q^T   (128-query blocks, N = 128)
+//                acc += P^T_hi q + P^T_lo q     (A = P^T in TMEM over S^T, N = d)
+// A new score tile is issued into TMEM columns that hold the previous P only
+// after the MMA consuming that P: tcgen05 MMAs of a thread run in issue order
+// and a commit arrives when every earlier MMA is complete, so "S(j+1) done"
+// also means "P z (j) done".
+//
+// Precision: k~ and z as hi/lo planes, q exact, L split into hi/lo planes in
+// the column pass, P single f16 with the rounded values summed, fp32
+// statistics; h arrives in bits (base-2 entropy).
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace monarch {
+namespace tc {
+
+constexpr int kThreads = 320;   // 2 softmax warpgroups + MMA warp + TMA warp
+constexpr int kMmaWarp = 8;
+constexpr int kLoadWarp = 9;
+constexpr int kKS = 3;          // k~ / h stages (row passes)
+constexpr int kQS = 2;          // query / lse stages (column pass)
+constexpr int kQBlk = 128;      // queries per column-pass block
+
+// Both kernels allocate all 512 TMEM columns, so their shared-memory
+// requests are at least 120 KB: one CTA per SM, none waits in tcgen05.alloc.
+constexpr size_t kExclusiveSmem = 120 * 1024;
+
+template <int D, bool OUT>
+constexpr size_t row_smem() {
+  constexpr int NH = D / 64;
+  constexpr size_t need = 1024 + (size_t)2 * NH * 2 * kBox /* q */ + (size_t)kKS * 2 * NH * kBox /* k~ */ +
+                          (OUT ? (size_t)2 * 2 * NH * kBox : 0) /* z */ + kKS * kBlk * 4 + 32 * 8;
+  return need > kExclusiveSmem ? need : kExclusiveSmem;
+}
+
+// ===========================================================================
+// Row pass over 64-key blocks for one (head, position a2, 256 query rows).
+//   OUT:  out[token(a1,a2)] = sum_c1 L z     (inverse permutation in the store)
+//   !OUT: lse[a1] = log2 sum_c1 2^(s q.k~ + h)
+// TMEM, tile t at column 256 t.  OUT: S [0, 128) (q.k~_hi in [0, 64), q.k~_lo
+// in [64, 128); P over [0, 32)), O [128, 128 + D).  !OUT: S buffers [0, 128),
+// [128, 256).
+template <typename TQ, typename TO, int D, bool OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t kQt = NH * 2 * kBox;    // q of one tile (128 rows)
+  constexpr uint32_t kKst = 2 * NH * kBox;   // k~ hi+lo, 64 rows: [d half][plane][64 rows]
+  constexpr uint32_t kZst = 2 * NH * kBox;   // z hi+lo, 64 rows:  [plane][d half][64 rows]
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = base;                                                 // [2 tiles]
+  uint8_t* sK = sQ + 2 * kQt;                                         // [kKS]
+  uint8_t* sZ = sK + kKS * kKst;                                      // [2] (OUT)
+  float* sH = reinterpret_cast<float*>(sZ + (OUT ? 2 * kZst : 0));    // [kKS][64]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sH + kKS * kBlk);
+  uint64_t* q_full = bar + 0;
+  uint64_t* k_full = bar + 1;    // [kKS]
+  uint64_t* k_free = bar + 4;    // [kKS]
+  uint64_t* z_full = bar + 7;    // [2]
+  uint64_t* z_free = bar + 9;    // [2]
+  uint64_t* s_full = bar + 11;   // [tile][buf]
+  uint64_t* s_free = bar + 15;   // [tile][buf]   (!OUT)
+  uint64_t* p_full = bar + 19;   // [tile]        (OUT)
+  uint64_t* o_done = bar + 21;   // [tile]        (OUT)
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 23);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int a2 = blockIdx.y, bh = blockIdx.z;
+  const int a1_base = blockIdx.x * 2 * kTile;
+  const int zrow = bh * g.b2 + a2;
+  const int plane_rows = g.BH * g.b2;
+  const int nkb = (g.b1k + kBlk - 1) / kBlk;
+  const int ntiles = (g.b1q - a1_base > kTile) ? 2 : 1;
+
+  if (tid == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int i = 0; i < kKS; ++i) {
+      ptx::mbar_init(k_full + i, 1);
+      ptx::mbar_init(k_free + i, 4 * ntiles);
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(z_full + i, 1);
+      ptx::mbar_init(z_free + i, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(p_full + t, 4);
+      ptx::mbar_init(o_done + t, 1);
+      for (int b = 0; b < 2; ++b) {
+        ptx::mbar_init(s_full + 2 * t + b, 1);
+        ptx::mbar_init(s_free + 2 * t + b, 4);
+      }
+    }
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
+  auto tO = [&](int t) { return tmem + 256 * t + 128; };
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      // --------------------------------------------------------- TMA producer
+      ptx::prefetch_tmap(&maps.kt);
+      ptx::mbar_expect_tx(q_full, 2 * kQt);
+      for (int t = 0; t < 2; ++t)
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh)
+            ptx::tma_load_3d(sQ + t * kQt + hf * 2 * kBox + rh * kBox, &maps.qb, q_full, hf * 64,
+                             a1_base + t * kTile + rh * kBlk, zrow);
+      bool ok = true;
+      for (int blk = 0; blk < nkb && ok; ++blk) {
+        const int ks = blk % kKS;
+        if (blk >= kKS) ok = ptx::mbar_wait(k_free + ks, ((blk / kKS) - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(k_full + ks, kKst + kBlk * 4);
+        for (int hf = 0; hf < NH; ++hf)
+          for (int p = 0; p < 2; ++p)
+            ptx::tma_load_3d(sK + ks * kKst + (hf * 2 + p) * kBox, &maps.kt, k_full + ks, hf * 64, blk * kBlk,
+                             p * plane_rows + zrow);
+        tma_load_2d(sH + ks * kBlk, &maps.h, k_full + ks, blk * kBlk, zrow);
+        if constexpr (OUT) {
+          const int zs = blk & 1;
+          if (blk >= 2) ok = ptx::mbar_wait(z_free + zs, ((blk >> 1) - 1) & 1);
+          if (!ok) break;
+          ptx::mbar_expect_tx(z_full + zs, kZst);
+          for (int p = 0; p < 2; ++p)
+            for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_load_3d(sZ + zs * kZst + (p * NH + hf) * kBox, &maps.z, z_full + zs, hf * 64, blk * kBlk,
+                               p * plane_rows + zrow);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
+      constexpr uint32_t idS = ptx::idesc_f16(128, 2 * kBlk, TcType<TQ>::kBf16, 0, 0);
+      constexpr uint32_t idPV = ptx::idesc_f16(128, D, 0, 0, 1);
+      const uint32_t aQ = ptx::smem_u32(sQ), aK = ptx::smem_u32(sK), aZ = ptx::smem_u32(sZ);
+      // S(t, blk) into buffer b: A = q tile (K-major), B = [k~_hi ; k~_lo] of
+      // one d half (128 rows).  Descriptors are built once; a byte offset adds
+      // (offset >> 4) to the start-address field.
+      auto issue_s = [&](int t, int blk, int b) {
+        const uint64_t a0 = ptx::sw128_desc(aQ + t * kQt, 16, 1024);
+        const uint64_t b0 = ptx::sw128_desc(aK + (blk % kKS) * kKst, 16, 1024);
+        const uint32_t td = tS(t, b);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ptx::mma_f16_ss(td, a0 + ((hf * 2 * kBox + k4 * 32) >> 4), b0 + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
+                            (hf | k4) != 0);
+        ptx::mma_commit(s_full + 2 * t + b);
+      };
+      bool ok = ptx::mbar_wait(q_full, 0) && ptx::mbar_wait(k_full, 0);
+      ptx::tc_fence_after();
+      if (ok) {
+        for (int t = 0; t < ntiles; ++t) issue_s(t, 0, 0);
+        if (!OUT && nkb > 1) {
+          ok = ptx::mbar_wait(k_full + 1, 0);
+          ptx::tc_fence_after();
+          if (ok)
+            for (int t = 0; t < ntiles; ++t) issue_s(t, 1, 1);
+        }
+      }
+      for (int j = 0; j < nkb && ok; ++j) {
+        if constexpr (OUT) {
+          ok = ptx::mbar_wait(z_full + (j & 1), (j >> 1) & 1);
+          const uint64_t z0 = ptx::sw128_desc(aZ + (j & 1) * kZst, kBox, 1024);
+          for (int t = 0; t < ntiles && ok; ++t) {
+            ok = ptx::mbar_wait(p_full + t, j & 1);
+            ptx::tc_fence_after();
+            if (!ok) break;
+            const uint32_t tp = tS(t, 0);
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+#pragma unroll
+              for (int kk = 0; kk < kBlk / 16; ++kk)
+                ptx::mma_f16_ts(tO(t), tp + kk * 8, z0 + ((p * NH * kBox + kk * 2048) >> 4), idPV,
+                                (j | p | kk) != 0);
+            if (t == ntiles - 1) ptx::mma_commit(z_free + (j & 1));
+            if (j + 1 < nkb) {
+              // S(t, j+1) overwrites P(t, j): the P z product above runs first
+              ok = ptx::mbar_wait(k_full + (j + 1) % kKS, ((j + 1) / kKS) & 1);
+              ptx::tc_fence_after();
+              if (ok) issue_s(t, j + 1, 0);
+            } else {
+              ptx::mma_commit(o_done + t);
+            }
+          }
+        } else {
+          const int b = j & 1;
+          const uint32_t ph = (j >> 1) & 1;
+          for (int t = 0; t < ntiles && ok; ++t) {
+            ok = ptx::mbar_wait(s_free + 2 * t + b, ph);
+            if (ok && j + 2 < nkb) {
+              ok = ptx::mbar_wait(k_full + (j + 2) % kKS, ((j + 2) / kKS) & 1);
+              ptx::tc_fence_after();
+              if (ok) issue_s(t, j + 2, b);
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- softmax warps
+    const int t = warp >> 2;
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int a1 = a1_base + t * kTile + r;
+    if (t < ntiles) {
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      const float2 sl2 = make_float2(g.sl2, g.sl2);
+      for (int j = 0; j < nkb; ++j) {
+        const int ks = j % kKS;
+        const int b = OUT ? 0 : (j & 1);
+        const uint32_t ph = OUT ? (j & 1) : ((j >> 1) & 1);
+        // after a timed-out wait the loop keeps its shape but skips waits
+        ok = ok && ptx::mbar_wait(s_full + 2 * t + b, ph) && ptx::mbar_wait(k_full + ks, (j / kKS) & 1);
+        ptx::tc_fence_after();
+        const float4* hv = reinterpret_cast<const float4*>(sH + ks * kBlk);
+        float2 x[32];
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // keys 32 hh .. 32 hh + 31
+          uint32_t shi[32], slo[32];
+          ptx::tmem_ld32(tS(t, b) + lane_off + 32 * hh, shi);
+          ptx::tmem_ld32(tS(t, b) + lane_off + 64 + 32 * hh, slo);
+          ptx::tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 h4 = hv[8 * hh + i];
+            const float2 s0 = add2(make_float2(__uint_as_float(shi[4 * i]), __uint_as_float(shi[4 * i + 1])),
+                                   make_float2(__uint_as_float(slo[4 * i]), __uint_as_float(slo[4 * i + 1])));
+            const float2 s1 = add2(make_float2(__uint_as_float(shi[4 * i + 2]), __uint_as_float(shi[4 * i + 3])),
+                                   make_float2(__uint_as_float(slo[4 * i + 2]), __uint_as_float(slo[4 * i + 3])));
+            x[16 * hh + 2 * i] = fma2(s0, sl2, make_float2(h4.x, h4.y));
+            x[16 * hh + 2 * i + 1] = fma2(s1, sl2, make_float2(h4.z, h4.w));
+          }
+        }
+        // S and h of this block are consumed: release the k~/h stage
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(k_free + ks);
+          if (!OUT) ptx::mbar_arrive(s_free + 2 * t + b);
+        }
+        const int valid = min(kBlk, g.b1k - j * kBlk);
+        if (valid < kBlk) {  // only the last block of a ragged row
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            if (2 * i >= valid) x[i].x = -INFINITY;
+            if (2 * i + 1 >= valid) x[i].y = -INFINITY;
+          }
+        }
+        float mb = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) mb = fmaxf(mb, fmaxf(x[i].x, x[i].y));
+        // the running shift moves only when the max grows by more than 2^8
+        const bool move = mb > m + kLazyRescale;
+        const float mn = move ? mb : m;
+        const float corr = ptx::ex2(m - mn);
+        const float2 nm = make_float2(-mn, -mn);
+        float2 acc2 = make_float2(0.f, 0.f);
+        if constexpr (OUT) {
+          // S(t, j) is complete, hence so is P z (j-1): O may be rescaled
+          if (j > 0 && __any_sync(0xffffffffu, move)) {
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              ptx::tmem_ld32(tO(t) + lane_off + cc * 32, o);
+              ptx::tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+              ptx::tmem_st32(tO(t) + lane_off + cc * 32, o);
+            }
+          }
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 d = add2(x[i], nm);
+            const __half2 hp = __floats2half2_rn(ptx::ex2(d.x), ptx::ex2(d.y));
+            acc2 = add2(acc2, __half22float2(hp));
+            pk[i] = *reinterpret_cast<const uint32_t*>(&hp);
+          }
+          // P (keys 2c, 2c+1 in column c) over the first 32 columns of S
+          ptx::tmem_st32(tS(t, 0) + lane_off, pk);
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(p_full + t);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const float2 d = add2(x[i], nm);
+            acc2 = add2(acc2, make_float2(ptx::ex2(d.x), ptx::ex2(d.y)));
+          }
+        }
+        l = fmaf(l, corr, acc2.x + acc2.y);
+        m = mn;
+      }
+      if constexpr (OUT) {
+        ok = ok && ptx::mbar_wait(o_done + t, 0);
+        ptx::tc_fence_after();
+        const float inv = 1.f / l;
+        TO* orow = out + ((long long)bh * g.Nq + (a1 < g.b1q ? token_of(g, a1, a2) : 0)) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO(t) + lane_off + cc * 32, o);
+          ptx::tmem_wait_ld();
+          if (a1 < g.b1q && ok) {
+#pragma unroll
+            for (int i = 0; i < 32; i += 4) {
+              if constexpr (sizeof(TO) == 4) {
+                *reinterpret_cast<float4*>(orow + cc * 32 + i) =
+                    make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
+                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+              } else {
+                TO v4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) v4[e] = from_f<TO>(__uint_as_float(o[i + e]) * inv);
+                *reinterpret_cast<uint2*>(orow + cc * 32 + i) = *reinterpret_cast<uint2*>(v4);
+              }
+            }
+          }
+        }
+      } else if (a1 < g.b1q) {
+        lse[(long long)zrow * g.b1q_pad + a1] = m + log2f(l);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ===========================================================================
+// Column pass for one (head, position a2, 256 key tiles), 128 queries per block:
+//   q~[c1,a2] = sum_a1 L q / sum_a1 L,  L = 2^(s q.k~ + h - lse[a1]).
+// TMEM, tile t at column 256 t:  S^T [0, 128) for 128 queries; P^T is written
+// over it as [hi q0-63 | lo q0-63 | hi q64-127 | lo q64-127] (32 columns
+// each);  acc [128, 128 + D).
+template <int D>
+constexpr size_t col_smem() {
+  constexpr int NH = D / 64;
+  constexpr size_t need = 1024 + (size_t)2 * 2 * NH * 2 * kBox /* k~ */ + (size_t)kQS * NH * 2 * kBox /* q */ +
+                          kQS * kQBlk * 4 + 32 * 8;
+  return need > kExclusiveSmem ? need : kExclusiveSmem;
+}
+
+template <typename TQ, int D>
+__global__ void __launch_bounds__(kThreads, 1)
+l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* __restrict__ qt, Geo g) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t kKt = 2 * NH * 2 * kBox;   // k~ hi+lo of one tile: [plane][d half][128 rows]
+  constexpr uint32_t kQst = NH * 2 * kBox;      // 128 query rows: [d half][128 rows]
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sK = base;                                        // [2 tiles]
+  uint8_t* sQ = sK + 2 * kKt;                                // [kQS]
+  float* sL = reinterpret_cast<float*>(sQ + kQS * kQst);     // [kQS][128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sL + kQS * kQBlk);
+  uint64_t* k_full = bar + 0;
+  uint64_t* q_full = bar + 1;    // [kQS]
+  uint64_t* q_free = bar + 3;    // [kQS]
+  uint64_t* s_full = bar + 5;    // [tile]
+  uint64_t* p_full = bar + 7;    // [tile]
+  uint64_t* o_done = bar + 9;    // [tile]
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 11);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int a2 = blockIdx.y, bh = blockIdx.z;
+  const int kb = blockIdx.x * 2 * kTile;
+  const int zrow = bh * g.b2 + a2;
+  const int plane_rows = g.BH * g.b2;
+  const int nqb = (g.b1q + kQBlk - 1) / kQBlk;
+  const int ntiles = (g.b1k - kb > kTile) ? 2 : 1;
+
+  if (tid == 0) {
+    ptx::mbar_init(k_full, 1);
+    for (int i = 0; i < kQS; ++i) {
+      ptx::mbar_init(q_full + i, 1);
+      ptx::mbar_init(q_free + i, 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      ptx::mbar_init(s_full + t, 1);
+      ptx::mbar_init(p_full + t, 4);
+      ptx::mbar_init(o_done + t, 1);
+    }
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  auto tS = [&](int t) { return tmem + 256 * t; };
+  auto tA = [&](int t) { return tmem + 256 * t + 128; };
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      ptx::prefetch_tmap(&maps.kt);
+      ptx::prefetch_tmap(&maps.qb);
+      ptx::mbar_expect_tx(k_full, 2 * kKt);
+      for (int t = 0; t < 2; ++t)
+        for (int p = 0; p < 2; ++p)
+          for (int hf = 0; hf < NH; ++hf)
+            for (int rh = 0; rh < 2; ++rh)
+              ptx::tma_load_3d(sK + t * kKt + (p * NH + hf) * 2 * kBox + rh * kBox, &maps.kt, k_full, hf * 64,
+                               kb + t * kTile + rh * kBlk, p * plane_rows + zrow);
+      bool ok = true;
+      for (int blk = 0; blk < nqb && ok; ++blk) {
+        const int qs = blk % kQS;
+        if (blk >= kQS) ok = ptx::mbar_wait(q_free + qs, ((blk / kQS) - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(q_full + qs, kQst + kQBlk * 4);
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh)
+            ptx::tma_load_3d(sQ + qs * kQst + hf * 2 * kBox + rh * kBox, &maps.qb, q_full + qs, hf * 64,
+                             blk * kQBlk + rh * kBlk, zrow);
+        for (int rh = 0; rh < 2; ++rh)
+          tma_load_2d(sL + qs * kQBlk + rh * kBlk, &maps.lse, q_full + qs, blk * kQBlk + rh * kBlk, zrow);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idS = ptx::idesc_f16(128, kQBlk, TcType<TQ>::kBf16, 0, 0);
+      constexpr uint32_t idPQ = ptx::idesc_f16(128, D, TcType<TQ>::kBf16, 0, 1);
+      const uint32_t aK = ptx::smem_u32(sK), aQ = ptx::smem_u32(sQ);
+      auto issue_s = [&](int t, int blk) {
+        const uint64_t a0 = ptx::sw128_desc(aK + t * kKt, 16, 1024);
+        const uint64_t b0 = ptx::sw128_desc(aQ + (blk % kQS) * kQst, 16, 1024);
+        const uint32_t td = tS(t);
+#pragma unroll
+        for (int p = 0; p < 2; ++p)
+#pragma unroll
+          for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+            for (int k4 = 0; k4 < 4; ++k4)
+              ptx::mma_f16_ss(td, a0 + (((p * NH + hf) * 2 * kBox + k4 * 32) >> 4),
+                              b0 + ((hf * 2 * kBox + k4 * 32) >> 4), idS, (p | hf | k4) != 0);
+        ptx::mma_commit(s_full + t);
+      };
+      bool ok = ptx::mbar_wait(k_full, 0) && ptx::mbar_wait(q_full, 0);
+      ptx::tc_fence_after();
+      if (ok)
+        for (int t = 0; t < ntiles; ++t) issue_s(t, 0);
+      for (int i = 0; i < nqb && ok; ++i) {
+        const int qs = i % kQS;
+        const uint64_t q0 = ptx::sw128_desc(aQ + qs * kQst, 2 * kBox, 1024);
+        for (int t = 0; t < ntiles && ok; ++t) {
+          ok = ptx::mbar_wait(p_full + t, i & 1);
+          ptx::tc_fence_after();
+          if (!ok) break;
+          const uint32_t tp = tS(t);
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+#pragma unroll
+            for (int kk = 0; kk < kQBlk / 16; ++kk)
+              ptx::mma_f16_ts(tA(t), tp + (kk >> 2) * 64 + p * 32 + (kk & 3) * 8, q0 + ((kk * 2048) >> 4), idPQ,
+                              (i | p | kk) != 0);
+          if (t == ntiles - 1) ptx::mma_commit(q_free + qs);
+          if (i + 1 < nqb) {
+            // S^T(t, i+1) overwrites P^T(t, i): the P^T q product above runs first
+            ok = ptx::mbar_wait(q_full + (i + 1) % kQS, ((i + 1) / kQS) & 1);
+            ptx::tc_fence_after();
+            if (ok) issue_s(t, i + 1);
+          } else {
+            ptx::mma_commit(o_done + t);
+          }
+        }
+      }
+    }
+  } else {
+    const int t = warp >> 2;
+    const int r = 32 * (warp & 3) + lane;   // key tile row / TMEM lane
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int c1 = kb + t * kTile + r;
+    if (t < ntiles) {
+      const float hb = (c1 < g.b1k) ? hbuf[(long long)zrow * g.b1k_pad + c1] + kColShift : 0.f;
+      const float2 sl2 = make_float2(g.sl2, g.sl2), hb2 = make_float2(hb, hb);
+      float2 beta2 = make_float2(0.f, 0.f);
+      bool ok = true;
+      for (int i = 0; i < nqb; ++i) {
+        const int qs = i % kQS;
+        ok = ok && ptx::mbar_wait(s_full + t, i & 1) && ptx::mbar_wait(q_full + qs, (i / kQS) & 1);
+        ptx::tc_fence_after();
+        const int valid = min(kQBlk, g.b1q - i * kQBlk);
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {  // queries 64 hh .. 64 hh + 63
+          uint32_t sr[64];
+          ptx::tmem_ld32(tS(t) + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sr));
+          ptx::tmem_ld32(tS(t) + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+          const float4* lv = reinterpret_cast<const float4*>(sL + qs * kQBlk + 64 * hh);
+          ptx::tmem_wait_ld();
+          uint32_t hi[32], lo[32];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float4 l4 = lv[e];
+            float2 x0 = fma2(make_float2(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1])), sl2, hb2);
+            float2 x1 =
+                fma2(make_float2(__uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3])), sl2, hb2);
+            x0 = sub2(x0, make_float2(l4.x, l4.y));
+            x1 = sub2(x1, make_float2(l4.z, l4.w));
+            float2 p0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
+            float2 p1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
+            if (valid < kQBlk) {  // only the last block of a ragged column
+              const int q0 = 64 * hh + 4 * e;
+              if (q0 >= valid) p0.x = 0.f;
+              if (q0 + 1 >= valid) p0.y = 0.f;
+              if (q0 + 2 >= valid) p1.x = 0.f;
+              if (q0 + 3 >= valid) p1.y = 0.f;
+            }
+            beta2 = add2(beta2, add2(p0, p1));
+            split2<TQ>(p0, hi[2 * e], lo[2 * e]);
+            split2<TQ>(p1, hi[2 * e + 1], lo[2 * e + 1]);
+          }
+          // P^T hi / lo of these 64 queries over the S^T columns just read
+          ptx::tmem_st32(tS(t) + lane_off + 64 * hh, hi);
+          ptx::tmem_st32(tS(t) + lane_off + 64 * hh + 32, lo);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(p_full + t);
+      }
+      ok = ok && ptx::mbar_wait(o_done + t, 0);
+      ptx::tc_fence_after();
+      const float inv = 1.f / (beta2.x + beta2.y);
+      float* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D;
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        ptx::tmem_ld32(tA(t) + lane_off + cc * 32, o);
+        ptx::tmem_wait_ld();
+        if (c1 < g.b1k && ok) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        }
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+}  // namespace tc
+}  // namespace monarch

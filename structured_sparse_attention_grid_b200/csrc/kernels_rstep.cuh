@@ -283,9 +283,9 @@ r_step_tc(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restri
   }
   const float i0 = 1.f / l0, i1 = 1.f / l1;
   if ((lane & 3) == 0) {
-    // h = -sum R ln R = ln l - ln2 * sum R (x - m)   (x in base-2 units)
-    if (r0 < g.b2) w.h[((long long)bh * g.b2 + r0) * g.b1k_pad + c1] = __logf(l0) - 0.6931471805599453f * x0 * i0;
-    if (r1 < g.b2) w.h[((long long)bh * g.b2 + r1) * g.b1k_pad + c1] = __logf(l1) - 0.6931471805599453f * x1 * i1;
+    // h in bits: -sum R log2 R = log2 l - sum R (x - m)   (x in base-2 units)
+    if (r0 < g.b2) w.h[((long long)bh * g.b2 + r0) * g.b1k_pad + c1] = log2f(l0) - x0 * i0;
+    if (r1 < g.b2) w.h[((long long)bh * g.b2 + r1) * g.b1k_pad + c1] = log2f(l1) - x1 * i1;
   }
   // ---- R as A fragments (K = c2), split hi + lo
   uint32_t rhi[4][4], rlo[4][4];

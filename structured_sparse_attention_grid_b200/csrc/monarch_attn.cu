@@ -19,7 +19,7 @@
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
 #include "kernels_rstep.cuh"
-#include "kernels_tc2.cuh"
+#include "kernels_l.cuh"
 
 using namespace monarch;
 
@@ -252,16 +252,16 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
 
   const CUtensorMapDataType dq =
       TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  v2::Maps maps;
+  tc::Maps maps;
   int rc;
   {
     const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
-    cuuint32_t box3[3] = {64, (cuuint32_t)v2::kBlk, 1};
+    cuuint32_t box3[3] = {64, (cuuint32_t)tc::kBlk, 1};
     cuuint64_t dq3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, rows};
     cuuint64_t sq3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1q * D * 2};
     cuuint64_t dk3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, 2 * rows};
     cuuint64_t sk3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1k * D * 2};
-    cuuint32_t box2[2] = {(cuuint32_t)v2::kBlk, 1};
+    cuuint32_t box2[2] = {(cuuint32_t)tc::kBlk, 1};
     cuuint64_t dh2[2] = {(cuuint64_t)g.b1k_pad, rows};
     cuuint64_t sh2[1] = {(cuuint64_t)g.b1k_pad * 4};
     cuuint64_t dl2[2] = {(cuuint64_t)g.b1q_pad, rows};
@@ -276,23 +276,23 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
       return rc;
   }
 
-  constexpr size_t smem_row = v2::l_row_smem<D, false>();
-  constexpr size_t smem_out = v2::l_row_smem<D, true>();
-  constexpr size_t smem_col = v2::l_col_smem<D>();
+  constexpr size_t smem_row = tc::row_smem<D, false>();
+  constexpr size_t smem_out = tc::row_smem<D, true>();
+  constexpr size_t smem_col = tc::col_smem<D>();
   const int mt = (g.b2 + 15) / 16, tpc = 4 / mt;
 
   static bool attrs_set = false;
   if (!attrs_set) {
     cudaError_t e;
-    if ((e = allow_smem(v2::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
-        (e = allow_smem(v2::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
-        (e = allow_smem(v2::l_col<TQ, D>, smem_col)) != cudaSuccess ||
+    if ((e = allow_smem(tc::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
+        (e = allow_smem(tc::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
+        (e = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
         (e = allow_smem(r_step_tc<TQ, D>, r_step_tc_smem<D>(64, 3))) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
     attrs_set = true;
   }
-  const dim3 grid_q((g.b1q + kTile - 1) / kTile, g.b2, g.BH);
-  const dim3 grid_k((g.b1k + kTile - 1) / kTile, g.b2, g.BH);
+  const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);  // two 128-row tiles per CTA
+  const dim3 grid_k((g.b1k + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
   const dim3 grid_r((g.b1k + tpc - 1) / tpc, g.BH);
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
@@ -303,7 +303,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
     } else {
       launch(MONARCH_PHASE_L_COL, st, [&] {
-        v2::l_col<TQ, D><<<grid_k, v2::kThreads, smem_col, st>>>(maps, w.h, w.qt, g);
+        tc::l_col<TQ, D><<<grid_k, tc::kThreads, smem_col, st>>>(maps, w.h, w.qt, g);
       });
     }
     const size_t smem_r = r_step_tc_smem<D>(g.b2, r_step_slots(mode, final_step));
@@ -312,11 +312,11 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
-        v2::l_row<TQ, TO, D, true><<<grid_q, v2::kThreads, smem_out, st>>>(out, maps, w.lse, g);
+        tc::l_row<TQ, TO, D, true><<<grid_q, tc::kThreads, smem_out, st>>>(out, maps, w.lse, g);
       });
     } else {
       launch(MONARCH_PHASE_L_ROW, st, [&] {
-        v2::l_row<TQ, TO, D, false><<<grid_q, v2::kThreads, smem_row, st>>>(out, maps, w.lse, g);
+        tc::l_row<TQ, TO, D, false><<<grid_q, tc::kThreads, smem_row, st>>>(out, maps, w.lse, g);
       });
     }
   }
