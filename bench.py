@@ -367,6 +367,21 @@ def run_reference(args, rank, world):
     }
 
 
+def profile_calls(args):
+    """A bare run of the workload for profiler captures: no timing, no bench line."""
+    import structured_sparse_attention_grid_b200 as m
+    w = WORKLOADS[args.workload]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    for _ in range(args.profile_calls):
+        m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    err = m.device_error()
+    print(f"profile case {w.name} B={w.B} heads={w.heads} calls={args.profile_calls} device_error={err}")
+    if err:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -375,7 +390,17 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiler cases)")
+    ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiler cases)")
+    ap.add_argument("--profile-calls", type=int, default=0,
+                    help="run this many forward calls of the workload and exit (for ncu); no timing")
     args = ap.parse_args()
+    if args.batch or args.heads:
+        import dataclasses
+        base = WORKLOADS[args.workload]
+        WORKLOADS[args.workload] = dataclasses.replace(base, B=args.batch or base.B, heads=args.heads or base.heads)
+    if args.profile_calls:
+        return profile_calls(args)
     if args.warmup < 3:
         args.warmup = 3
     world = int(os.environ.get("WORLD_SIZE", "1"))

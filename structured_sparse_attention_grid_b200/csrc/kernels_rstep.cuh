@@ -1,18 +1,25 @@
-// R step for bf16 / f16 inputs on the tensor cores (warp-level mma.sync
-// m16n8k16: the per-tile products are b2 x b2 x d with b2 <= 64, far below
-// the 128-row tcgen05 tile, so a warp owns 16 positions of one key tile).
+// R step for bf16 / f16 inputs (warp-level mma.sync m16n8k16: the per-tile
+// products are b2 x b2 x d with b2 <= 64, far below the 128-row tcgen05 tile,
+// so a warp owns 16 positions of one key tile).
 //
 // For key tile c1 and positions a2 (16 per warp):
 //   S[a2,c2] = s q~[c1,a2].k[c1,c2]      (q~ split hi+lo when it is computed)
 //   R = softmax_c2(S), h = entropy(R)
 //   k~[c1,a2] = sum_c2 R k[c1,c2]        (R split hi+lo; k~ stored as hi/lo planes)
 //   z[c1,a2]  = sum_c2 R v[c1,c2]        (final step; stored as f16 hi/lo planes)
-// k and v tiles are gathered from the grid layout straight into shared memory.
+//
+// The kernel is persistent and HBM-bound: one warp issues TMA loads into a
+// ring of shared-memory stages while four warps compute.  The grid-to-block
+// permutation is done by the TMA box itself: a 4-D map over (d, W, H, frames)
+// with box (64, tw, th, 1) lands one key tile as b2 consecutive rows in the
+// in-tile order c2 = (y mod th) * tw + x mod tw.  q~ rows (one per a2, stride
+// b1k*d) come through a 3-D map over the q~ buffer.
 #pragma once
 
 #include "common.cuh"
 #include "ptx.cuh"
 #include "kernels_tc.cuh"
+#include "tc_common.cuh"
 
 namespace monarch {
 
@@ -82,280 +89,335 @@ __device__ __forceinline__ void split_pair(float x, float y, uint32_t& hi, uint3
   lo = TcType<TQ>::pack(x - hx, y - hy);
 }
 
-template <int D>
-constexpr int r_step_tc_pitch() { return D + 8; }  // 16-bit elements per shared row (16-byte pad)
 
-// Gathered [rows][PITCH] tiles per key tile: k always, v in the final step,
-// the exact query rows in the first step.
-__host__ __device__ inline int r_step_slots(int mode, int final_step) {
-  return 1 + (final_step ? 1 : 0) + (mode != QT_BUFFER ? 1 : 0);
+// Tensor maps of one R step (128-byte swizzle everywhere).
+struct RMaps {
+  CUtensorMap q;    // queries   {d, W, H, BH*T},    box {64, tw, th, 1}
+  CUtensorMap k;    // keys      {d, W, H, BH*Tk},   box {64, tw, th, 1}
+  CUtensorMap v;    // values    {d, W, H, BH*Tk},   box {64, tw, th, 1}
+  CUtensorMap qt;   // q~ (f32)  {d, b1k, BH*b2},    box {32, 1, b2}
+};
+
+// Shared-memory layout of one key tile in a stage.  Every region is a stack
+// of [r8 rows][128 B] swizzled boxes (r8 = b2 rounded up to 8, so each box
+// starts on a 1024-byte boundary):
+//   A  q~ as d/32 f32 boxes (step with a q~ buffer); afterwards this warp's
+//      output stage, [plane][d/64][r8][128 B] of 16-bit values
+//   K  keys, d/64 boxes;  V values (final step);  X exact query rows (first step)
+struct RStepLayout {
+  int r8, tp, offK, offV, offX, tile_bytes, stage_bytes;
+};
+
+__host__ __device__ inline RStepLayout r_step_layout(int b2, int d, int mode, int final_step) {
+  RStepLayout L;
+  L.r8 = (b2 + 7) & ~7;
+  L.tp = 4 / ((b2 + 15) >> 4);
+  L.offK = L.r8 * d * 4;
+  L.offV = L.offK + L.r8 * d * 2;
+  L.offX = L.offV + (final_step ? L.r8 * d * 2 : 0);
+  L.tile_bytes = L.offX + (mode != QT_BUFFER ? L.r8 * d * 2 : 0);
+  L.stage_bytes = L.tp * L.tile_bytes;
+  return L;
 }
 
-// Shared memory of r_step_tc: the gathered tiles plus a per-warp
-// [2 planes][16 rows][PITCH] output stage and the row-offset table.
-template <int D>
-size_t r_step_tc_smem(int b2, int slots) {
-  const int mt = (b2 + 15) / 16, rows = 16 * mt, tpc = 4 / mt;
-  return (size_t)tpc * slots * rows * r_step_tc_pitch<D>() * 2 + 4 * 2 * 16 * r_step_tc_pitch<D>() * 2 + 64 * 4;
-}
+constexpr int kRThreads = 160;           // 4 compute warps + 1 TMA warp
+constexpr int kRMaxStages = 4;
+constexpr int kRFixedSmem = 1024 + 128 + 2 * kRMaxStages * 8;  // alignment slack, zero row, barriers
 
-// grid (ceil(b1k / tiles_per_cta), BH), block 128 (4 warps; a warp owns 16
-// positions of one key tile), tiles_per_cta = 4 / ceil(b2/16).
+// Byte offset of 16-byte chunk `ch` of row `r` in a [rows][128 B] swizzled box.
+__device__ __forceinline__ uint32_t swz(int r, int ch) { return (uint32_t)(r * 128 + ((ch ^ (r & 7)) << 4)); }
+
+// grid: persistent (a multiple of the SM count); block kRThreads.  A work
+// item is tp consecutive key tiles of one head; CTA b takes items b,
+// b + gridDim.x, ...
 template <typename TQ, int D>
-__global__ void __launch_bounds__(128, 3)
-r_step_tc(const TQ* __restrict__ q, const TQ* __restrict__ k, const TQ* __restrict__ v, Work w,
-          TcPlanes<TQ> out, Geo g, int mode, int final_step) {
-  constexpr int PITCH = r_step_tc_pitch<D>();
+__global__ void __launch_bounds__(kRThreads, 2)
+r_step_tc(const __grid_constant__ RMaps maps, Work w, TcPlanes<TQ> out, Geo g, int mode, int final_step,
+          int stages) {
   constexpr int CH = D / 8;     // 16-byte chunks per row
   constexpr int bf16 = TcType<TQ>::kBf16;
-  extern __shared__ uint8_t smem_raw[];
-  TQ* smem = reinterpret_cast<TQ*>(smem_raw);
-  const int mt = (g.b2 + 15) >> 4;
-  const int rows = mt * 16;
-  const int tpc = 4 / mt;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const RStepLayout L = r_step_layout(g.b2, D, mode, final_step);
+  uint8_t* zero = base + stages * L.stage_bytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(zero + 128);
+  uint64_t* empty = full + kRMaxStages;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
-  const int slots = r_step_slots(mode, final_step);
-  const int slot_v = 1, slot_x = final_step ? 2 : 1;
-  TQ* stage = smem + tpc * slots * rows * PITCH + warp * 2 * 16 * PITCH;  // this warp's output stage
-  int* roff = reinterpret_cast<int*>(smem + tpc * slots * rows * PITCH + 4 * 2 * 16 * PITCH);
-  const TQ* kh = k + (long long)bh * g.Nk * D;
-  const TQ* vh = v + (long long)bh * g.Nk * D;
-  const TQ* qh = q + (long long)bh * g.Nq * D;
+  const int n_groups = (g.b1k + L.tp - 1) / L.tp;
+  const int n_items = g.BH * n_groups;
 
-  // token offset of position c2 inside its tile: (c2 / tw) * W + c2 % tw
-  if (tid < g.b2) roff[tid] = (tid / g.tw) * g.W + tid % g.tw;
+  if (tid < 32) reinterpret_cast<uint32_t*>(zero)[tid] = 0u;
+  if (tid == 0) {
+    for (int s = 0; s < stages; ++s) {
+      ptx::mbar_init(full + s, 1);
+      ptx::mbar_init(empty + s, 4);
+    }
+    ptx::fence_mbar_init();
+  }
   __syncthreads();
 
-  // ---- gather k, v (final step) and the exact q rows (first step) of each tile
-  for (int tt = 0; tt < tpc; ++tt) {
-    const int c1 = blockIdx.x * tpc + tt;
-    if (c1 >= g.b1k) break;
-    const bool exact_q = mode != QT_BUFFER && !(mode == QT_KVINIT && c1 < g.off);
-    const int cq = mode == QT_KVINIT ? c1 - g.off : c1;
-    for (int mat = 0; mat < 3; ++mat) {
-      if ((mat == 1 && !final_step) || (mat == 2 && !exact_q)) continue;
-      const int ct = mat == 2 ? cq : c1;
-      const long long tbase = token_of(g, ct, 0);
-      const TQ* src0 = mat == 0 ? kh : (mat == 1 ? vh : qh);
-      TQ* dst0 = smem + (tt * slots + (mat == 0 ? 0 : mat == 1 ? slot_v : slot_x)) * rows * PITCH;
-      for (int row = tid / CH; row < rows; row += 128 / CH) {
-        const int ch = tid % CH;
-        const bool valid = row < g.b2;
-        const TQ* src = src0 + (valid ? (tbase + roff[row]) * D + ch * 8 : 0);
-        ptx::cp_async_16(ptx::smem_u32(dst0 + row * PITCH + ch * 8), src, valid ? 16u : 0u);
+  if (warp == 4) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      ptx::prefetch_tmap(&maps.k);
+      if (mode == QT_BUFFER) ptx::prefetch_tmap(&maps.qt);
+      int it = 0;
+      for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+        const int s = it % stages;
+        if (it >= stages && !ptx::mbar_wait(empty + s, ((it / stages) - 1) & 1)) break;
+        const int bh = item / n_groups, c1_0 = (item - bh * n_groups) * L.tp;
+        const int ntile = min(L.tp, g.b1k - c1_0);
+        uint32_t bytes = 0;
+        for (int tt = 0; tt < ntile; ++tt) {
+          const int c1 = c1_0 + tt;
+          const bool exact_q = mode != QT_BUFFER && !(mode == QT_KVINIT && c1 < g.off);
+          bytes += g.b2 * D * ((mode == QT_BUFFER ? 4 : 0) + 2 + (final_step ? 2 : 0) + (exact_q ? 2 : 0));
+        }
+        ptx::mbar_expect_tx(full + s, bytes);
+        for (int tt = 0; tt < ntile; ++tt) {
+          const int c1 = c1_0 + tt;
+          uint8_t* tb = base + s * L.stage_bytes + tt * L.tile_bytes;
+          const int t = c1 / g.P, rem = c1 - t * g.P, ty = rem / g.ntx, tx = rem - ty * g.ntx;
+          if (mode == QT_BUFFER)
+            for (int qq = 0; qq < D / 32; ++qq)
+              ptx::tma_load_3d(tb + qq * L.r8 * 128, &maps.qt, full + s, qq * 32, c1, bh * g.b2);
+          for (int hf = 0; hf < D / 64; ++hf) {
+            ptx::tma_load_4d(tb + L.offK + hf * L.r8 * 128, &maps.k, full + s, hf * 64, tx * g.tw, ty * g.th,
+                             bh * g.Tk + t);
+            if (final_step)
+              ptx::tma_load_4d(tb + L.offV + hf * L.r8 * 128, &maps.v, full + s, hf * 64, tx * g.tw, ty * g.th,
+                               bh * g.Tk + t);
+          }
+          const bool exact_q = mode != QT_BUFFER && !(mode == QT_KVINIT && c1 < g.off);
+          if (exact_q) {
+            const int tq = t - (g.Tk - g.T);   // the aligned query frame (== t without a cache)
+            for (int hf = 0; hf < D / 64; ++hf)
+              ptx::tma_load_4d(tb + L.offX + hf * L.r8 * 128, &maps.q, full + s, hf * 64, tx * g.tw, ty * g.th,
+                               bh * g.T + tq);
+          }
+        }
       }
     }
+    return;
   }
-  ptx::cp_async_commit();
 
+  // ------------------------------------------------------------ compute warps
+  const int mt = (g.b2 + 15) >> 4;
   const int tt = warp / mt, mi = warp % mt;
-  const int c1 = blockIdx.x * tpc + tt;
-  const bool active = tt < tpc && c1 < g.b1k;
-  const bool exact_q = mode != QT_BUFFER && !(mode == QT_KVINIT && c1 < g.off);
   const int r0 = mi * 16 + (lane >> 2), r1 = r0 + 8;  // positions a2 of this thread's rows
   const int qc = 2 * (lane & 3);
   const int lr = lane & 7, lm = lane >> 3;
+  const int nt = 2 * mt;                               // n-tiles of 8 over c2
+  const uint32_t zaddr = ptx::smem_u32(zero);
+  const uint32_t box = (uint32_t)L.r8 * 128;          // bytes of one swizzled box
 
-  // ---- A fragments of a computed q~ (fp32 rows, split hi + lo); issued before the gather completes
-  uint32_t ahi[D / 16][4], alo[D / 16][4];
-  if (active && !exact_q) {
-    const float* qr0 = nullptr;
-    const float* qr1 = nullptr;
-    if (mode == QT_BUFFER) {
-      if (r0 < g.b2) qr0 = w.qt + (((long long)bh * g.b2 + r0) * g.b1k + c1) * D;
-      if (r1 < g.b2) qr1 = w.qt + (((long long)bh * g.b2 + r1) * g.b1k + c1) * D;
-    } else {
-      if (r0 < g.b2) qr0 = w.qbar + ((long long)bh * g.b2 + r0) * D;
-      if (r1 < g.b2) qr1 = w.qbar + ((long long)bh * g.b2 + r1) * D;
-    }
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int cA = ks * 16 + qc, cB = cA + 8;
-      const float2 v0 = qr0 ? *reinterpret_cast<const float2*>(qr0 + cA) : make_float2(0.f, 0.f);
-      const float2 v1 = qr1 ? *reinterpret_cast<const float2*>(qr1 + cA) : make_float2(0.f, 0.f);
-      const float2 v2 = qr0 ? *reinterpret_cast<const float2*>(qr0 + cB) : make_float2(0.f, 0.f);
-      const float2 v3 = qr1 ? *reinterpret_cast<const float2*>(qr1 + cB) : make_float2(0.f, 0.f);
-      split_pair<TQ>(v0.x, v0.y, ahi[ks][0], alo[ks][0]);
-      split_pair<TQ>(v1.x, v1.y, ahi[ks][1], alo[ks][1]);
-      split_pair<TQ>(v2.x, v2.y, ahi[ks][2], alo[ks][2]);
-      split_pair<TQ>(v3.x, v3.y, ahi[ks][3], alo[ks][3]);
-    }
-  }
-  ptx::cp_async_wait<0>();
-  __syncthreads();
+  int it = 0;
+  for (int item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
+    const int s = it % stages;
+    if (!ptx::mbar_wait(full + s, (it / stages) & 1)) break;
+    const int bh = item / n_groups;
+    const int c1 = (item - bh * n_groups) * L.tp + tt;
+    uint8_t* tb = base + s * L.stage_bytes + tt * L.tile_bytes;
+    if (tt < L.tp && c1 < g.b1k) {
+      const bool exact_q = mode != QT_BUFFER && !(mode == QT_KVINIT && c1 < g.off);
+      const int cq = mode == QT_KVINIT ? c1 - g.off : c1;
+      const uint32_t aA = ptx::smem_u32(tb), aK = aA + L.offK, aV = aA + L.offV, aX = aA + L.offX;
+      // address of the 16-byte chunk holding column col (a multiple of 8) of row `row` of a
+      // 16-bit region; rows past b2 read the zero row
+      auto rowaddr = [&](uint32_t region, int row, int col) -> uint32_t {
+        return row < g.b2 ? region + (col >> 6) * box + swz(row, (col >> 3) & 7) : zaddr;
+      };
 
-  // ---- first step: write the exact query rows in block-major order (coalesced)
-  for (int t2 = 0; t2 < tpc; ++t2) {
-    const int cc1 = blockIdx.x * tpc + t2;
-    if (cc1 >= g.b1k) break;
-    if (mode == QT_BUFFER || (mode == QT_KVINIT && cc1 < g.off)) continue;
-    const int cq = mode == QT_KVINIT ? cc1 - g.off : cc1;
-    const TQ* src0 = smem + (t2 * slots + slot_x) * rows * PITCH;
-    TQ* qb = reinterpret_cast<TQ*>(w.qb);
-    for (int i = tid; i < g.b2 * CH; i += 128) {
-      const int row = i / CH, ch = i % CH;
-      *reinterpret_cast<uint4*>(qb + (((long long)bh * g.b2 + row) * g.b1q + cq) * D + ch * 8) =
-          *reinterpret_cast<const uint4*>(src0 + row * PITCH + ch * 8);
-    }
-  }
-  if (!active) return;
-
-  const uint32_t aK = ptx::smem_u32(smem + (tt * slots + 0) * rows * PITCH);
-  const uint32_t aV = ptx::smem_u32(smem + (tt * slots + slot_v) * rows * PITCH);
-  const uint32_t aX = ptx::smem_u32(smem + (tt * slots + slot_x) * rows * PITCH);
-  if (exact_q) {
-    // A fragments straight from the gathered exact rows: matrices (rows 0-7 | 8-15) x (k lo | k hi)
-#pragma unroll
-    for (int ks = 0; ks < D / 16; ++ks) {
-      const int row = mi * 16 + (lm & 1) * 8 + lr;
-      const int col = ks * 16 + (lm >> 1) * 8;
-      rs::ldsm_x4(aX + (row * PITCH + col) * 2, ahi[ks][0], ahi[ks][1], ahi[ks][2], ahi[ks][3]);
-    }
-  }
-  const int nt = rows / 8;  // n-tiles over c2 (even)
-
-  // ---- S = q~ k^T
-  float s[8][4];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-  for (int ks = 0; ks < D / 16; ++ks) {
-#pragma unroll
-    for (int j = 0; j < 8; j += 2) {
-      if (j < nt) {
-        const int row = (j + (lm >> 1)) * 8 + lr;
-        const int col = ks * 16 + (lm & 1) * 8;
-        uint32_t b0, b1, b2, b3;
-        rs::ldsm_x4(aK + (row * PITCH + col) * 2, b0, b1, b2, b3);
-        rs::mma16816(s[j], ahi[ks], b0, b1, bf16);
-        rs::mma16816(s[j + 1], ahi[ks], b2, b3, bf16);
-        if (!exact_q) {
-          rs::mma16816(s[j], alo[ks], b0, b1, bf16);
-          rs::mma16816(s[j + 1], alo[ks], b2, b3, bf16);
+      // ---- first step: the exact query rows of this tile, copied block-major
+      if (exact_q) {
+        TQ* qb = reinterpret_cast<TQ*>(w.qb);
+        for (int i = mi * 32 + lane; i < g.b2 * CH; i += mt * 32) {
+          const int row = i / CH, ch = i - row * CH;
+          *reinterpret_cast<uint4*>(qb + (((long long)bh * g.b2 + row) * g.b1q + cq) * D + ch * 8) =
+              *reinterpret_cast<const uint4*>(tb + L.offX + (ch >> 3) * box + swz(row, ch & 7));
         }
       }
-    }
-  }
 
-  // ---- softmax over c2 for rows r0 (s[.][0..1]) and r1 (s[.][2..3])
-  float m0 = -INFINITY, m1 = -INFINITY;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const bool colok = j * 8 + qc + e < g.b2;
-        s[j][e] = colok ? s[j][e] * g.sl2 : -INFINITY;
-        s[j][2 + e] = colok ? s[j][2 + e] * g.sl2 : -INFINITY;
-        m0 = fmaxf(m0, s[j][e]);
-        m1 = fmaxf(m1, s[j][2 + e]);
-      }
-    }
-  }
-  m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-  m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
-  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-  m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
-  float l0 = 0.f, l1 = 0.f, x0 = 0.f, x1 = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    if (j < nt) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float d0 = s[j][e] - m0, d1 = s[j][2 + e] - m1;
-        const float p0 = ptx::ex2(d0), p1 = ptx::ex2(d1);
-        s[j][e] = p0;
-        s[j][2 + e] = p1;
-        l0 += p0;
-        l1 += p1;
-        x0 += p0 > 0.f ? p0 * d0 : 0.f;
-        x1 += p1 > 0.f ? p1 * d1 : 0.f;
-      }
-    }
-  }
-#pragma unroll
-  for (int o = 1; o <= 2; o <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, o);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, o);
-    x0 += __shfl_xor_sync(0xffffffffu, x0, o);
-    x1 += __shfl_xor_sync(0xffffffffu, x1, o);
-  }
-  const float i0 = 1.f / l0, i1 = 1.f / l1;
-  if ((lane & 3) == 0) {
-    // h in bits: -sum R log2 R = log2 l - sum R (x - m)   (x in base-2 units)
-    if (r0 < g.b2) w.h[((long long)bh * g.b2 + r0) * g.b1k_pad + c1] = log2f(l0) - x0 * i0;
-    if (r1 < g.b2) w.h[((long long)bh * g.b2 + r1) * g.b1k_pad + c1] = log2f(l1) - x1 * i1;
-  }
-  // ---- R as A fragments (K = c2), split hi + lo
-  uint32_t rhi[4][4], rlo[4][4];
-#pragma unroll
-  for (int kq = 0; kq < 4; ++kq) {
-    if (2 * kq < nt) {
-      split_pair<TQ>(s[2 * kq][0] * i0, s[2 * kq][1] * i0, rhi[kq][0], rlo[kq][0]);
-      split_pair<TQ>(s[2 * kq][2] * i1, s[2 * kq][3] * i1, rhi[kq][1], rlo[kq][1]);
-      split_pair<TQ>(s[2 * kq + 1][0] * i0, s[2 * kq + 1][1] * i0, rhi[kq][2], rlo[kq][2]);
-      split_pair<TQ>(s[2 * kq + 1][2] * i1, s[2 * kq + 1][3] * i1, rhi[kq][3], rlo[kq][3]);
-    }
-  }
+      // element (r, c) of the f32 q~ boxes: box c/32, chunk (c mod 32)/4
+      auto qrow = [&](int r, int c) -> float2 {
+        if (r >= g.b2) return make_float2(0.f, 0.f);
+        if (mode == QT_BUFFER)
+          return *reinterpret_cast<const float2*>(tb + (c >> 5) * box + swz(r, (c & 31) >> 2) + (c & 3) * 4);
+        return *reinterpret_cast<const float2*>(w.qbar + ((long long)bh * g.b2 + r) * D + c);
+      };
 
-  // ---- k~ = R k and z = R v, staged per warp, then written as coalesced 16-byte rows
-  for (int which = 0; which < (final_step ? 2 : 1); ++which) {
-    const uint32_t aB = which ? aV : aK;
-    float acc[D / 8][4];
+      // ---- S = q~ k^T; the A fragments of each k-step (q~ rows split hi + lo, or
+      // the exact query rows) are built just before use
+      float sc[8][4];
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      for (int j = 0; j < 8; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
 #pragma unroll
-    for (int kq = 0; kq < 4; ++kq) {
-      if (2 * kq < nt) {
+      for (int ks = 0; ks < D / 16; ++ks) {
+        uint32_t ahi[4], alo[4];
+        if (exact_q) {
+          rs::ldsm_x4(rowaddr(aX, mi * 16 + (lm & 1) * 8 + lr, ks * 16 + (lm >> 1) * 8), ahi[0], ahi[1], ahi[2],
+                      ahi[3]);
+        } else {
+          const int cA = ks * 16 + qc, cB = cA + 8;
+          const float2 v0 = qrow(r0, cA), v1 = qrow(r1, cA), v2 = qrow(r0, cB), v3 = qrow(r1, cB);
+          split_pair<TQ>(v0.x, v0.y, ahi[0], alo[0]);
+          split_pair<TQ>(v1.x, v1.y, ahi[1], alo[1]);
+          split_pair<TQ>(v2.x, v2.y, ahi[2], alo[2]);
+          split_pair<TQ>(v3.x, v3.y, ahi[3], alo[3]);
+        }
 #pragma unroll
-        for (int j = 0; j < D / 8; j += 2) {
-          const int row = kq * 16 + (lm & 1) * 8 + lr;
-          const int col = (j + (lm >> 1)) * 8;
-          uint32_t b0, b1, b2, b3;
-          rs::ldsm_x4_t(aB + (row * PITCH + col) * 2, b0, b1, b2, b3);
-          rs::mma16816(acc[j], rhi[kq], b0, b1, bf16);
-          rs::mma16816(acc[j], rlo[kq], b0, b1, bf16);
-          rs::mma16816(acc[j + 1], rhi[kq], b2, b3, bf16);
-          rs::mma16816(acc[j + 1], rlo[kq], b2, b3, bf16);
+        for (int j = 0; j < 8; j += 2) {
+          if (j < nt) {
+            uint32_t b0, b1, b2, b3;
+            rs::ldsm_x4(rowaddr(aK, (j + (lm >> 1)) * 8 + lr, ks * 16 + (lm & 1) * 8), b0, b1, b2, b3);
+            rs::mma16816(sc[j], ahi, b0, b1, bf16);
+            rs::mma16816(sc[j + 1], ahi, b2, b3, bf16);
+            if (!exact_q) {
+              rs::mma16816(sc[j], alo, b0, b1, bf16);
+              rs::mma16816(sc[j + 1], alo, b2, b3, bf16);
+            }
+          }
         }
       }
-    }
-    __syncwarp();
-    // stage rows (lane/4) and (lane/4 + 8) of this warp's 16, hi plane then lo plane
+
+      // ---- softmax over c2 for rows r0 (sc[.][0..1]) and r1 (sc[.][2..3])
+      float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-    for (int j = 0; j < D / 8; ++j) {
-      uint32_t h0, l0w, h1, l1w;
-      if (which == 0) {
-        split_pair<TQ>(acc[j][0], acc[j][1], h0, l0w);
-        split_pair<TQ>(acc[j][2], acc[j][3], h1, l1w);
-      } else {
-        split_pair<__half>(acc[j][0], acc[j][1], h0, l0w);
-        split_pair<__half>(acc[j][2], acc[j][3], h1, l1w);
-      }
-      const int col = j * 8 + qc;
-      const int ra = lane >> 2, rb = ra + 8;
-      *reinterpret_cast<uint32_t*>(stage + ra * PITCH + col) = h0;
-      *reinterpret_cast<uint32_t*>(stage + rb * PITCH + col) = h1;
-      *reinterpret_cast<uint32_t*>(stage + (16 + ra) * PITCH + col) = l0w;
-      *reinterpret_cast<uint32_t*>(stage + (16 + rb) * PITCH + col) = l1w;
-    }
-    __syncwarp();
-    uint16_t* gbase = which ? reinterpret_cast<uint16_t*>(out.z_hi) : reinterpret_cast<uint16_t*>(out.kt_hi);
+      for (int j = 0; j < 8; ++j) {
+        if (j < nt) {
 #pragma unroll
-    for (int it = 0; it < (2 * 16 * CH) / 32; ++it) {
-      const int idx = it * 32 + lane;
-      const int plane = idx / (16 * CH);
-      const int row = (idx / CH) % 16;
-      const int ch = idx % CH;
-      const int a2 = mi * 16 + row;
-      if (a2 < g.b2) {
-        const long long o = (((long long)bh * g.b2 + a2) * g.b1k + c1) * D + ch * 8;
-        *reinterpret_cast<uint4*>(gbase + plane * out.plane + o) =
-            *reinterpret_cast<const uint4*>(stage + (plane * 16 + row) * PITCH + ch * 8);
+          for (int e = 0; e < 2; ++e) {
+            const bool colok = j * 8 + qc + e < g.b2;
+            sc[j][e] = colok ? sc[j][e] * g.sl2 : -INFINITY;
+            sc[j][2 + e] = colok ? sc[j][2 + e] * g.sl2 : -INFINITY;
+            m0 = fmaxf(m0, sc[j][e]);
+            m1 = fmaxf(m1, sc[j][2 + e]);
+          }
+        }
+      }
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 2));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 2));
+      float l0 = 0.f, l1 = 0.f, x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < nt) {
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float d0 = sc[j][e] - m0, d1 = sc[j][2 + e] - m1;
+            const float p0 = ptx::ex2(d0), p1 = ptx::ex2(d1);
+            sc[j][e] = p0;
+            sc[j][2 + e] = p1;
+            l0 += p0;
+            l1 += p1;
+            x0 += p0 > 0.f ? p0 * d0 : 0.f;
+            x1 += p1 > 0.f ? p1 * d1 : 0.f;
+          }
+        }
+      }
+#pragma unroll
+      for (int o = 1; o <= 2; o <<= 1) {
+        l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+        l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        x0 += __shfl_xor_sync(0xffffffffu, x0, o);
+        x1 += __shfl_xor_sync(0xffffffffu, x1, o);
+      }
+      const float i0 = 1.f / l0, i1 = 1.f / l1;
+      if ((lane & 3) == 0) {
+        // h in bits: -sum R log2 R = log2 l - sum R (x - m)   (x in base-2 units)
+        if (r0 < g.b2) w.h[((long long)bh * g.b2 + r0) * g.b1k_pad + c1] = log2f(l0) - x0 * i0;
+        if (r1 < g.b2) w.h[((long long)bh * g.b2 + r1) * g.b1k_pad + c1] = log2f(l1) - x1 * i1;
+      }
+      // ---- R as A fragments (K = c2), split hi + lo
+      uint32_t rhi[4][4], rlo[4][4];
+#pragma unroll
+      for (int kq = 0; kq < 4; ++kq) {
+        if (2 * kq < nt) {
+          split_pair<TQ>(sc[2 * kq][0] * i0, sc[2 * kq][1] * i0, rhi[kq][0], rlo[kq][0]);
+          split_pair<TQ>(sc[2 * kq][2] * i1, sc[2 * kq][3] * i1, rhi[kq][1], rlo[kq][1]);
+          split_pair<TQ>(sc[2 * kq + 1][0] * i0, sc[2 * kq + 1][1] * i0, rhi[kq][2], rlo[kq][2]);
+          split_pair<TQ>(sc[2 * kq + 1][2] * i1, sc[2 * kq + 1][3] * i1, rhi[kq][3], rlo[kq][3]);
+        }
+      }
+      // this warp's q~ rows are in registers: its rows of region A become the output stage
+      __syncwarp();
+
+      // ---- k~ = R k and z = R v, staged in region A, written as 16-byte rows
+      for (int which = 0; which < (final_step ? 2 : 1); ++which) {
+        const uint32_t aB = which ? aV : aK;
+        const uint32_t lo_plane = (D / 64) * box;
+#pragma unroll 1
+        for (int hf = 0; hf < D / 64; ++hf) {  // 64 output columns at a time
+          float acc[8][4];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+#pragma unroll
+          for (int kq = 0; kq < 4; ++kq) {
+            if (2 * kq < nt) {
+#pragma unroll
+              for (int j = 0; j < 8; j += 2) {
+                uint32_t b0, b1, b2, b3;
+                rs::ldsm_x4_t(rowaddr(aB, kq * 16 + (lm & 1) * 8 + lr, hf * 64 + (j + (lm >> 1)) * 8), b0, b1, b2,
+                              b3);
+                rs::mma16816(acc[j], rhi[kq], b0, b1, bf16);
+                rs::mma16816(acc[j], rlo[kq], b0, b1, bf16);
+                rs::mma16816(acc[j + 1], rhi[kq], b2, b3, bf16);
+                rs::mma16816(acc[j + 1], rlo[kq], b2, b3, bf16);
+              }
+            }
+          }
+          // stage rows r0, r1: [plane][d/64][r8][128 B]
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            uint32_t h0, l0w, h1, l1w;
+            if (which == 0) {
+              split_pair<TQ>(acc[j][0], acc[j][1], h0, l0w);
+              split_pair<TQ>(acc[j][2], acc[j][3], h1, l1w);
+            } else {
+              split_pair<__half>(acc[j][0], acc[j][1], h0, l0w);
+              split_pair<__half>(acc[j][2], acc[j][3], h1, l1w);
+            }
+            const int ch = j, cb = qc * 2;  // chunk within the 128-byte row, byte within the chunk
+            const uint32_t o0 = hf * box + swz(r0, ch) + cb;
+            const uint32_t o1 = hf * box + swz(r1, ch) + cb;
+            if (r0 < g.b2) {
+              *reinterpret_cast<uint32_t*>(tb + o0) = h0;
+              *reinterpret_cast<uint32_t*>(tb + lo_plane + o0) = l0w;
+            }
+            if (r1 < g.b2) {
+              *reinterpret_cast<uint32_t*>(tb + o1) = h1;
+              *reinterpret_cast<uint32_t*>(tb + lo_plane + o1) = l1w;
+            }
+          }
+        }
+        __syncwarp();
+        uint16_t* gbase = which ? reinterpret_cast<uint16_t*>(out.z_hi) : reinterpret_cast<uint16_t*>(out.kt_hi);
+#pragma unroll
+        for (int k = 0; k < (2 * 16 * CH) / 32; ++k) {
+          const int idx = k * 32 + lane;
+          const int plane = idx / (16 * CH);
+          const int row = (idx / CH) % 16;
+          const int ch = idx % CH;
+          const int a2 = mi * 16 + row;
+          if (a2 < g.b2) {
+            const long long o = (((long long)bh * g.b2 + a2) * g.b1k + c1) * D + ch * 8;
+            *reinterpret_cast<uint4*>(gbase + plane * out.plane + o) = *reinterpret_cast<const uint4*>(
+                tb + (plane * (D / 64) + (ch >> 3)) * box + swz(a2, ch & 7));
+          }
+        }
+        __syncwarp();
       }
     }
+    // every read of this stage by this warp is done
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(empty + s);
   }
+}
+
+// Shared memory of one r_step_tc launch with `stages` stages.
+inline size_t r_step_smem(const RStepLayout& L, int stages) {
+  return (size_t)stages * L.stage_bytes + kRFixedSmem;
 }
 
 }  // namespace monarch

@@ -40,7 +40,6 @@ template <> struct TcType<__half> {
 };
 
 constexpr int kTile = 128;          // rows of every tensor-core tile
-constexpr int kHalfBytes = 16384;   // one [128 rows][128 B] swizzled half
 constexpr float kColShift = 15.f;   // L^T q: L scaled by 2^15 (the ratio is unchanged)
 constexpr float kLazyRescale = 8.f; // row pass: shift moves only when the max grows by > 2^8
 

@@ -1,6 +1,7 @@
 // Host side of the Monarch video-attention forward: argument validation,
 // geometry, workspace layout and the launch sequence of one call.  Every
 // step of the computation runs in this library's kernels.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -222,7 +223,7 @@ int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int ran
              const cuuint64_t* strides, const cuuint32_t* box, CUtensorMapSwizzle swz) {
   auto enc = tensor_map_encoder();
   if (!enc) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled is not available");
-  cuuint32_t estr[3] = {1, 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   CUresult r = enc(map, dt, rank, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MONARCH_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -275,11 +276,31 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
                        CU_TENSOR_MAP_SWIZZLE_NONE)))
       return rc;
   }
+  // R-step maps: the key / value / query grids as (d, W, H, frames) with one
+  // tile per box, and the q~ buffer as (d, b1k, BH*b2) with one key tile per box
+  RMaps rmaps;
+  {
+    cuuint32_t box4[4] = {64, (cuuint32_t)g.tw, (cuuint32_t)g.th, 1};
+    cuuint64_t dk4[4] = {(cuuint64_t)D, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH * g.Tk};
+    cuuint64_t dq4[4] = {(cuuint64_t)D, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH * g.T};
+    cuuint64_t s4[3] = {(cuuint64_t)D * 2, (cuuint64_t)g.W * D * 2, (cuuint64_t)g.H * g.W * D * 2};
+    cuuint32_t boxt[3] = {32, 1, (cuuint32_t)g.b2};
+    cuuint64_t dt3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, (cuuint64_t)g.BH * g.b2};
+    cuuint64_t st3[2] = {(cuuint64_t)D * 4, (cuuint64_t)g.b1k * D * 4};
+    if ((rc = make_map(&rmaps.q, q, dq, 4, dq4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.k, k, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.v, v, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.qt, w.qt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dt3, st3, boxt,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+  }
 
   constexpr size_t smem_row = tc::row_smem<D, false>();
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_col = tc::col_smem<D>();
-  const int mt = (g.b2 + 15) / 16, tpc = 4 / mt;
+  int dev = 0, sms = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
 
   static bool attrs_set = false;
   if (!attrs_set) {
@@ -287,13 +308,12 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     if ((e = allow_smem(tc::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
         (e = allow_smem(tc::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
         (e = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc<TQ, D>, r_step_tc_smem<D>(64, 3))) != cudaSuccess)
+        (e = allow_smem(r_step_tc<TQ, D>, tc::kMaxSmem)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
     attrs_set = true;
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);  // two 128-row tiles per CTA
   const dim3 grid_k((g.b1k + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
-  const dim3 grid_r((g.b1k + tpc - 1) / tpc, g.BH);
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
     int mode = QT_BUFFER;
@@ -306,9 +326,16 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         tc::l_col<TQ, D><<<grid_k, tc::kThreads, smem_col, st>>>(maps, w.h, w.qt, g);
       });
     }
-    const size_t smem_r = r_step_tc_smem<D>(g.b2, r_step_slots(mode, final_step));
+    // persistent R step: a ring of stages within ~113 KB so that two CTAs share an SM
+    const RStepLayout rl = r_step_layout(g.b2, D, mode, final_step);
+    const int stages = std::max(2, std::min(kRMaxStages, (115712 - kRFixedSmem) / rl.stage_bytes));
+    const size_t smem_r = r_step_smem(rl, stages);
+    int occ = 1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, r_step_tc<TQ, D>, kRThreads, smem_r);
+    const long long items = (long long)g.BH * ((g.b1k + rl.tp - 1) / rl.tp);
+    const int grid_r = (int)std::min<long long>(items, (long long)std::max(occ, 1) * sms);
     launch(MONARCH_PHASE_R_STEP, st, [&] {
-      r_step_tc<TQ, D><<<grid_r, 128, smem_r, st>>>(q, k, v, w, planes, g, mode, final_step);
+      r_step_tc<TQ, D><<<grid_r, kRThreads, smem_r, st>>>(rmaps, w, planes, g, mode, final_step, stages);
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {

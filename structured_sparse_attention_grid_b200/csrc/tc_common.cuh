@@ -48,42 +48,11 @@ __device__ __forceinline__ void split2(float2 p, uint32_t& hi, uint32_t& lo) {
   lo = TcType<TQ>::pack(r.x, r.y);
 }
 
-__device__ __forceinline__ void named_bar(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];"
       ::"r"(ptx::smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(ptx::smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
-}
-
-// Writes D/4 packed 32-bit columns (D/2 16-bit elements) of a global row
-// into this thread's TMEM lane starting at `taddr` (zeros when src is null).
-template <int D>
-__device__ __forceinline__ void row_half_to_tmem(const void* src, uint32_t taddr) {
-  constexpr int NC = D / 4;  // 32-bit columns in half a row
-  uint32_t r[NC];
-  if (src) {
-    const uint4* s4 = reinterpret_cast<const uint4*>(src);
-#pragma unroll
-    for (int i = 0; i < NC / 4; ++i) {
-      const uint4 v = s4[i];
-      r[4 * i] = v.x;
-      r[4 * i + 1] = v.y;
-      r[4 * i + 2] = v.z;
-      r[4 * i + 3] = v.w;
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < NC; ++i) r[i] = 0u;
-  }
-  if constexpr (NC == 32) {
-    ptx::tmem_st32(taddr, r);
-  } else {
-    ptx::tmem_st16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
-  }
 }
 
 struct Maps {
@@ -94,14 +63,6 @@ struct Maps {
   CUtensorMap lse;  // row LSE        {b1q_pad, BH*b2},     box {64, 1}
 };
 
-
-// Writes a whole row of D 16-bit elements (D/2 packed columns) into this
-// thread's TMEM lane starting at `taddr` (zeros when src is null).
-template <int D>
-__device__ __forceinline__ void row_to_tmem(const void* src, uint32_t taddr) {
-  row_half_to_tmem<D>(src, taddr);
-  row_half_to_tmem<D>(src ? static_cast<const uint8_t*>(src) + D : nullptr, taddr + D / 4);
-}
 
 }  // namespace tc
 }  // namespace monarch
