@@ -2,10 +2,13 @@
 // column pass).
 //
 // A CTA owns two 128-row tiles (A and B) of one (head, position a2) problem.
-// Warps 0-3 run the softmax of tile A and warps 4-7 that of tile B (thread r
-// of a warpgroup owns row r of its tile = TMEM lane r); warp 8 issues the
-// MMAs and warp 9 the TMA loads, each from one lane.  The issuer alternates
-// between the tiles, so one tile's MMAs run while the other's softmax works.
+// Warps 0-7 run the softmax of tile A and warps 8-15 that of tile B.  Thread
+// r of a tile's warps w and w + 4 owns row r of the tile (TMEM lane r, lane
+// quadrant w mod 4); warp w takes the first half of the block's columns and
+// warp w + 4 the second, so one tile's softmax finishes in about half the time
+// it takes a single warp per row.  Warp 16 issues the MMAs and warp 17 the
+// TMA loads, each from one lane.  The issuer alternates between the tiles, so
+// one tile's MMAs run while the other's softmax works.
 //
 // Every MMA is N >= 128 wide: a single thread issues about one tcgen05.mma per
 // 60 cycles, so an N = 64 instruction (32 cycles of math) would leave the
@@ -20,6 +23,13 @@
 // and a commit arrives when every earlier MMA is complete, so "S(j+1) done"
 // also means "P z (j) done".
 //
+// The two column halves of a row share one running shift in the output pass:
+// they exchange block maxima through shared memory at a per-tile named
+// barrier, which also orders every read of S before the P stores over it.  The
+// LSE pass keeps a shift per half and merges the halves at the end; there the
+// exponentials (one per score, as many as the score MMA has columns) are split
+// between the MUFU unit and an FMA-pipe polynomial.
+//
 // Precision: k~ and z as hi/lo planes, q exact, L split into hi/lo planes in
 // the column pass, P single f16 with the rounded values summed, fp32
 // statistics; h arrives in bits (base-2 entropy).
@@ -30,9 +40,26 @@
 namespace monarch {
 namespace tc {
 
-constexpr int kThreads = 320;   // 2 softmax warpgroups + MMA warp + TMA warp
-constexpr int kMmaWarp = 8;
-constexpr int kLoadWarp = 9;
+constexpr int kSoftWarps = 16;  // 8 per tile: 4 lane quadrants x 2 column halves
+constexpr int kThreads = 32 * (kSoftWarps + 2);   // + MMA warp + TMA warp
+constexpr int kMmaWarp = kSoftWarps;
+constexpr int kLoadWarp = kSoftWarps + 1;
+constexpr int kTileThreads = 256;                  // softmax threads of one tile
+
+// Exchange area of one tile between its two column halves (bytes):
+//   output pass   bf16 block maxima [parity][half][128], then f32 row sums [half][128]
+//   LSE pass      f32 [m, l][half][128]
+//   column pass   f32 column sums [half][128]
+template <int KIND> constexpr int xchg_tile_bytes() { return KIND == 1 ? 1024 : (KIND == 0 ? 2048 : 1024); }
+
+// Dynamic shared memory starts 1024-byte aligned (no static shared memory in
+// these kernels); the 128-byte swizzle of the TMA boxes needs that.  A kernel
+// that finds otherwise records kErrSmemAlign and returns before any TMA.
+__device__ __forceinline__ bool smem_misaligned(const void* p) {
+  if ((ptx::smem_u32(p) & 1023u) == 0) return false;
+  if (threadIdx.x == 0) atomicExch(&ptx::g_device_error, ptx::kErrSmemAlign);
+  return true;
+}
 constexpr int kKS = 3;          // k~ / h stages (row passes)
 constexpr int kQS = 2;          // query / lse stages (column pass)
 constexpr int kQBlk = 128;      // queries per column-pass block
@@ -44,8 +71,9 @@ constexpr size_t kExclusiveSmem = 120 * 1024;
 template <int D, bool OUT>
 constexpr size_t row_smem() {
   constexpr int NH = D / 64;
-  constexpr size_t need = 1024 + (size_t)2 * NH * 2 * kBox /* q */ + (size_t)kKS * 2 * NH * kBox /* k~ */ +
-                          (OUT ? (size_t)2 * 2 * NH * kBox : 0) /* z */ + kKS * kBlk * 4 + 32 * 8;
+  constexpr size_t need = (size_t)2 * NH * 2 * kBox /* q */ + (size_t)kKS * 2 * NH * kBox /* k~ */ +
+                          (OUT ? (size_t)2 * 2 * NH * kBox : 0) /* z */ + kKS * kBlk * 4 +
+                          2 * xchg_tile_bytes<OUT ? 1 : 0>() + 32 * 8;
   return need > kExclusiveSmem ? need : kExclusiveSmem;
 }
 
@@ -64,12 +92,14 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
   constexpr uint32_t kKst = 2 * NH * kBox;   // k~ hi+lo, 64 rows: [d half][plane][64 rows]
   constexpr uint32_t kZst = 2 * NH * kBox;   // z hi+lo, 64 rows:  [plane][d half][64 rows]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sQ = base;                                                 // [2 tiles]
+  if (smem_misaligned(smem_raw)) return;
+  uint8_t* sQ = smem_raw;                                             // [2 tiles]
   uint8_t* sK = sQ + 2 * kQt;                                         // [kKS]
   uint8_t* sZ = sK + kKS * kKst;                                      // [2] (OUT)
   float* sH = reinterpret_cast<float*>(sZ + (OUT ? 2 * kZst : 0));    // [kKS][64]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sH + kKS * kBlk);
+  constexpr int kXt = xchg_tile_bytes<OUT ? 1 : 0>();
+  uint8_t* sX = reinterpret_cast<uint8_t*>(sH + kKS * kBlk);          // [tile][kXt bytes]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * kXt);
   uint64_t* q_full = bar + 0;
   uint64_t* k_full = bar + 1;    // [kKS]
   uint64_t* k_free = bar + 4;    // [kKS]
@@ -93,18 +123,18 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     ptx::mbar_init(q_full, 1);
     for (int i = 0; i < kKS; ++i) {
       ptx::mbar_init(k_full + i, 1);
-      ptx::mbar_init(k_free + i, 4 * ntiles);
+      ptx::mbar_init(k_free + i, 8 * ntiles);
     }
     for (int i = 0; i < 2; ++i) {
       ptx::mbar_init(z_full + i, 1);
       ptx::mbar_init(z_free + i, 1);
     }
     for (int t = 0; t < 2; ++t) {
-      ptx::mbar_init(p_full + t, 4);
+      ptx::mbar_init(p_full + t, 8);
       ptx::mbar_init(o_done + t, 1);
       for (int b = 0; b < 2; ++b) {
         ptx::mbar_init(s_full + 2 * t + b, 1);
-        ptx::mbar_init(s_free + 2 * t + b, 4);
+        ptx::mbar_init(s_free + 2 * t + b, 8);
       }
     }
     ptx::fence_mbar_init();
@@ -226,7 +256,8 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     }
   } else {
     // ------------------------------------------------------- softmax warps
-    const int t = warp >> 2;
+    const int t = warp >> 3;                 // tile
+    const int hf = (warp >> 2) & 1;          // column half: keys 32 hf .. 32 hf + 31 of a block
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int a1 = a1_base + t * kTile + r;
@@ -238,117 +269,152 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
         const int ks = j % kKS;
         const int b = OUT ? 0 : (j & 1);
         const uint32_t ph = OUT ? (j & 1) : ((j >> 1) & 1);
-        // after a timed-out wait the loop keeps its shape but skips waits
+        // after a timed-out wait the loop keeps its shape (and its named
+        // barriers) but skips waits
         ok = ok && ptx::mbar_wait(s_full + 2 * t + b, ph) && ptx::mbar_wait(k_full + ks, (j / kKS) & 1);
         ptx::tc_fence_after();
-        const float4* hv = reinterpret_cast<const float4*>(sH + ks * kBlk);
-        float2 x[32];
+        const float4* hv = reinterpret_cast<const float4*>(sH + ks * kBlk + 32 * hf);
+        float2 x[16];   // x[i] = keys 32 hf + 2i, 32 hf + 2i + 1
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // keys 32 hh .. 32 hh + 31
-          uint32_t shi[32], slo[32];
-          ptx::tmem_ld32(tS(t, b) + lane_off + 32 * hh, shi);
-          ptx::tmem_ld32(tS(t, b) + lane_off + 64 + 32 * hh, slo);
+        for (int hh = 0; hh < 2; ++hh) {  // 16 keys at a time
+          uint32_t shi[16], slo[16];
+          ptx::tmem_ld16(tS(t, b) + lane_off + 32 * hf + 16 * hh, shi);
+          ptx::tmem_ld16(tS(t, b) + lane_off + 64 + 32 * hf + 16 * hh, slo);
           ptx::tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const float4 h4 = hv[8 * hh + i];
+          for (int i = 0; i < 4; ++i) {
+            const float4 h4 = hv[4 * hh + i];
             const float2 s0 = add2(make_float2(__uint_as_float(shi[4 * i]), __uint_as_float(shi[4 * i + 1])),
                                    make_float2(__uint_as_float(slo[4 * i]), __uint_as_float(slo[4 * i + 1])));
             const float2 s1 = add2(make_float2(__uint_as_float(shi[4 * i + 2]), __uint_as_float(shi[4 * i + 3])),
                                    make_float2(__uint_as_float(slo[4 * i + 2]), __uint_as_float(slo[4 * i + 3])));
-            x[16 * hh + 2 * i] = fma2(s0, sl2, make_float2(h4.x, h4.y));
-            x[16 * hh + 2 * i + 1] = fma2(s1, sl2, make_float2(h4.z, h4.w));
+            x[8 * hh + 2 * i] = fma2(s0, sl2, make_float2(h4.x, h4.y));
+            x[8 * hh + 2 * i + 1] = fma2(s1, sl2, make_float2(h4.z, h4.w));
           }
         }
-        // S and h of this block are consumed: release the k~/h stage
+        // S and h of this block are read: release the k~/h stage
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) {
           ptx::mbar_arrive(k_free + ks);
           if (!OUT) ptx::mbar_arrive(s_free + 2 * t + b);
         }
-        const int valid = min(kBlk, g.b1k - j * kBlk);
-        if (valid < kBlk) {  // only the last block of a ragged row
+        const int valid = min(kBlk, g.b1k - j * kBlk) - 32 * hf;   // keys of this half (may be <= 0)
+        if (valid < 32) {  // only the last block of a ragged row
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 16; ++i) {
             if (2 * i >= valid) x[i].x = -INFINITY;
             if (2 * i + 1 >= valid) x[i].y = -INFINITY;
           }
         }
         float mb = -INFINITY;
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mb = fmaxf(mb, fmaxf(x[i].x, x[i].y));
+        for (int i = 0; i < 16; ++i) mb = fmaxf(mb, fmaxf(x[i].x, x[i].y));
+        if constexpr (OUT) {
+          // one shift per row: merge the two halves' block maxima.  The
+          // barrier also orders every S read of this tile before the P stores.
+          // Both halves use the maxima rounded up to bf16, so they agree on
+          // the shift; rounding up keeps every exponent <= 8.
+          __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(sX + t * kXt) + (j & 1) * 2 * kTile;
+          const __nv_bfloat16 mine = __float2bfloat16_ru(mb);
+          xs[hf * kTile + r] = mine;
+          ptx::tc_fence_before();
+          ptx::named_bar(1 + t, kTileThreads);
+          ptx::tc_fence_after();
+          mb = fmaxf(__bfloat162float(mine), __bfloat162float(xs[(hf ^ 1) * kTile + r]));
+        }
         // the running shift moves only when the max grows by more than 2^8
         const bool move = mb > m + kLazyRescale;
         const float mn = move ? mb : m;
-        const float corr = ptx::ex2(m - mn);
-        const float2 nm = make_float2(-mn, -mn);
+        const float corr = (mn == m) ? 1.f : ptx::ex2(m - mn);
+        const float nmv = (mn == -INFINITY) ? 0.f : -mn;   // a half with no key yet
+        const float2 nm = make_float2(nmv, nmv);
         float2 acc2 = make_float2(0.f, 0.f);
         if constexpr (OUT) {
-          // S(t, j) is complete, hence so is P z (j-1): O may be rescaled
+          // S(t, j) is complete, hence so is P z (j-1): O may be rescaled.
+          // The decision is the same in both halves; each scales its half of O.
           if (j > 0 && __any_sync(0xffffffffu, move)) {
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
-              uint32_t o[32];
-              ptx::tmem_ld32(tO(t) + lane_off + cc * 32, o);
+              uint32_t o[16];
+              ptx::tmem_ld16(tO(t) + lane_off + hf * (D / 2) + cc * 16, o);
               ptx::tmem_wait_ld();
 #pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
-              ptx::tmem_st32(tO(t) + lane_off + cc * 32, o);
+              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * corr);
+              ptx::tmem_st16(tO(t) + lane_off + hf * (D / 2) + cc * 16, o);
             }
           }
-          uint32_t pk[32];
+          uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 16; ++i) {
             const float2 d = add2(x[i], nm);
             const __half2 hp = __floats2half2_rn(ptx::ex2(d.x), ptx::ex2(d.y));
             acc2 = add2(acc2, __half22float2(hp));
             pk[i] = *reinterpret_cast<const uint32_t*>(&hp);
           }
-          // P (keys 2c, 2c+1 in column c) over the first 32 columns of S
-          ptx::tmem_st32(tS(t, 0) + lane_off, pk);
+          // P: keys 2c, 2c + 1 in column c of the first 32 columns of S
+          ptx::tmem_st16(tS(t, 0) + lane_off + 16 * hf, pk);
           ptx::tmem_wait_st();
           ptx::tc_fence_before();
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(p_full + t);
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 16; ++i) {
             const float2 d = add2(x[i], nm);
-            acc2 = add2(acc2, make_float2(ptx::ex2(d.x), ptx::ex2(d.y)));
+            // one pair in four on the FMA pipe, the rest on the MUFU unit
+            const float2 e = ((i & 3) == 3) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
+            acc2 = add2(acc2, e);
           }
         }
         l = fmaf(l, corr, acc2.x + acc2.y);
         m = mn;
       }
       if constexpr (OUT) {
+        // row sum = the two halves' sums (same shift); the first barrier ends
+        // every read of the block maxima that share these bytes
+        float* xs = reinterpret_cast<float*>(sX + t * kXt);
+        ptx::named_bar(1 + t, kTileThreads);
+        xs[hf * kTile + r] = l;
+        ptx::named_bar(1 + t, kTileThreads);
+        const float lt = l + xs[(hf ^ 1) * kTile + r];
         ok = ok && ptx::mbar_wait(o_done + t, 0);
         ptx::tc_fence_after();
-        const float inv = 1.f / l;
-        TO* orow = out + ((long long)bh * g.Nq + (a1 < g.b1q ? token_of(g, a1, a2) : 0)) * D;
+        const float inv = 1.f / lt;
+        TO* orow = out + ((long long)bh * g.Nq + (a1 < g.b1q ? token_of(g, a1, a2) : 0)) * D + hf * (D / 2);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          ptx::tmem_ld32(tO(t) + lane_off + cc * 32, o);
+          uint32_t o[16];
+          ptx::tmem_ld16(tO(t) + lane_off + hf * (D / 2) + cc * 16, o);
           ptx::tmem_wait_ld();
           if (a1 < g.b1q && ok) {
 #pragma unroll
-            for (int i = 0; i < 32; i += 4) {
+            for (int i = 0; i < 16; i += 4) {
               if constexpr (sizeof(TO) == 4) {
-                *reinterpret_cast<float4*>(orow + cc * 32 + i) =
+                *reinterpret_cast<float4*>(orow + cc * 16 + i) =
                     make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
                                 __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
               } else {
                 TO v4[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) v4[e] = from_f<TO>(__uint_as_float(o[i + e]) * inv);
-                *reinterpret_cast<uint2*>(orow + cc * 32 + i) = *reinterpret_cast<uint2*>(v4);
+                *reinterpret_cast<uint2*>(orow + cc * 16 + i) = *reinterpret_cast<uint2*>(v4);
               }
             }
           }
         }
-      } else if (a1 < g.b1q) {
-        lse[(long long)zrow * g.b1q_pad + a1] = m + log2f(l);
+      } else {
+        // merge the halves: (m, l) of each, shifts may differ
+        float* xs = reinterpret_cast<float*>(sX + t * kXt);   // [m, l][half][128]
+        xs[hf * kTile + r] = m;
+        xs[2 * kTile + hf * kTile + r] = l;
+        ptx::named_bar(1 + t, kTileThreads);
+        if (hf == 0 && a1 < g.b1q) {
+          const float mo = xs[kTile + r], lo = xs[3 * kTile + r];
+          const float M = fmaxf(m, mo);
+          const float L = (m == -INFINITY ? 0.f : l * ptx::ex2(m - M)) + (mo == -INFINITY ? 0.f : lo * ptx::ex2(mo - M));
+          lse[(long long)zrow * g.b1q_pad + a1] = M + log2f(L);
+        }
       }
     }
   }
@@ -361,13 +427,13 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
 // Column pass for one (head, position a2, 256 key tiles), 128 queries per block:
 //   q~[c1,a2] = sum_a1 L q / sum_a1 L,  L = 2^(s q.k~ + h - lse[a1]).
 // TMEM, tile t at column 256 t:  S^T [0, 128) for 128 queries; P^T is written
-// over it as [hi q0-63 | lo q0-63 | hi q64-127 | lo q64-127] (32 columns
-// each);  acc [128, 128 + D).
+// over it per 32-query chunk c as [hi | lo] in columns [32 c, 32 c + 32)
+// (16 columns each, two queries per column);  acc [128, 128 + D).
 template <int D>
 constexpr size_t col_smem() {
   constexpr int NH = D / 64;
-  constexpr size_t need = 1024 + (size_t)2 * 2 * NH * 2 * kBox /* k~ */ + (size_t)kQS * NH * 2 * kBox /* q */ +
-                          kQS * kQBlk * 4 + 32 * 8;
+  constexpr size_t need = (size_t)2 * 2 * NH * 2 * kBox /* k~ */ + (size_t)kQS * NH * 2 * kBox /* q */ +
+                          kQS * kQBlk * 4 + 2 * xchg_tile_bytes<2>() + 32 * 8;
   return need > kExclusiveSmem ? need : kExclusiveSmem;
 }
 
@@ -378,11 +444,12 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
   constexpr uint32_t kKt = 2 * NH * 2 * kBox;   // k~ hi+lo of one tile: [plane][d half][128 rows]
   constexpr uint32_t kQst = NH * 2 * kBox;      // 128 query rows: [d half][128 rows]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sK = base;                                        // [2 tiles]
+  if (smem_misaligned(smem_raw)) return;
+  uint8_t* sK = smem_raw;                                    // [2 tiles]
   uint8_t* sQ = sK + 2 * kKt;                                // [kQS]
   float* sL = reinterpret_cast<float*>(sQ + kQS * kQst);     // [kQS][128]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sL + kQS * kQBlk);
+  float* sX = sL + kQS * kQBlk;                              // [tile][half][128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * xchg_tile_bytes<2>() / 4);
   uint64_t* k_full = bar + 0;
   uint64_t* q_full = bar + 1;    // [kQS]
   uint64_t* q_free = bar + 3;    // [kQS]
@@ -407,7 +474,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
     }
     for (int t = 0; t < 2; ++t) {
       ptx::mbar_init(s_full + t, 1);
-      ptx::mbar_init(p_full + t, 4);
+      ptx::mbar_init(p_full + t, 8);
       ptx::mbar_init(o_done + t, 1);
     }
     ptx::fence_mbar_init();
@@ -483,7 +550,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
           for (int p = 0; p < 2; ++p)
 #pragma unroll
             for (int kk = 0; kk < kQBlk / 16; ++kk)
-              ptx::mma_f16_ts(tA(t), tp + (kk >> 2) * 64 + p * 32 + (kk & 3) * 8, q0 + ((kk * 2048) >> 4), idPQ,
+              ptx::mma_f16_ts(tA(t), tp + (kk >> 1) * 32 + p * 16 + (kk & 1) * 8, q0 + ((kk * 2048) >> 4), idPQ,
                               (i | p | kk) != 0);
           if (t == ntiles - 1) ptx::mma_commit(q_free + qs);
           if (i + 1 < nqb) {
@@ -498,8 +565,9 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
       }
     }
   } else {
-    const int t = warp >> 2;
-    const int r = 32 * (warp & 3) + lane;   // key tile row / TMEM lane
+    const int t = warp >> 3;                 // tile
+    const int hf = (warp >> 2) & 1;          // column half: queries 64 hf .. 64 hf + 63 of a block
+    const int r = 32 * (warp & 3) + lane;    // key tile row / TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int c1 = kb + t * kTile + r;
     if (t < ntiles) {
@@ -513,15 +581,15 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
         ptx::tc_fence_after();
         const int valid = min(kQBlk, g.b1q - i * kQBlk);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // queries 64 hh .. 64 hh + 63
-          uint32_t sr[64];
-          ptx::tmem_ld32(tS(t) + lane_off + 64 * hh, *reinterpret_cast<uint32_t(*)[32]>(sr));
-          ptx::tmem_ld32(tS(t) + lane_off + 64 * hh + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-          const float4* lv = reinterpret_cast<const float4*>(sL + qs * kQBlk + 64 * hh);
+        for (int hh = 0; hh < 2; ++hh) {  // 32 queries at a time
+          const int cb = 64 * hf + 32 * hh;   // first S^T column (query) of this chunk
+          uint32_t sr[32];
+          ptx::tmem_ld32(tS(t) + lane_off + cb, sr);
+          const float4* lv = reinterpret_cast<const float4*>(sL + qs * kQBlk + cb);
           ptx::tmem_wait_ld();
-          uint32_t hi[32], lo[32];
+          uint32_t hi[16], lo[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
+          for (int e = 0; e < 8; ++e) {
             const float4 l4 = lv[e];
             float2 x0 = fma2(make_float2(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1])), sl2, hb2);
             float2 x1 =
@@ -531,7 +599,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
             float2 p0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
             float2 p1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
             if (valid < kQBlk) {  // only the last block of a ragged column
-              const int q0 = 64 * hh + 4 * e;
+              const int q0 = cb + 4 * e;
               if (q0 >= valid) p0.x = 0.f;
               if (q0 + 1 >= valid) p0.y = 0.f;
               if (q0 + 2 >= valid) p1.x = 0.f;
@@ -541,23 +609,28 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
             split2<TQ>(p0, hi[2 * e], lo[2 * e]);
             split2<TQ>(p1, hi[2 * e + 1], lo[2 * e + 1]);
           }
-          // P^T hi / lo of these 64 queries over the S^T columns just read
-          ptx::tmem_st32(tS(t) + lane_off + 64 * hh, hi);
-          ptx::tmem_st32(tS(t) + lane_off + 64 * hh + 32, lo);
+          // P^T of these 32 queries over the chunk's own S^T columns:
+          // hi in [cb, cb + 16), lo in [cb + 16, cb + 32)
+          ptx::tmem_st16(tS(t) + lane_off + cb, hi);
+          ptx::tmem_st16(tS(t) + lane_off + cb + 16, lo);
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(p_full + t);
       }
+      // beta = the two halves' column sums
+      sX[(t * 2 + hf) * kTile + r] = beta2.x + beta2.y;
+      ptx::named_bar(1 + t, kTileThreads);
+      const float beta = beta2.x + beta2.y + sX[(t * 2 + (hf ^ 1)) * kTile + r];
       ok = ok && ptx::mbar_wait(o_done + t, 0);
       ptx::tc_fence_after();
-      const float inv = 1.f / (beta2.x + beta2.y);
-      float* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D;
+      const float inv = 1.f / beta;
+      float* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
+      for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t o[32];
-        ptx::tmem_ld32(tA(t) + lane_off + cc * 32, o);
+        ptx::tmem_ld32(tA(t) + lane_off + hf * (D / 2) + cc * 32, o);
         ptx::tmem_wait_ld();
         if (c1 < g.b1k && ok) {
 #pragma unroll

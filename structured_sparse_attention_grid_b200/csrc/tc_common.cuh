@@ -33,6 +33,30 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return u2f(d);
 }
 
+// 2^x of a pair on the FMA pipe (the MUFU unit is the other source of 2^x;
+// the row pass sends part of its exponentials here to balance the two).
+// x = n + f with n = rint(x) (the 1.5 * 2^23 rounding constant) and f in
+// [-1/2, 1/2]; 2^f by the degree-5 equal-ripple polynomial of gen_exp2_poly.py
+// (relative error 1.6e-7 in float32); 2^n is added to the exponent field.
+// Inputs are clamped to -127, so -inf and anything below -127 give 0 or a
+// value below 2^-126.  Inputs must be at most 127.
+__device__ __forceinline__ float2 ex2_fma2(float2 x) {
+  x.x = fmaxf(x.x, -127.f);
+  x.y = fmaxf(x.y, -127.f);
+  const float2 rc = make_float2(12582912.f, 12582912.f);
+  const float2 t = add2(x, rc);
+  const float2 f = sub2(x, sub2(t, rc));
+  float2 p = fma2(make_float2(1.326821395e-03f, 1.326821395e-03f), f,
+                  make_float2(9.671511129e-03f, 9.671511129e-03f));
+  p = fma2(p, f, make_float2(5.550721660e-02f, 5.550721660e-02f));
+  p = fma2(p, f, make_float2(2.402224243e-01f, 2.402224243e-01f));
+  p = fma2(p, f, make_float2(6.931470037e-01f, 6.931470037e-01f));
+  p = fma2(p, f, make_float2(1.f, 1.f));
+  // the low bits of t hold n: (bits(t) << 23) is n in the exponent field
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // hi = round(p) and lo = round(p - hi) of a pair, packed, in the operand type.
 template <typename TQ>
 __device__ __forceinline__ void split2(float2 p, uint32_t& hi, uint32_t& lo) {
