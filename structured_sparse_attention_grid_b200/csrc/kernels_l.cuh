@@ -52,14 +52,6 @@ constexpr int kTileThreads = 256;                  // softmax threads of one til
 //   column pass   f32 column sums [half][128]
 template <int KIND> constexpr int xchg_tile_bytes() { return KIND == 1 ? 1024 : (KIND == 0 ? 2048 : 1024); }
 
-// Dynamic shared memory starts 1024-byte aligned (no static shared memory in
-// these kernels); the 128-byte swizzle of the TMA boxes needs that.  A kernel
-// that finds otherwise records kErrSmemAlign and returns before any TMA.
-__device__ __forceinline__ bool smem_misaligned(const void* p) {
-  if ((ptx::smem_u32(p) & 1023u) == 0) return false;
-  if (threadIdx.x == 0) atomicExch(&ptx::g_device_error, ptx::kErrSmemAlign);
-  return true;
-}
 constexpr int kKS = 3;          // k~ / h stages (row passes)
 constexpr int kQS = 2;          // query / lse stages (column pass)
 constexpr int kQBlk = 128;      // queries per column-pass block
@@ -425,7 +417,8 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
 
 // ===========================================================================
 // Column pass for one (head, position a2, 256 key tiles), 128 queries per block:
-//   q~[c1,a2] = sum_a1 L q / sum_a1 L,  L = 2^(s q.k~ + h - lse[a1]).
+//   q~[c1,a2] = sum_a1 L q / sum_a1 L,  L = 2^(s q.k~ + h - lse[a1]),
+// stored as hi / lo planes of the input type ([plane][BH][b2][b1k][d]).
 // TMEM, tile t at column 256 t:  S^T [0, 128) for 128 queries; P^T is written
 // over it per 32-query chunk c as [hi | lo] in columns [32 c, 32 c + 32)
 // (16 columns each, two queries per column);  acc [128, 128 + D).
@@ -439,7 +432,7 @@ constexpr size_t col_smem() {
 
 template <typename TQ, int D>
 __global__ void __launch_bounds__(kThreads, 1)
-l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* __restrict__ qt, Geo g) {
+l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __restrict__ qt, Geo g) {
   constexpr int NH = D / 64;
   constexpr uint32_t kKt = 2 * NH * 2 * kBox;   // k~ hi+lo of one tile: [plane][d half][128 rows]
   constexpr uint32_t kQst = NH * 2 * kBox;      // 128 query rows: [d half][128 rows]
@@ -626,18 +619,27 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, float* 
       ok = ok && ptx::mbar_wait(o_done + t, 0);
       ptx::tc_fence_after();
       const float inv = 1.f / beta;
-      float* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);
+      // q~ as hi / lo planes of the input type: the A operand of the next R step
+      const long long plane = (long long)g.BH * g.b2 * g.b1k * D;
+      TQ* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);
+      const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
       for (int cc = 0; cc < D / 64; ++cc) {
         uint32_t o[32];
         ptx::tmem_ld32(tA(t) + lane_off + hf * (D / 2) + cc * 32, o);
         ptx::tmem_wait_ld();
-        if (c1 < g.b1k && ok) {
+        uint32_t hi[16], lo[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            *reinterpret_cast<float4*>(dst + cc * 32 + e) =
-                make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                            __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
+        for (int e = 0; e < 16; ++e)
+          split2<TQ>(mul2(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), inv2), hi[e], lo[e]);
+        if (c1 < g.b1k && ok) {
+          uint4* ph = reinterpret_cast<uint4*>(dst + cc * 32);
+          uint4* pl = reinterpret_cast<uint4*>(dst + plane + cc * 32);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            ph[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+            pl[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+          }
         }
       }
     }

@@ -1,0 +1,399 @@
+// R step on the tensor cores for bf16 / f16 inputs.
+//
+// A CTA takes a group of G = floor(128 / r8) consecutive key tiles of one head
+// (r8 = b2 rounded up to 8) and stacks their rows: row r = g r8 + a2 holds
+// position a2 of key tile c1_0 + g.  With A = the stacked q~ rows (hi and lo
+// planes, or the exact query rows) and B = the stacked key rows, one
+// 128 x 128 score block
+//     S = A K^T                     (tcgen05, N = 128, fp32 in TMEM)
+// holds every tile's b2 x b2 scores on its diagonal.  Thread r (TMEM lane r)
+// masks its row to the columns of its own tile and takes the softmax over c2
+// (R = softmax_c2(s q~ . k)) and its entropy h, then writes R back over S as
+// the hi / lo planes of the A operand of
+//     k~ = R K,   z = R V           (A from TMEM, B = keys / values in shared
+//                                    memory, N = d)
+// R is zero outside the diagonal blocks, so these are the per-tile products.
+// The epilogue splits each row into hi / lo planes, stages them in shared
+// memory in the swizzled box layout and one thread stores them with per-tile
+// TMA boxes into [plane][BH][b2][b1k][d] (position-major), the layout the L
+// step reads.  In the first step the exact query rows, already in shared
+// memory, go out the same way as the block-major copy of q.
+//
+// Loads: keys, values and exact query rows come through the 4-D grid map
+// (d, W, H, frames) with one tile per box, so the grid -> block permutation is
+// done by the TMA unit; q~ planes come through a 3-D map with one tile per box.
+// Shared memory: A (two planes) and K, [d half][128 rows][128 B] boxes with the
+// 128-byte swizzle; V reuses the A hi plane once the score MMAs are complete.
+// That is 96 KB for d = 128 and 256 TMEM columns, so two CTAs share an SM and
+// one CTA's loads overlap the other's arithmetic.
+#pragma once
+
+#include "common.cuh"
+#include "ptx.cuh"
+#include "kernels_tc.cuh"
+#include "tc_common.cuh"
+
+namespace monarch {
+
+struct RtcMaps {
+  CUtensorMap q;    // queries    {d, W, H, BH*T},        box {64, tw, th, 1}
+  CUtensorMap k;    // keys       {d, W, H, BH*Tk},       box {64, tw, th, 1}
+  CUtensorMap v;    // values     {d, W, H, BH*Tk},       box {64, tw, th, 1}
+  CUtensorMap qt;   // q~ planes  {d, b1k, 2*BH*b2},      box {64, 1, b2}
+  CUtensorMap qb;   // block-major q (store) {d, b1q, BH*b2},     box {64, 1, b2}
+  CUtensorMap kt;   // k~ planes (store)     {d, b1k, 2*BH*b2},   box {64, 1, b2}
+  CUtensorMap z;    // z planes, f16 (store) {d, b1k, 2*BH*b2},   box {64, 1, b2}
+};
+
+// Planes written by the R step.
+template <typename TQ>
+struct TcPlanes {
+  TQ* kt_hi;        // [BH][b2][b1k][d], then the lo plane at kt_hi + plane
+  __half* z_hi;     // [BH][b2][b1k][d], then the lo plane
+  long long plane;  // elements per plane
+};
+
+constexpr int kRtcThreads = 160;      // 4 row warps (TMEM lanes 0-127) + a control warp
+constexpr int kRtcRows = 128;
+constexpr uint32_t kRBox = 128 * 128; // one [128 rows][128 B] swizzled box
+
+// At least 80 KB so that at most two CTAs (2 x 256 TMEM columns) share an SM.
+template <int D>
+constexpr size_t rtc_smem() {
+  constexpr size_t need = (size_t)3 * (D / 64) * kRBox + 8 * 8;
+  return need > 80 * 1024 ? need : 80 * 1024;
+}
+
+// grid (ceil(b1k / G), BH), block kRtcThreads.
+template <typename TQ, int D>
+__global__ void __launch_bounds__(kRtcThreads, 2)
+r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work w, TcPlanes<TQ> out, Geo g,
+           int mode, int final_step) {
+  constexpr int NH = D / 64;
+  constexpr int bf16 = TcType<TQ>::kBf16;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (tc::smem_misaligned(smem_raw)) return;
+  uint8_t* sA = smem_raw;                  // [plane][d half] boxes; V in plane 0 later
+  uint8_t* sK = sA + 2 * NH * kRBox;       // [d half] boxes
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sK + NH * kRBox);
+  uint64_t* bar_ld = bar + 0;    // TMA: keys and query rows
+  uint64_t* bar_a = bar + 1;     // row warps: query rows written by threads (KV init)
+  uint64_t* bar_s = bar + 2;     // MMA: S complete
+  uint64_t* bar_r = bar + 3;     // row warps: R in TMEM
+  uint64_t* bar_acc = bar + 4;   // MMA: k~ (phase 0), z (phase 1) complete
+  uint64_t* bar_free = bar + 5;  // row warps: k~ read out of TMEM
+  uint64_t* bar_v = bar + 6;     // TMA: values
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 7);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y;
+  const int r8 = (g.b2 + 7) & ~7;
+  const int G = kRtcRows / r8;
+  const int c1_0 = blockIdx.x * G;
+  const int Gn = min(G, g.b1k - c1_0);
+
+  if (tid == 128) {
+    ptx::mbar_init(bar_ld, 1);
+    ptx::mbar_init(bar_a, 4);
+    ptx::mbar_init(bar_s, 1);
+    ptx::mbar_init(bar_r, 4);
+    ptx::mbar_init(bar_acc, 1);
+    ptx::mbar_init(bar_free, 4);
+    ptx::mbar_init(bar_v, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 256);
+    ptx::tmem_relinquish();
+  }
+  // Zero every row that no load writes (in-tile padding, tiles past the end):
+  // K and V rows there meet zero R entries, and 0 * NaN would not be zero.
+  for (int i = tid; i < kRtcRows * NH * 8; i += kRtcThreads) {
+    const int row = i / (NH * 8), rem = i - row * (NH * 8), hf = rem >> 3, ch = rem & 7;
+    const int gg = row / r8, a = row - gg * r8;
+    if (gg >= Gn || a >= g.b2) {
+      const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t o = hf * kRBox + row * 128 + ch * 16;
+      *reinterpret_cast<uint4*>(sK + o) = z4;
+      *reinterpret_cast<uint4*>(sA + o) = z4;
+      *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = z4;
+    }
+  }
+  ptx::fence_proxy_async();
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  const uint32_t tS = tmem, tAcc = tmem + 128;
+
+  // tile c1 -> (frame, tile row, tile column) of its grid box
+  auto tile_coords = [&](int c1, int& t, int& y0, int& x0) {
+    t = c1 / g.P;
+    const int rem = c1 - t * g.P, ty = rem / g.ntx;
+    y0 = ty * g.th;
+    x0 = (rem - ty * g.ntx) * g.tw;
+  };
+  auto exact_q = [&](int c1) { return mode == QT_IDENTITY || (mode == QT_KVINIT && c1 >= g.off); };
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ------------------------------------------------ loads and MMA issue
+      ptx::prefetch_tmap(&maps.k);
+      bool ok = true;
+      uint32_t bytes = 0;
+      for (int gg = 0; gg < Gn; ++gg) {
+        const int c1 = c1_0 + gg;
+        const int planes = mode == QT_BUFFER ? 2 : (exact_q(c1) ? 1 : 0);
+        bytes += (uint32_t)(NH * g.b2 * 128 * (1 + planes));
+      }
+      ptx::mbar_expect_tx(bar_ld, bytes);
+      for (int gg = 0; gg < Gn; ++gg) {
+        const int c1 = c1_0 + gg;
+        int t, y0, x0;
+        tile_coords(c1, t, y0, x0);
+        const uint32_t row0 = (uint32_t)(gg * r8) * 128;
+        for (int hf = 0; hf < NH; ++hf)
+          ptx::tma_load_4d(sK + hf * kRBox + row0, &maps.k, bar_ld, hf * 64, x0, y0, bh * g.Tk + t);
+        if (mode == QT_BUFFER) {
+          for (int p = 0; p < 2; ++p)
+            for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_load_3d(sA + (p * NH + hf) * kRBox + row0, &maps.qt, bar_ld, hf * 64, c1,
+                               (p * g.BH + bh) * g.b2);
+        } else if (exact_q(c1)) {
+          const int tq = t - (g.Tk - g.T);   // the aligned query frame (== t without a cache)
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_load_4d(sA + hf * kRBox + row0, &maps.q, bar_ld, hf * 64, x0, y0, bh * g.T + tq);
+        }
+      }
+      ok = ptx::mbar_wait(bar_ld, 0);
+      if (ok && mode != QT_BUFFER) {
+        // first step: the exact query rows just loaded are also the block-major
+        // copy of q that the L step reads
+        for (int gg = 0; gg < Gn; ++gg) {
+          const int c1 = c1_0 + gg;
+          if (!exact_q(c1)) continue;
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_store_3d(&maps.qb, sA + hf * kRBox + (uint32_t)(gg * r8) * 128, hf * 64, c1 - g.off,
+                              bh * g.b2);
+        }
+        ptx::bulk_commit();
+      }
+      if (mode == QT_KVINIT) ok = ok && ptx::mbar_wait(bar_a, 0);
+      ptx::tc_fence_after();
+      // S = A K^T: both operands K-major (d along the 128-byte rows)
+      if (ok) {
+        constexpr uint32_t idS = ptx::idesc_f16(128, 128, bf16, 0, 0);
+        const uint64_t dA = ptx::sw128_desc(ptx::smem_u32(sA), 16, 1024);
+        const uint64_t dK = ptx::sw128_desc(ptx::smem_u32(sK), 16, 1024);
+        const bool use_lo = mode != QT_IDENTITY;
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const uint32_t off = (hf * kRBox + k4 * 32) >> 4;
+            ptx::mma_f16_ss(tS, dA + off, dK + off, idS, (hf | k4) != 0);
+            if (use_lo) ptx::mma_f16_ss(tS, dA + ((NH * kRBox) >> 4) + off, dK + off, idS, 1);
+          }
+        ptx::mma_commit(bar_s);
+      }
+      if (final_step) {
+        // V lands in the A hi plane once the score MMAs and the q copy (its
+        // readers) are done
+        ok = ok && ptx::mbar_wait(bar_s, 0);
+        ptx::bulk_wait_read();
+        if (ok) {
+          ptx::mbar_expect_tx(bar_v, (uint32_t)(Gn * NH * g.b2 * 128));
+          for (int gg = 0; gg < Gn; ++gg) {
+            int t, y0, x0;
+            tile_coords(c1_0 + gg, t, y0, x0);
+            for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_load_4d(sA + hf * kRBox + (uint32_t)(gg * r8) * 128, &maps.v, bar_v, hf * 64, x0, y0,
+                               bh * g.Tk + t);
+          }
+        }
+      }
+      // k~ = R K and z = R V: A = R in TMEM as 32-key chunks [hi 16 | lo 16]
+      // columns, B MN-major (d along the 128-byte rows, keys down the rows)
+      auto issue_rb = [&](const uint8_t* sB) {
+        constexpr uint32_t idV = ptx::idesc_f16(128, D, bf16, 0, 1);
+        const uint64_t dB = ptx::sw128_desc(ptx::smem_u32(sB), kRBox, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kRtcRows / 16; ++kk)
+#pragma unroll
+          for (int p = 0; p < 2; ++p)
+            ptx::mma_f16_ts(tAcc, tS + (kk >> 1) * 32 + p * 16 + (kk & 1) * 8, dB + ((kk * 2048) >> 4), idV,
+                            (kk | p) != 0);
+        ptx::mma_commit(bar_acc);
+      };
+      ok = ok && ptx::mbar_wait(bar_r, 0);
+      ptx::tc_fence_after();
+      if (ok) issue_rb(sK);
+      if (final_step) {
+        ok = ok && ptx::mbar_wait(bar_free, 0) && ptx::mbar_wait(bar_v, 0);
+        ptx::tc_fence_after();
+        if (ok) issue_rb(sA);
+      }
+      ptx::bulk_wait_read();
+    }
+  } else {
+    // ------------------------------------------------------------- row warps
+    const int r = tid;                          // stacked row = TMEM lane
+    const int gg = r / r8, a2 = r - gg * r8;
+    const int c1 = c1_0 + gg;
+    const bool valid = gg < Gn && a2 < g.b2;
+    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    bool ok = true;
+
+    if (mode == QT_KVINIT) {
+      // rows no load brings: cached tiles take the mean query (split into hi /
+      // lo), the lo plane of exact rows is zero
+      if (valid) {
+        const bool ex = exact_q(c1);
+        const float* qm = w.qbar + ((long long)bh * g.b2 + a2) * D;
+#pragma unroll 1
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            uint4 hi4 = make_uint4(0u, 0u, 0u, 0u), lo4 = make_uint4(0u, 0u, 0u, 0u);
+            if (!ex) {
+              const float4 u = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8);
+              const float4 v4 = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8 + 4);
+              tc::split2<TQ>(make_float2(u.x, u.y), hi4.x, lo4.x);
+              tc::split2<TQ>(make_float2(u.z, u.w), hi4.y, lo4.y);
+              tc::split2<TQ>(make_float2(v4.x, v4.y), hi4.z, lo4.z);
+              tc::split2<TQ>(make_float2(v4.z, v4.w), hi4.w, lo4.w);
+            }
+            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+            if (!ex) *reinterpret_cast<uint4*>(sA + o) = hi4;
+            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = lo4;
+          }
+      }
+      ptx::fence_proxy_async();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_a);
+    }
+
+    // ---- R = softmax over this row's tile columns [cb, cb + b2) of S.  The
+    // rows of a warp need at most three 32-column chunks, from ch_lo on: they
+    // are read from TMEM once and kept in registers.
+    ok = ptx::mbar_wait(bar_s, 0);
+    ptx::tc_fence_after();
+    const int cb = gg * r8;
+    const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
+    const int ch_lo = (wg0 * r8) >> 5, ch_hi = min((wg1 * r8 + g.b2 - 1) >> 5, 3);
+    auto in_tile = [&](int c) { return (unsigned)(c - cb) < (unsigned)g.b2; };
+    uint32_t sv[3][32];
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      if (ch_lo + j <= ch_hi) ptx::tmem_ld32(tS + lane_off + 32 * (ch_lo + j), sv[j]);
+    ptx::tmem_wait_ld();
+    float m = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i)) m = fmaxf(m, __uint_as_float(sv[j][i]));
+    const float ms = m * g.sl2;   // base-2 units
+    float l = 0.f, xe = 0.f;
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const bool in = ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i);
+        const float dx = in ? fmaf(__uint_as_float(sv[j][i]), g.sl2, -ms) : 0.f;
+        const float p = in ? ptx::ex2(dx) : 0.f;
+        l += p;
+        xe = fmaf(p, dx, xe);
+        sv[j][i] = __float_as_uint(p);
+      }
+    const float inv = 1.f / l;
+    const float2 inv2 = make_float2(inv, inv);
+    // R over S: chunk ch -> columns [32 ch, 32 ch + 16) hi, [32 ch + 16, 32 ch + 32) lo
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      if (ch_lo + j > ch_hi) continue;
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        tc::split2<TQ>(tc::mul2(make_float2(__uint_as_float(sv[j][2 * i]), __uint_as_float(sv[j][2 * i + 1])), inv2),
+                       hi[i], lo[i]);
+      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j), hi);
+      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j) + 16, lo);
+    }
+    {
+      uint32_t zero[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) zero[i] = 0u;
+      for (int ch = 0; ch < 4; ++ch)
+        if (ch < ch_lo || ch > ch_hi) {
+          ptx::tmem_st16(tS + lane_off + 32 * ch, zero);
+          ptx::tmem_st16(tS + lane_off + 32 * ch + 16, zero);
+        }
+    }
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar_r);
+    // h in bits: -sum R log2 R = log2 l - sum R (x - m)
+    if (valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
+
+    // ---- epilogue: a row of k~ (or z) from TMEM, split into hi / lo planes,
+    // staged in two swizzled [d half][128 rows][128 B] regions
+    auto stage_row = [&](uint8_t* shi, uint8_t* slo, auto tag) {
+      using TP = decltype(tag);
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t a[32];
+        ptx::tmem_ld32(tAcc + lane_off + 32 * cc, a);
+        ptx::tmem_wait_ld();
+        uint32_t hi[16], lo[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          tc::split2<TP>(make_float2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), hi[i], lo[i]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const int ch8 = (cc & 1) * 4 + v;
+          const uint32_t o = (cc >> 1) * kRBox + r * 128 + ((ch8 ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(shi + o) = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+          *reinterpret_cast<uint4*>(slo + o) = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+        }
+      }
+      ptx::fence_proxy_async();
+    };
+    // one thread: a box of b2 rows per (tile, plane, d half)
+    auto store_tiles = [&](const CUtensorMap* map, const uint8_t* shi, const uint8_t* slo) {
+      for (int t = 0; t < Gn; ++t)
+        for (int p = 0; p < 2; ++p)
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_store_3d(map, (p ? slo : shi) + hf * kRBox + (uint32_t)(t * r8) * 128, hf * 64, c1_0 + t,
+                              (p * g.BH + bh) * g.b2);
+      ptx::bulk_commit();
+    };
+    ok = ok && ptx::mbar_wait(bar_acc, 0);
+    ptx::tc_fence_after();
+    // k~: hi plane staged over the A lo plane, lo plane over K (both read by
+    // now: S and k~ are complete)
+    stage_row(sA + NH * kRBox, sK, TQ{});
+    ptx::tc_fence_before();
+    ptx::named_bar(1, 128);
+    if (final_step && lane == 0) ptx::mbar_arrive(bar_free);   // TMEM accumulator read out
+    if (tid == 0 && ok) store_tiles(&maps.kt, sA + NH * kRBox, sK);
+    if (final_step) {
+      ok = ok && ptx::mbar_wait(bar_acc, 1);
+      ptx::tc_fence_after();
+      if (tid == 0) ptx::bulk_wait_read();   // the k~ stores have read their staging
+      ptx::named_bar(1, 128);
+      // z: hi plane over the A hi plane (V is consumed), lo over the A lo plane
+      stage_row(sA, sA + NH * kRBox, __half{});
+      ptx::tc_fence_before();
+      ptx::named_bar(1, 128);
+      if (tid == 0 && ok) store_tiles(&maps.z, sA, sA + NH * kRBox);
+    }
+    if (tid == 0) ptx::bulk_wait_read();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 256);
+}
+
+}  // namespace monarch

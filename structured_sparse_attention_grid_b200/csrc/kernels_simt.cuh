@@ -11,15 +11,40 @@ namespace monarch {
 
 // ---------------------------------------------------------------------------
 // Mean query per (head, position) over all query tiles: the q~ of cached key
-// tiles in the first R step of a KV-cache call.  grid (b2, BH), block d.
+// tiles in the first R step of a KV-cache call.  grid (b2, BH), block
+// kQbarThreads: thread (group, pair) sums column pair `pair` over the query
+// tiles group, group + groups, ... (a warp reads 32 consecutive pairs of one
+// token row), then the groups are added in shared memory.
+constexpr int kQbarThreads = 512;
+
 template <typename T>
-__global__ void qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, Geo g) {
-  const int a2 = blockIdx.x, bh = blockIdx.y, c = threadIdx.x;
-  if (c >= g.d) return;
-  const T* qh = q + (long long)bh * g.Nq * g.d;
-  float acc = 0.f;
-  for (int a1 = 0; a1 < g.b1q; ++a1) acc += to_f(qh[token_of(g, a1, a2) * g.d + c]);
-  qbar[((long long)bh * g.b2 + a2) * g.d + c] = acc / (float)g.b1q;
+__global__ void __launch_bounds__(kQbarThreads)
+qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, Geo g) {
+  __shared__ float2 part[kQbarThreads];
+  const int a2 = blockIdx.x, bh = blockIdx.y;
+  const int npair = g.d / 2, groups = kQbarThreads / npair;
+  const int pair = threadIdx.x % npair, grp = threadIdx.x / npair;
+  const T* qh = q + (long long)bh * g.Nq * g.d + 2 * pair;
+  float2 acc = make_float2(0.f, 0.f);
+#pragma unroll 4
+  for (int a1 = grp; a1 < g.b1q; a1 += groups) {
+    const T* p = qh + token_of(g, a1, a2) * g.d;
+    acc.x += to_f(p[0]);
+    acc.y += to_f(p[1]);
+  }
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  if (grp == 0) {
+    for (int i = 1; i < groups; ++i) {
+      const float2 o = part[i * npair + pair];
+      acc.x += o.x;
+      acc.y += o.y;
+    }
+    const float inv = 1.f / (float)g.b1q;
+    float* dst = qbar + ((long long)bh * g.b2 + a2) * g.d + 2 * pair;
+    dst[0] = acc.x * inv;
+    dst[1] = acc.y * inv;
+  }
 }
 
 // ---------------------------------------------------------------------------

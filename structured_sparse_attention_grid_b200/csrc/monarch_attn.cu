@@ -19,7 +19,7 @@
 #include "common.cuh"
 #include "kernels_simt.cuh"
 #include "kernels_tc.cuh"
-#include "kernels_rstep.cuh"
+#include "kernels_rtc.cuh"
 #include "kernels_l.cuh"
 
 using namespace monarch;
@@ -277,30 +277,33 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
       return rc;
   }
   // R-step maps: the key / value / query grids as (d, W, H, frames) with one
-  // tile per box, and the q~ buffer as (d, b1k, BH*b2) with one key tile per box
-  RMaps rmaps;
+  // tile per box, and the q~ planes as (d, b1k, 2*BH*b2) with one key tile per box
+  RtcMaps rmaps;
   {
     cuuint32_t box4[4] = {64, (cuuint32_t)g.tw, (cuuint32_t)g.th, 1};
     cuuint64_t dk4[4] = {(cuuint64_t)D, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH * g.Tk};
     cuuint64_t dq4[4] = {(cuuint64_t)D, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH * g.T};
     cuuint64_t s4[3] = {(cuuint64_t)D * 2, (cuuint64_t)g.W * D * 2, (cuuint64_t)g.H * g.W * D * 2};
-    cuuint32_t boxt[3] = {32, 1, (cuuint32_t)g.b2};
-    cuuint64_t dt3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, (cuuint64_t)g.BH * g.b2};
-    cuuint64_t st3[2] = {(cuuint64_t)D * 4, (cuuint64_t)g.b1k * D * 4};
+    cuuint32_t boxt[3] = {64, 1, (cuuint32_t)g.b2};
+    cuuint64_t dt3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, 2 * (cuuint64_t)g.BH * g.b2};
+    cuuint64_t st3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1k * D * 2};
     if ((rc = make_map(&rmaps.q, q, dq, 4, dq4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.k, k, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.v, v, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&rmaps.qt, w.qt, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dt3, st3, boxt,
+        (rc = make_map(&rmaps.qt, w.qt, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.kt, planes.kt_hi, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
                        CU_TENSOR_MAP_SWIZZLE_128B)))
       return rc;
+    cuuint64_t db3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, (cuuint64_t)g.BH * g.b2};
+    cuuint64_t sb3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1q * D * 2};
+    if ((rc = make_map(&rmaps.qb, w.qb, dq, 3, db3, sb3, boxt, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
   }
 
   constexpr size_t smem_row = tc::row_smem<D, false>();
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_col = tc::col_smem<D>();
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  constexpr size_t smem_r = rtc_smem<D>();
 
   static bool attrs_set = false;
   if (!attrs_set) {
@@ -308,34 +311,28 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     if ((e = allow_smem(tc::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
         (e = allow_smem(tc::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
         (e = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc<TQ, D>, tc::kMaxSmem)) != cudaSuccess)
+        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
     attrs_set = true;
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);  // two 128-row tiles per CTA
   const dim3 grid_k((g.b1k + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
+  const int r_group = kRtcRows / ((g.b2 + 7) & ~7);   // key tiles per R-step CTA
+  const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
     int mode = QT_BUFFER;
     if (it == 0) {
       mode = p.kv ? QT_KVINIT : QT_IDENTITY;
       if (p.kv)
-        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
+        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), kQbarThreads, 0, st>>>(q, w.qbar, g); });
     } else {
       launch(MONARCH_PHASE_L_COL, st, [&] {
-        tc::l_col<TQ, D><<<grid_k, tc::kThreads, smem_col, st>>>(maps, w.h, w.qt, g);
+        tc::l_col<TQ, D><<<grid_k, tc::kThreads, smem_col, st>>>(maps, w.h, reinterpret_cast<TQ*>(w.qt), g);
       });
     }
-    // persistent R step: a ring of stages within ~113 KB so that two CTAs share an SM
-    const RStepLayout rl = r_step_layout(g.b2, D, mode, final_step);
-    const int stages = std::max(2, std::min(kRMaxStages, (115712 - kRFixedSmem) / rl.stage_bytes));
-    const size_t smem_r = r_step_smem(rl, stages);
-    int occ = 1;
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, r_step_tc<TQ, D>, kRThreads, smem_r);
-    const long long items = (long long)g.BH * ((g.b1k + rl.tp - 1) / rl.tp);
-    const int grid_r = (int)std::min<long long>(items, (long long)std::max(occ, 1) * sms);
     launch(MONARCH_PHASE_R_STEP, st, [&] {
-      r_step_tc<TQ, D><<<grid_r, kRThreads, smem_r, st>>>(rmaps, w, planes, g, mode, final_step, stages);
+      r_step_tc5<TQ, D><<<grid_r, kRtcThreads, smem_r, st>>>(rmaps, q, w, planes, g, mode, final_step);
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
@@ -374,7 +371,7 @@ int run(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* ws, cu
     if (it == 0) {
       mode = p.kv ? QT_KVINIT : QT_IDENTITY;
       if (p.kv)
-        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<T><<<dim3(g.b2, g.BH), g.d, 0, st>>>(q, w.qbar, g); });
+        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<T><<<dim3(g.b2, g.BH), kQbarThreads, 0, st>>>(q, w.qbar, g); });
     } else {
       dim3 grid((g.b1k + kRows - 1) / kRows, g.b2, g.BH);
       launch(MONARCH_PHASE_L_COL, st, [&] {

@@ -27,6 +27,11 @@ __device__ __forceinline__ float2 add2(float2 a, float2 b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
   return u2f(d);
 }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
+  return u2f(d);
+}
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   uint64_t d;
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2u(a)), "l"(f2u(b)));
@@ -70,6 +75,15 @@ __device__ __forceinline__ void split2(float2 p, uint32_t& hi, uint32_t& lo) {
   }
   const float2 r = sub2(p, h);
   lo = TcType<TQ>::pack(r.x, r.y);
+}
+
+// Dynamic shared memory starts 1024-byte aligned (no static shared memory in
+// these kernels); the 128-byte swizzle of the TMA boxes needs that.  A kernel
+// that finds otherwise records kErrSmemAlign and returns before any TMA.
+__device__ __forceinline__ bool smem_misaligned(const void* p) {
+  if ((ptx::smem_u32(p) & 1023u) == 0) return false;
+  if (threadIdx.x == 0) atomicExch(&ptx::g_device_error, ptx::kErrSmemAlign);
+  return true;
 }
 
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
