@@ -416,9 +416,235 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
 }
 
 // ===========================================================================
+// LSE pass over 128-key blocks for one (head, position a2, 256 query rows):
+//   lse[a1] = log2 sum_c1 2^(s q.k~ + h)
+// with k~ rounded once to f16 (the hi plane) and q exact in f16: the row sums
+// only weight whole rows in the column pass, and this rounding keeps the
+// result within the tolerance (a fp64 replay of the GPU roundings shows it).
+// S = q k~_hi^T is one N = 128 MMA group per (tile, block); TMEM: tile t,
+// buffer b at column 256 t + 128 b, so block j + 1 is computed while the
+// softmax reads block j.  The two column halves of a row keep their own
+// running shift and sum and are merged at the end.  About 3/8 of the
+// exponentials run on the FMA pipe (ex2_fma2): with one plane the score MMA
+// has half the columns per exponential of the two-plane passes, so the MUFU
+// unit alone would be the bound.
+constexpr int kLBlk = 128;   // keys per LSE-pass block
+constexpr int kLS = 3;       // k~ / h stages
+
+template <int D>
+constexpr size_t lse_smem() {
+  constexpr int NH = D / 64;
+  constexpr size_t need = (size_t)2 * NH * 2 * kBox /* q */ + (size_t)kLS * NH * 2 * kBox /* k~ hi */ +
+                          kLS * kLBlk * 4 + 2 * xchg_tile_bytes<0>() + 32 * 8;
+  return need > kExclusiveSmem ? need : kExclusiveSmem;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t kQt = NH * 2 * kBox;    // q of one tile: [d half][128 rows]
+  constexpr uint32_t kKst = NH * 2 * kBox;   // k~ hi of one block: [d half][128 keys]
+  constexpr int kXt = xchg_tile_bytes<0>();
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_misaligned(smem_raw)) return;
+  uint8_t* sQ = smem_raw;                                      // [2 tiles]
+  uint8_t* sK = sQ + 2 * kQt;                                  // [kLS]
+  float* sH = reinterpret_cast<float*>(sK + kLS * kKst);       // [kLS][128]
+  uint8_t* sX = reinterpret_cast<uint8_t*>(sH + kLS * kLBlk);  // [tile][kXt bytes]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * kXt);
+  uint64_t* q_full = bar + 0;
+  uint64_t* k_full = bar + 1;    // [kLS]
+  uint64_t* k_free = bar + 4;    // [kLS]
+  uint64_t* s_full = bar + 7;    // [tile][buf]
+  uint64_t* s_free = bar + 11;   // [tile][buf]
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 15);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int a2 = blockIdx.y, bh = blockIdx.z;
+  const int a1_base = blockIdx.x * 2 * kTile;
+  const int zrow = bh * g.b2 + a2;
+  const int nkb = (g.b1k + kLBlk - 1) / kLBlk;
+  const int ntiles = (g.b1q - a1_base > kTile) ? 2 : 1;
+
+  if (tid == 0) {
+    ptx::mbar_init(q_full, 1);
+    for (int i = 0; i < kLS; ++i) {
+      ptx::mbar_init(k_full + i, 1);
+      ptx::mbar_init(k_free + i, 8 * ntiles);
+    }
+    for (int i = 0; i < 4; ++i) {
+      ptx::mbar_init(s_full + i, 1);
+      ptx::mbar_init(s_free + i, 8);
+    }
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *sTmem;
+  auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      // --------------------------------------------------------- TMA producer
+      ptx::prefetch_tmap(&maps.kt);
+      ptx::mbar_expect_tx(q_full, 2 * kQt);
+      for (int t = 0; t < 2; ++t)
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh)
+            ptx::tma_load_3d(sQ + t * kQt + hf * 2 * kBox + rh * kBox, &maps.qb, q_full, hf * 64,
+                             a1_base + t * kTile + rh * kBlk, zrow);
+      bool ok = true;
+      for (int blk = 0; blk < nkb && ok; ++blk) {
+        const int ks = blk % kLS;
+        if (blk >= kLS) ok = ptx::mbar_wait(k_free + ks, ((blk / kLS) - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(k_full + ks, kKst + kLBlk * 4);
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh)
+            ptx::tma_load_3d(sK + ks * kKst + hf * 2 * kBox + rh * kBox, &maps.kt, k_full + ks, hf * 64,
+                             blk * kLBlk + rh * kBlk, zrow);
+        for (int rh = 0; rh < 2; ++rh)
+          tma_load_2d(sH + ks * kLBlk + rh * kBlk, &maps.h, k_full + ks, blk * kLBlk + rh * kBlk, zrow);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
+      constexpr uint32_t idS = ptx::idesc_f16(128, kLBlk, 0, 0, 0);
+      const uint32_t aQ = ptx::smem_u32(sQ), aK = ptx::smem_u32(sK);
+      auto issue_s = [&](int t, int blk, int b) {
+        const uint64_t a0 = ptx::sw128_desc(aQ + t * kQt, 16, 1024);
+        const uint64_t b0 = ptx::sw128_desc(aK + (blk % kLS) * kKst, 16, 1024);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ptx::mma_f16_ss(tS(t, b), a0 + ((hf * 2 * kBox + k4 * 32) >> 4), b0 + ((hf * 2 * kBox + k4 * 32) >> 4),
+                            idS, (hf | k4) != 0);
+        ptx::mma_commit(s_full + 2 * t + b);
+      };
+      bool ok = ptx::mbar_wait(q_full, 0) && ptx::mbar_wait(k_full, 0);
+      ptx::tc_fence_after();
+      if (ok) {
+        for (int t = 0; t < ntiles; ++t) issue_s(t, 0, 0);
+        if (nkb > 1) {
+          ok = ptx::mbar_wait(k_full + 1, 0);
+          ptx::tc_fence_after();
+          if (ok)
+            for (int t = 0; t < ntiles; ++t) issue_s(t, 1, 1);
+        }
+      }
+      for (int j = 0; j < nkb && ok; ++j) {
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        for (int t = 0; t < ntiles && ok; ++t) {
+          ok = ptx::mbar_wait(s_free + 2 * t + b, ph);
+          if (ok && j + 2 < nkb) {
+            ok = ptx::mbar_wait(k_full + (j + 2) % kLS, ((j + 2) / kLS) & 1);
+            ptx::tc_fence_after();
+            if (ok) issue_s(t, j + 2, b);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------- softmax warps
+    const int t = warp >> 3;                 // tile
+    const int hf = (warp >> 2) & 1;          // column half: keys 64 hf .. 64 hf + 63 of a block
+    const int r = 32 * (warp & 3) + lane;
+    const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
+    const int a1 = a1_base + t * kTile + r;
+    if (t < ntiles) {
+      float m = -INFINITY, l = 0.f;
+      bool ok = true;
+      const float2 sl2 = make_float2(g.sl2, g.sl2);
+      for (int j = 0; j < nkb; ++j) {
+        const int ks = j % kLS;
+        const int b = j & 1;
+        const uint32_t ph = (j >> 1) & 1;
+        ok = ok && ptx::mbar_wait(s_full + 2 * t + b, ph) && ptx::mbar_wait(k_full + ks, (j / kLS) & 1);
+        ptx::tc_fence_after();
+        const float4* hv = reinterpret_cast<const float4*>(sH + ks * kLBlk + 64 * hf);
+#pragma unroll
+        for (int sb = 0; sb < 2; ++sb) {   // 32 keys at a time: an online update each
+          uint32_t s[32];
+          ptx::tmem_ld32(tS(t, b) + lane_off + 64 * hf + 32 * sb, s);
+          ptx::tmem_wait_ld();
+          float2 x[16];   // x[i] = keys 64 hf + 32 sb + 2i, + 1
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 h4 = hv[8 * sb + i];
+            x[2 * i] = fma2(make_float2(__uint_as_float(s[4 * i]), __uint_as_float(s[4 * i + 1])), sl2,
+                            make_float2(h4.x, h4.y));
+            x[2 * i + 1] = fma2(make_float2(__uint_as_float(s[4 * i + 2]), __uint_as_float(s[4 * i + 3])), sl2,
+                                make_float2(h4.z, h4.w));
+          }
+          if (sb == 1) {
+            // S and h of this block are read: release the k~/h stage and the S buffer
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::mbar_arrive(k_free + ks);
+              ptx::mbar_arrive(s_free + 2 * t + b);
+            }
+          }
+          const int valid = min(kLBlk, g.b1k - j * kLBlk) - 64 * hf - 32 * sb;
+          if (valid < 32) {  // only the last block of a ragged row
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              if (2 * i >= valid) x[i].x = -INFINITY;
+              if (2 * i + 1 >= valid) x[i].y = -INFINITY;
+            }
+          }
+          float mb = -INFINITY;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) mb = fmaxf(mb, fmaxf(x[i].x, x[i].y));
+          const bool move = mb > m + kLazyRescale;
+          const float mn = move ? mb : m;
+          const float corr = (mn == m) ? 1.f : ptx::ex2(m - mn);
+          const float nmv = (mn == -INFINITY) ? 0.f : -mn;   // a half with no key yet
+          const float2 nm = make_float2(nmv, nmv);
+          float2 acc2 = make_float2(0.f, 0.f);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float2 d = add2(x[i], nm);
+            // three pairs in eight on the FMA pipe, the rest on the MUFU unit
+            const float2 e = ((i & 7) >= 5) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
+            acc2 = add2(acc2, e);
+          }
+          l = fmaf(l, corr, acc2.x + acc2.y);
+          m = mn;
+        }
+      }
+      // merge the halves: (m, l) of each, shifts may differ
+      float* xs = reinterpret_cast<float*>(sX + t * kXt);   // [m, l][half][128]
+      xs[hf * kTile + r] = m;
+      xs[2 * kTile + hf * kTile + r] = l;
+      ptx::named_bar(1 + t, kTileThreads);
+      if (hf == 0 && a1 < g.b1q) {
+        const float mo = xs[kTile + r], lo = xs[3 * kTile + r];
+        const float M = fmaxf(m, mo);
+        const float L = (m == -INFINITY ? 0.f : l * ptx::ex2(m - M)) + (mo == -INFINITY ? 0.f : lo * ptx::ex2(mo - M));
+        lse[(long long)zrow * g.b1q_pad + a1] = M + log2f(L);
+      }
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ===========================================================================
 // Column pass for one (head, position a2, 256 key tiles), 128 queries per block:
 //   q~[c1,a2] = sum_a1 L q / sum_a1 L,  L = 2^(s q.k~ + h - lse[a1]),
-// stored as hi / lo planes of the input type ([plane][BH][b2][b1k][d]).
+// with q, k~ and L in f16 and q~ stored as hi / lo planes of the input type TQ
+// ([plane][BH][b2][b1k][d]), the A operand of the next R step.
 // TMEM, tile t at column 256 t:  S^T [0, 128) for 128 queries; P^T is written
 // over it per 32-query chunk c as [hi | lo] in columns [32 c, 32 c + 32)
 // (16 columns each, two queries per column);  acc [128, 128 + D).
@@ -510,8 +736,8 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idS = ptx::idesc_f16(128, kQBlk, TcType<TQ>::kBf16, 0, 0);
-      constexpr uint32_t idPQ = ptx::idesc_f16(128, D, TcType<TQ>::kBf16, 0, 1);
+      constexpr uint32_t idS = ptx::idesc_f16(128, kQBlk, 0, 0, 0);   // f16 operands
+      constexpr uint32_t idPQ = ptx::idesc_f16(128, D, 0, 0, 1);
       const uint32_t aK = ptx::smem_u32(sK), aQ = ptx::smem_u32(sQ);
       auto issue_s = [&](int t, int blk) {
         const uint64_t a0 = ptx::sw128_desc(aK + t * kKt, 16, 1024);
@@ -599,8 +825,8 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
               if (q0 + 3 >= valid) p1.y = 0.f;
             }
             beta2 = add2(beta2, add2(p0, p1));
-            split2<TQ>(p0, hi[2 * e], lo[2 * e]);
-            split2<TQ>(p1, hi[2 * e + 1], lo[2 * e + 1]);
+            split2<__half>(p0, hi[2 * e], lo[2 * e]);
+            split2<__half>(p1, hi[2 * e + 1], lo[2 * e + 1]);
           }
           // P^T of these 32 queries over the chunk's own S^T columns:
           // hi in [cb, cb + 16), lo in [cb + 16, cb + 32)

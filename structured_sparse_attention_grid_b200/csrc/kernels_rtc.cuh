@@ -40,15 +40,15 @@ struct RtcMaps {
   CUtensorMap k;    // keys       {d, W, H, BH*Tk},       box {64, tw, th, 1}
   CUtensorMap v;    // values     {d, W, H, BH*Tk},       box {64, tw, th, 1}
   CUtensorMap qt;   // q~ planes  {d, b1k, 2*BH*b2},      box {64, 1, b2}
-  CUtensorMap qb;   // block-major q (store) {d, b1q, BH*b2},     box {64, 1, b2}
-  CUtensorMap kt;   // k~ planes (store)     {d, b1k, 2*BH*b2},   box {64, 1, b2}
+  CUtensorMap qb;   // block-major q, f16 (store) {d, b1q, BH*b2},   box {64, 1, b2}
+  CUtensorMap kt;   // k~ planes, f16 (store)     {d, b1k, 2*BH*b2}, box {64, 1, b2}
   CUtensorMap z;    // z planes, f16 (store) {d, b1k, 2*BH*b2},   box {64, 1, b2}
 };
 
 // Planes written by the R step.
 template <typename TQ>
 struct TcPlanes {
-  TQ* kt_hi;        // [BH][b2][b1k][d], then the lo plane at kt_hi + plane
+  __half* kt_hi;    // [BH][b2][b1k][d], then the lo plane at kt_hi + plane
   __half* z_hi;     // [BH][b2][b1k][d], then the lo plane
   long long plane;  // elements per plane
 };
@@ -60,7 +60,7 @@ constexpr uint32_t kRBox = 128 * 128; // one [128 rows][128 B] swizzled box
 // At least 80 KB so that at most two CTAs (2 x 256 TMEM columns) share an SM.
 template <int D>
 constexpr size_t rtc_smem() {
-  constexpr size_t need = (size_t)3 * (D / 64) * kRBox + 8 * 8;
+  constexpr size_t need = (size_t)3 * (D / 64) * kRBox + 16 * 8;
   return need > 80 * 1024 ? need : 80 * 1024;
 }
 
@@ -83,7 +83,8 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   uint64_t* bar_acc = bar + 4;   // MMA: k~ (phase 0), z (phase 1) complete
   uint64_t* bar_free = bar + 5;  // row warps: k~ read out of TMEM
   uint64_t* bar_v = bar + 6;     // TMA: values
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 7);
+  uint64_t* bar_q = bar + 7;     // row warps: query rows read (first step, bf16, before V lands)
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -100,6 +101,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     ptx::mbar_init(bar_acc, 1);
     ptx::mbar_init(bar_free, 4);
     ptx::mbar_init(bar_v, 1);
+    ptx::mbar_init(bar_q, 4);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -166,9 +168,9 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         }
       }
       ok = ptx::mbar_wait(bar_ld, 0);
-      if (ok && mode != QT_BUFFER) {
-        // first step: the exact query rows just loaded are also the block-major
-        // copy of q that the L step reads
+      if (ok && mode != QT_BUFFER && !bf16) {
+        // first step, f16 input: the exact query rows just loaded are also the
+        // block-major copy of q that the L step reads
         for (int gg = 0; gg < Gn; ++gg) {
           const int c1 = c1_0 + gg;
           if (!exact_q(c1)) continue;
@@ -200,6 +202,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         // V lands in the A hi plane once the score MMAs and the q copy (its
         // readers) are done
         ok = ok && ptx::mbar_wait(bar_s, 0);
+        if (bf16 && mode != QT_BUFFER) ok = ok && ptx::mbar_wait(bar_q, 0);
         ptx::bulk_wait_read();
         if (ok) {
           ptx::mbar_expect_tx(bar_v, (uint32_t)(Gn * NH * g.b2 * 128));
@@ -278,6 +281,45 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     // are read from TMEM once and kept in registers.
     ok = ptx::mbar_wait(bar_s, 0);
     ptx::tc_fence_after();
+    if (bf16 && mode != QT_BUFFER) {
+      // first step, bf16 input: the L step reads q in f16 (exact for |q| <
+      // 65504; larger magnitudes set kErrRange).  Convert the loaded rows into
+      // the A lo plane, free once S is done, and store them from there.
+      if (valid && exact_q(c1)) {
+        bool over = false;
+#pragma unroll 1
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+            uint4 u = *reinterpret_cast<const uint4*>(sA + o);
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+              const __half2 hv = __floats2half2_rn(f.x, f.y);
+              const float2 back = __half22float2(hv);
+              over |= (isinf(back.x) && !isinf(f.x)) || (isinf(back.y) && !isinf(f.y));
+              wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
+          }
+        if (over) atomicExch(&ptx::g_device_error, ptx::kErrRange);
+      }
+      ptx::fence_proxy_async();
+      __syncwarp();
+      if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
+      ptx::named_bar(1, 128);
+      if (tid == 0 && ok) {
+        for (int t = 0; t < Gn; ++t) {
+          if (!exact_q(c1_0 + t)) continue;
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * r8) * 128, hf * 64,
+                              c1_0 + t - g.off, bh * g.b2);
+        }
+        ptx::bulk_commit();
+      }
+    }
     const int cb = gg * r8;
     const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
     const int ch_lo = (wg0 * r8) >> 5, ch_hi = min((wg1 * r8 + g.b2 - 1) >> 5, 3);
@@ -371,9 +413,13 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     };
     ok = ok && ptx::mbar_wait(bar_acc, 0);
     ptx::tc_fence_after();
-    // k~: hi plane staged over the A lo plane, lo plane over K (both read by
-    // now: S and k~ are complete)
-    stage_row(sA + NH * kRBox, sK, TQ{});
+    if (bf16 && mode != QT_BUFFER) {
+      if (tid == 0) ptx::bulk_wait_read();   // the q copy has read the A lo plane
+      ptx::named_bar(1, 128);
+    }
+    // k~ (f16 planes): hi plane staged over the A lo plane, lo plane over K
+    // (both read by now: S and k~ are complete)
+    stage_row(sA + NH * kRBox, sK, __half{});
     ptx::tc_fence_before();
     ptx::named_bar(1, 128);
     if (final_step && lane == 0) ptx::mbar_arrive(bar_free);   // TMEM accumulator read out

@@ -247,7 +247,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
   w.qb = ws + p.off[6];
   TcPlanes<TQ> planes;
-  planes.kt_hi = reinterpret_cast<TQ*>(w.kt);
+  planes.kt_hi = reinterpret_cast<__half*>(w.kt);
   planes.z_hi = reinterpret_cast<__half*>(w.z);
   planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
 
@@ -267,8 +267,11 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     cuuint64_t sh2[1] = {(cuuint64_t)g.b1k_pad * 4};
     cuuint64_t dl2[2] = {(cuuint64_t)g.b1q_pad, rows};
     cuuint64_t sl2[1] = {(cuuint64_t)g.b1q_pad * 4};
-    if ((rc = make_map(&maps.qb, w.qb, dq, 3, dq3, sq3, box3, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&maps.kt, planes.kt_hi, dq, 3, dk3, sk3, box3, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+    // the L step computes in f16: q (block-major copy) and the k~ planes are f16
+    if ((rc = make_map(&maps.qb, w.qb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dq3, sq3, box3,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&maps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&maps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&maps.h, w.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dh2, sh2, box2, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
@@ -291,16 +294,19 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         (rc = make_map(&rmaps.k, k, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.v, v, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.qt, w.qt, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&rmaps.kt, planes.kt_hi, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
                        CU_TENSOR_MAP_SWIZZLE_128B)))
       return rc;
     cuuint64_t db3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, (cuuint64_t)g.BH * g.b2};
     cuuint64_t sb3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1q * D * 2};
-    if ((rc = make_map(&rmaps.qb, w.qb, dq, 3, db3, sb3, boxt, CU_TENSOR_MAP_SWIZZLE_128B))) return rc;
+    if ((rc = make_map(&rmaps.qb, w.qb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, db3, sb3, boxt,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
   }
 
-  constexpr size_t smem_row = tc::row_smem<D, false>();
+  constexpr size_t smem_lse = tc::lse_smem<D>();
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_col = tc::col_smem<D>();
   constexpr size_t smem_r = rtc_smem<D>();
@@ -308,8 +314,8 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   static bool attrs_set = false;
   if (!attrs_set) {
     cudaError_t e;
-    if ((e = allow_smem(tc::l_row<TQ, TO, D, false>, smem_row)) != cudaSuccess ||
-        (e = allow_smem(tc::l_row<TQ, TO, D, true>, smem_out)) != cudaSuccess ||
+    if ((e = allow_smem(tc::l_lse<D>, smem_lse)) != cudaSuccess ||
+        (e = allow_smem(tc::l_row<__half, TO, D, true>, smem_out)) != cudaSuccess ||
         (e = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
         (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
@@ -336,11 +342,11 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
-        tc::l_row<TQ, TO, D, true><<<grid_q, tc::kThreads, smem_out, st>>>(out, maps, w.lse, g);
+        tc::l_row<__half, TO, D, true><<<grid_q, tc::kThreads, smem_out, st>>>(out, maps, w.lse, g);
       });
     } else {
       launch(MONARCH_PHASE_L_ROW, st, [&] {
-        tc::l_row<TQ, TO, D, false><<<grid_q, tc::kThreads, smem_row, st>>>(out, maps, w.lse, g);
+        tc::l_lse<D><<<grid_q, tc::kThreads, smem_lse, st>>>(maps, w.lse, g);
       });
     }
   }

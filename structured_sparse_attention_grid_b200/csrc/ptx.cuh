@@ -12,7 +12,7 @@ namespace ptx {
 // Set by a kernel whose bounded wait gave up; read by the host on request.
 __device__ int g_device_error;
 
-enum DeviceError : int { kErrMbarTimeout = 1, kErrSmemAlign = 2 };
+enum DeviceError : int { kErrMbarTimeout = 1, kErrSmemAlign = 2, kErrRange = 3 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
