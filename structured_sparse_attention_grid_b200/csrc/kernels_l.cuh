@@ -652,7 +652,7 @@ template <int D>
 constexpr size_t col_smem() {
   constexpr int NH = D / 64;
   constexpr size_t need = (size_t)2 * 2 * NH * 2 * kBox /* k~ */ + (size_t)kQS * NH * 2 * kBox /* q */ +
-                          kQS * kQBlk * 4 + 2 * xchg_tile_bytes<2>() + 32 * 8;
+                          kQS * kQBlk * 4 + 2 * 2 * xchg_tile_bytes<2>() + 32 * 8;
   return need > kExclusiveSmem ? need : kExclusiveSmem;
 }
 
@@ -667,26 +667,33 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   uint8_t* sK = smem_raw;                                    // [2 tiles]
   uint8_t* sQ = sK + 2 * kKt;                                // [kQS]
   float* sL = reinterpret_cast<float*>(sQ + kQS * kQst);     // [kQS][128]
-  float* sX = sL + kQS * kQBlk;                              // [tile][half][128]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * xchg_tile_bytes<2>() / 4);
+  float* sX = sL + kQS * kQBlk;                              // [item parity][tile][half][128]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * 2 * xchg_tile_bytes<2>() / 4);
   uint64_t* k_full = bar + 0;
-  uint64_t* q_full = bar + 1;    // [kQS]
-  uint64_t* q_free = bar + 3;    // [kQS]
-  uint64_t* s_full = bar + 5;    // [tile]
-  uint64_t* p_full = bar + 7;    // [tile]
-  uint64_t* o_done = bar + 9;    // [tile]
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 11);
+  uint64_t* k_empty = bar + 1;   // the score MMAs of an item are done with sK
+  uint64_t* q_full = bar + 2;    // [kQS]
+  uint64_t* q_free = bar + 4;    // [kQS]
+  uint64_t* s_full = bar + 6;    // [tile]
+  uint64_t* p_full = bar + 8;    // [tile]
+  uint64_t* o_done = bar + 10;   // [tile]
+  uint64_t* acc_free = bar + 12; // [tile] the epilogue has read the accumulator
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 14);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int a2 = blockIdx.y, bh = blockIdx.z;
-  const int kb = blockIdx.x * 2 * kTile;
-  const int zrow = bh * g.b2 + a2;
   const int plane_rows = g.BH * g.b2;
   const int nqb = (g.b1q + kQBlk - 1) / kQBlk;
-  const int ntiles = (g.b1k - kb > kTile) ? 2 : 1;
+  const int nchunk = (g.b1k + 2 * kTile - 1) / (2 * kTile);
+  const int n_items = g.BH * g.b2 * nchunk;
+  // item -> (row of the [BH][b2] planes, first key tile, tiles in it)
+  auto item_of = [&](int it, int& zrow, int& kb, int& ntiles) {
+    zrow = it / nchunk;
+    kb = (it - zrow * nchunk) * 2 * kTile;
+    ntiles = (g.b1k - kb > kTile) ? 2 : 1;
+  };
 
   if (tid == 0) {
     ptx::mbar_init(k_full, 1);
+    ptx::mbar_init(k_empty, 1);
     for (int i = 0; i < kQS; ++i) {
       ptx::mbar_init(q_full + i, 1);
       ptx::mbar_init(q_free + i, 1);
@@ -695,6 +702,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
       ptx::mbar_init(s_full + t, 1);
       ptx::mbar_init(p_full + t, 8);
       ptx::mbar_init(o_done + t, 1);
+      ptx::mbar_init(acc_free + t, 8);
     }
     ptx::fence_mbar_init();
   }
@@ -711,37 +719,46 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
 
   if (warp == kLoadWarp) {
     if (lane == 0) {
+      // --------------------------------------------------------- TMA producer
       ptx::prefetch_tmap(&maps.kt);
       ptx::prefetch_tmap(&maps.qb);
-      ptx::mbar_expect_tx(k_full, 2 * kKt);
-      for (int t = 0; t < 2; ++t)
-        for (int p = 0; p < 2; ++p)
+      bool ok = true;
+      int gq = 0, ni = 0;   // query blocks and items loaded so far
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ni) {
+        int zrow, kb, ntiles;
+        item_of(it, zrow, kb, ntiles);
+        if (ni > 0) ok = ptx::mbar_wait(k_empty, (ni - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(k_full, 2 * kKt);
+        for (int t = 0; t < 2; ++t)
+          for (int p = 0; p < 2; ++p)
+            for (int hf = 0; hf < NH; ++hf)
+              for (int rh = 0; rh < 2; ++rh)
+                ptx::tma_load_3d(sK + t * kKt + (p * NH + hf) * 2 * kBox + rh * kBox, &maps.kt, k_full, hf * 64,
+                                 kb + t * kTile + rh * kBlk, p * plane_rows + zrow);
+        for (int blk = 0; blk < nqb && ok; ++blk, ++gq) {
+          const int qs = gq % kQS;
+          if (gq >= kQS) ok = ptx::mbar_wait(q_free + qs, ((gq / kQS) - 1) & 1);
+          if (!ok) break;
+          ptx::mbar_expect_tx(q_full + qs, kQst + kQBlk * 4);
           for (int hf = 0; hf < NH; ++hf)
             for (int rh = 0; rh < 2; ++rh)
-              ptx::tma_load_3d(sK + t * kKt + (p * NH + hf) * 2 * kBox + rh * kBox, &maps.kt, k_full, hf * 64,
-                               kb + t * kTile + rh * kBlk, p * plane_rows + zrow);
-      bool ok = true;
-      for (int blk = 0; blk < nqb && ok; ++blk) {
-        const int qs = blk % kQS;
-        if (blk >= kQS) ok = ptx::mbar_wait(q_free + qs, ((blk / kQS) - 1) & 1);
-        if (!ok) break;
-        ptx::mbar_expect_tx(q_full + qs, kQst + kQBlk * 4);
-        for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_load_3d(sQ + qs * kQst + hf * 2 * kBox + rh * kBox, &maps.qb, q_full + qs, hf * 64,
+                               blk * kQBlk + rh * kBlk, zrow);
           for (int rh = 0; rh < 2; ++rh)
-            ptx::tma_load_3d(sQ + qs * kQst + hf * 2 * kBox + rh * kBox, &maps.qb, q_full + qs, hf * 64,
-                             blk * kQBlk + rh * kBlk, zrow);
-        for (int rh = 0; rh < 2; ++rh)
-          tma_load_2d(sL + qs * kQBlk + rh * kBlk, &maps.lse, q_full + qs, blk * kQBlk + rh * kBlk, zrow);
+            tma_load_2d(sL + qs * kQBlk + rh * kBlk, &maps.lse, q_full + qs, blk * kQBlk + rh * kBlk, zrow);
+        }
       }
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
+      // ----------------------------------------------------------- MMA issuer
       constexpr uint32_t idS = ptx::idesc_f16(128, kQBlk, 0, 0, 0);   // f16 operands
       constexpr uint32_t idPQ = ptx::idesc_f16(128, D, 0, 0, 1);
       const uint32_t aK = ptx::smem_u32(sK), aQ = ptx::smem_u32(sQ);
-      auto issue_s = [&](int t, int blk) {
+      auto issue_s = [&](int t, int gblk) {
         const uint64_t a0 = ptx::sw128_desc(aK + t * kKt, 16, 1024);
-        const uint64_t b0 = ptx::sw128_desc(aQ + (blk % kQS) * kQst, 16, 1024);
+        const uint64_t b0 = ptx::sw128_desc(aQ + (gblk % kQS) * kQst, 16, 1024);
         const uint32_t td = tS(t);
 #pragma unroll
         for (int p = 0; p < 2; ++p)
@@ -753,34 +770,52 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
                               b0 + ((hf * 2 * kBox + k4 * 32) >> 4), idS, (p | hf | k4) != 0);
         ptx::mma_commit(s_full + t);
       };
-      bool ok = ptx::mbar_wait(k_full, 0) && ptx::mbar_wait(q_full, 0);
-      ptx::tc_fence_after();
-      if (ok)
-        for (int t = 0; t < ntiles; ++t) issue_s(t, 0);
-      for (int i = 0; i < nqb && ok; ++i) {
-        const int qs = i % kQS;
-        const uint64_t q0 = ptx::sw128_desc(aQ + qs * kQst, 2 * kBox, 1024);
-        for (int t = 0; t < ntiles && ok; ++t) {
-          ok = ptx::mbar_wait(p_full + t, i & 1);
-          ptx::tc_fence_after();
-          if (!ok) break;
-          const uint32_t tp = tS(t);
-#pragma unroll
-          for (int p = 0; p < 2; ++p)
-#pragma unroll
-            for (int kk = 0; kk < kQBlk / 16; ++kk)
-              ptx::mma_f16_ts(tA(t), tp + (kk >> 1) * 32 + p * 16 + (kk & 1) * 8, q0 + ((kk * 2048) >> 4), idPQ,
-                              (i | p | kk) != 0);
-          if (t == ntiles - 1) ptx::mma_commit(q_free + qs);
-          if (i + 1 < nqb) {
-            // S^T(t, i+1) overwrites P^T(t, i): the P^T q product above runs first
-            ok = ptx::mbar_wait(q_full + (i + 1) % kQS, ((i + 1) / kQS) & 1);
+      bool ok = true;
+      int gq = 0, ni = 0;
+      int cnt0 = 0, cnt1 = 0, icnt0 = 0, icnt1 = 0;   // blocks / items processed per tile
+      for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ni) {
+        int zrow, kb, ntiles;
+        item_of(it, zrow, kb, ntiles);
+        ok = ptx::mbar_wait(k_full, ni & 1) && ptx::mbar_wait(q_full + gq % kQS, (gq / kQS) & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
+        for (int t = 0; t < ntiles; ++t) issue_s(t, gq);
+        if (nqb == 1) ptx::mma_commit(k_empty);
+        for (int i = 0; i < nqb && ok; ++i) {
+          const int qs = (gq + i) % kQS;
+          const uint64_t q0 = ptx::sw128_desc(aQ + qs * kQst, 2 * kBox, 1024);
+          for (int t = 0; t < ntiles && ok; ++t) {
+            const int ct = t ? cnt1 : cnt0, it_t = t ? icnt1 : icnt0;
+            ok = ptx::mbar_wait(p_full + t, ct & 1);
+            // the first product of an item overwrites the accumulator the
+            // previous item's epilogue reads
+            if (ok && i == 0 && it_t > 0) ok = ptx::mbar_wait(acc_free + t, (it_t - 1) & 1);
             ptx::tc_fence_after();
-            if (ok) issue_s(t, i + 1);
-          } else {
-            ptx::mma_commit(o_done + t);
+            if (!ok) break;
+            const uint32_t tp = tS(t);
+#pragma unroll
+            for (int p = 0; p < 2; ++p)
+#pragma unroll
+              for (int kk = 0; kk < kQBlk / 16; ++kk)
+                ptx::mma_f16_ts(tA(t), tp + (kk >> 1) * 32 + p * 16 + (kk & 1) * 8, q0 + ((kk * 2048) >> 4), idPQ,
+                                (i | p | kk) != 0);
+            if (t == ntiles - 1) ptx::mma_commit(q_free + qs);
+            if (i + 1 < nqb) {
+              // S^T(t, i+1) overwrites P^T(t, i): the P^T q product above runs first
+              ok = ptx::mbar_wait(q_full + (gq + i + 1) % kQS, ((gq + i + 1) / kQS) & 1);
+              ptx::tc_fence_after();
+              if (ok) issue_s(t, gq + i + 1);
+            } else {
+              ptx::mma_commit(o_done + t);
+            }
+            if (t) ++cnt1; else ++cnt0;
           }
+          // after the item's last score MMA, sK may take the next item's tiles
+          if (i + 2 == nqb) ptx::mma_commit(k_empty);
         }
+        ++icnt0;
+        if (ntiles > 1) ++icnt1;
+        gq += nqb;
       }
     }
   } else {
@@ -788,86 +823,103 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
     const int hf = (warp >> 2) & 1;          // column half: queries 64 hf .. 64 hf + 63 of a block
     const int r = 32 * (warp & 3) + lane;    // key tile row / TMEM lane
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
-    const int c1 = kb + t * kTile + r;
-    if (t < ntiles) {
-      const float hb = (c1 < g.b1k) ? hbuf[(long long)zrow * g.b1k_pad + c1] + kColShift : 0.f;
-      const float2 sl2 = make_float2(g.sl2, g.sl2), hb2 = make_float2(hb, hb);
-      float2 beta2 = make_float2(0.f, 0.f);
-      bool ok = true;
-      for (int i = 0; i < nqb; ++i) {
-        const int qs = i % kQS;
-        ok = ok && ptx::mbar_wait(s_full + t, i & 1) && ptx::mbar_wait(q_full + qs, (i / kQS) & 1);
-        ptx::tc_fence_after();
-        const int valid = min(kQBlk, g.b1q - i * kQBlk);
+    const float2 sl2 = make_float2(g.sl2, g.sl2);
+    const long long plane = (long long)g.BH * g.b2 * g.b1k * D;
+    bool ok = true;
+    int gq = 0, cnt = 0, icnt = 0;
+    for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
+      int zrow, kb, ntiles;
+      item_of(it, zrow, kb, ntiles);
+      if (t < ntiles) {
+        const int c1 = kb + t * kTile + r;
+        const float hb = (c1 < g.b1k) ? hbuf[(long long)zrow * g.b1k_pad + c1] + kColShift : 0.f;
+        const float2 hb2 = make_float2(hb, hb);
+        float2 beta2 = make_float2(0.f, 0.f);
+        for (int i = 0; i < nqb; ++i, ++cnt) {
+          const int qs = (gq + i) % kQS;
+          ok = ok && ptx::mbar_wait(s_full + t, cnt & 1) && ptx::mbar_wait(q_full + qs, ((gq + i) / kQS) & 1);
+          ptx::tc_fence_after();
+          const int valid = min(kQBlk, g.b1q - i * kQBlk);
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {  // 32 queries at a time
-          const int cb = 64 * hf + 32 * hh;   // first S^T column (query) of this chunk
-          uint32_t sr[32];
-          ptx::tmem_ld32(tS(t) + lane_off + cb, sr);
-          const float4* lv = reinterpret_cast<const float4*>(sL + qs * kQBlk + cb);
-          ptx::tmem_wait_ld();
-          uint32_t hi[16], lo[16];
+          for (int hh = 0; hh < 2; ++hh) {  // 32 queries at a time
+            const int cb = 64 * hf + 32 * hh;   // first S^T column (query) of this chunk
+            uint32_t sr[32];
+            ptx::tmem_ld32(tS(t) + lane_off + cb, sr);
+            const float4* lv = reinterpret_cast<const float4*>(sL + qs * kQBlk + cb);
+            ptx::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float4 l4 = lv[e];
-            float2 x0 = fma2(make_float2(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1])), sl2, hb2);
-            float2 x1 =
-                fma2(make_float2(__uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3])), sl2, hb2);
-            x0 = sub2(x0, make_float2(l4.x, l4.y));
-            x1 = sub2(x1, make_float2(l4.z, l4.w));
-            float2 p0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
-            float2 p1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
-            if (valid < kQBlk) {  // only the last block of a ragged column
-              const int q0 = cb + 4 * e;
-              if (q0 >= valid) p0.x = 0.f;
-              if (q0 + 1 >= valid) p0.y = 0.f;
-              if (q0 + 2 >= valid) p1.x = 0.f;
-              if (q0 + 3 >= valid) p1.y = 0.f;
+            for (int q8 = 0; q8 < 2; ++q8) {   // 16 queries: 8 packed columns per plane
+            uint32_t hi[8], lo[8];
+#pragma unroll
+            for (int e4 = 0; e4 < 4; ++e4) {
+              const int e = 4 * q8 + e4;
+              const float4 l4 = lv[e];
+              float2 x0 = fma2(make_float2(__uint_as_float(sr[4 * e]), __uint_as_float(sr[4 * e + 1])), sl2, hb2);
+              float2 x1 =
+                  fma2(make_float2(__uint_as_float(sr[4 * e + 2]), __uint_as_float(sr[4 * e + 3])), sl2, hb2);
+              x0 = sub2(x0, make_float2(l4.x, l4.y));
+              x1 = sub2(x1, make_float2(l4.z, l4.w));
+              float2 p0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
+              float2 p1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
+              if (valid < kQBlk) {  // only the last block of a ragged column
+                const int q0 = cb + 4 * e;
+                if (q0 >= valid) p0.x = 0.f;
+                if (q0 + 1 >= valid) p0.y = 0.f;
+                if (q0 + 2 >= valid) p1.x = 0.f;
+                if (q0 + 3 >= valid) p1.y = 0.f;
+              }
+              beta2 = add2(beta2, add2(p0, p1));
+              split2<__half>(p0, hi[2 * e4], lo[2 * e4]);
+              split2<__half>(p1, hi[2 * e4 + 1], lo[2 * e4 + 1]);
             }
-            beta2 = add2(beta2, add2(p0, p1));
-            split2<__half>(p0, hi[2 * e], lo[2 * e]);
-            split2<__half>(p1, hi[2 * e + 1], lo[2 * e + 1]);
+            // P^T of these queries over the chunk's own S^T columns (all read
+            // already): hi in [cb, cb + 16), lo in [cb + 16, cb + 32)
+            ptx::tmem_st8(tS(t) + lane_off + cb + 8 * q8, hi);
+            ptx::tmem_st8(tS(t) + lane_off + cb + 16 + 8 * q8, lo);
+            }
           }
-          // P^T of these 32 queries over the chunk's own S^T columns:
-          // hi in [cb, cb + 16), lo in [cb + 16, cb + 32)
-          ptx::tmem_st16(tS(t) + lane_off + cb, hi);
-          ptx::tmem_st16(tS(t) + lane_off + cb + 16, lo);
+          ptx::tmem_wait_st();
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(p_full + t);
         }
-        ptx::tmem_wait_st();
+        // beta = the two halves' column sums (slots alternate between items)
+        float* xs = sX + ((icnt & 1) * 2 + t) * 2 * kTile;
+        xs[hf * kTile + r] = beta2.x + beta2.y;
+        ptx::named_bar(1 + t, kTileThreads);
+        const float beta = beta2.x + beta2.y + xs[(hf ^ 1) * kTile + r];
+        ok = ok && ptx::mbar_wait(o_done + t, icnt & 1);
+        ptx::tc_fence_after();
+        const float inv = 1.f / beta;
+        const float2 inv2 = make_float2(inv, inv);
+        // q~ as hi / lo planes of the input type: the A operand of the next R step
+        TQ* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {   // 16 columns at a time
+          uint32_t o[16];
+          ptx::tmem_ld16(tA(t) + lane_off + hf * (D / 2) + cc * 16, o);
+          ptx::tmem_wait_ld();
+          uint32_t hi[8], lo[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            split2<TQ>(mul2(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), inv2), hi[e], lo[e]);
+          if (c1 < g.b1k && ok) {
+            uint4* ph = reinterpret_cast<uint4*>(dst + cc * 16);
+            uint4* pl = reinterpret_cast<uint4*>(dst + plane + cc * 16);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              ph[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+              pl[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+            }
+          }
+        }
+        // the accumulator is read: the next item may overwrite it
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(p_full + t);
+        if (lane == 0) ptx::mbar_arrive(acc_free + t);
+        ++icnt;
       }
-      // beta = the two halves' column sums
-      sX[(t * 2 + hf) * kTile + r] = beta2.x + beta2.y;
-      ptx::named_bar(1 + t, kTileThreads);
-      const float beta = beta2.x + beta2.y + sX[(t * 2 + (hf ^ 1)) * kTile + r];
-      ok = ok && ptx::mbar_wait(o_done + t, 0);
-      ptx::tc_fence_after();
-      const float inv = 1.f / beta;
-      // q~ as hi / lo planes of the input type: the A operand of the next R step
-      const long long plane = (long long)g.BH * g.b2 * g.b1k * D;
-      TQ* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);
-      const float2 inv2 = make_float2(inv, inv);
-#pragma unroll
-      for (int cc = 0; cc < D / 64; ++cc) {
-        uint32_t o[32];
-        ptx::tmem_ld32(tA(t) + lane_off + hf * (D / 2) + cc * 32, o);
-        ptx::tmem_wait_ld();
-        uint32_t hi[16], lo[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e)
-          split2<TQ>(mul2(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), inv2), hi[e], lo[e]);
-        if (c1 < g.b1k && ok) {
-          uint4* ph = reinterpret_cast<uint4*>(dst + cc * 32);
-          uint4* pl = reinterpret_cast<uint4*>(dst + plane + cc * 32);
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            ph[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
-            pl[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
-          }
-        }
-      }
+      gq += nqb;
     }
   }
   ptx::tc_fence_before();

@@ -322,7 +322,16 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     attrs_set = true;
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);  // two 128-row tiles per CTA
-  const dim3 grid_k((g.b1k + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
+  // persistent column pass: one CTA per SM over (head, position, 256 key tiles) items
+  static int sm_count = 0;
+  if (!sm_count) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
+    if (sm_count <= 0) sm_count = 1;
+  }
+  const long long col_items = (long long)g.BH * g.b2 * ((g.b1k + 2 * kTile - 1) / (2 * kTile));
+  const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
   const int r_group = kRtcRows / ((g.b2 + 7) & ~7);   // key tiles per R-step CTA
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   for (int it = 0; it < p.iters; ++it) {
