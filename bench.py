@@ -70,7 +70,7 @@ def work_model(w):
     hb = BH * g["b2"] * g["b1k"] * 4
     phases = {
         "l_out": dict(flops=BH * 2 * FL, bytes=nq + 2 * nk + hb + no),   # q, k~, z, h -> out
-        "l_row": dict(flops=BH * FL, bytes=nq + nk + hb + lse),          # q, k~, h -> lse
+        "l_lse": dict(flops=BH * FL, bytes=nq + nk + hb + lse),          # q, k~, h -> lse
         "l_col": dict(flops=BH * FL, bytes=nq + nk + hb + lse + nk),     # q, k~, h, lse -> q~
         "r_step": dict(flops=BH * 2 * FR, bytes=3 * nk),                 # q~, k -> k~ (final: +v, z)
         "qbar": dict(flops=0.0, bytes=nq),

@@ -143,7 +143,7 @@ size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int 
 enum {
   MONARCH_PHASE_QBAR = 0,   /* mean query per position (KV-cache init)        */
   MONARCH_PHASE_R_STEP = 1, /* R step: per-tile softmax, entropy, k~ (and z)  */
-  MONARCH_PHASE_L_ROW = 2,  /* L step row pass of a non-final iteration (LSE) */
+  MONARCH_PHASE_L_LSE = 2,  /* L step LSE pass of a non-final iteration      */
   MONARCH_PHASE_L_OUT = 3,  /* final L step fused with y = L z and the store  */
   MONARCH_PHASE_L_COL = 4,  /* column pass q~ = L^T q / L^T 1                 */
   MONARCH_NUM_PHASES = 5

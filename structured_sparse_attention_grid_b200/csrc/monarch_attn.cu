@@ -85,7 +85,7 @@ template <typename F>
 void launch(int phase, cudaStream_t st, F&& f) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (debug_sync()) {
-    static const char* names[] = {"qbar", "r_step", "l_row", "l_out", "l_col"};
+    static const char* names[] = {"qbar", "r_step", "l_lse", "l_out", "l_col"};
     fprintf(stderr, "[monarch] launch %s ...\n", names[phase]);
     auto t0 = std::chrono::steady_clock::now();
     f();
@@ -354,7 +354,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         tc::l_row<__half, TO, D, true><<<grid_q, tc::kThreads, smem_out, st>>>(out, maps, w.lse, g);
       });
     } else {
-      launch(MONARCH_PHASE_L_ROW, st, [&] {
+      launch(MONARCH_PHASE_L_LSE, st, [&] {
         tc::l_lse<D><<<grid_q, tc::kThreads, smem_lse, st>>>(maps, w.lse, g);
       });
     }
@@ -398,7 +398,7 @@ int run(const Plan& p, const T* q, const T* k, const T* v, TO* out, char* ws, cu
       r_step_simt<T><<<dim3(g.b1k, g.BH), 128, r_smem, st>>>(q, k, v, w, g, mode, final_step);
     });
     dim3 grid((g.b1q + kRows - 1) / kRows, g.b2, g.BH);
-    launch(final_step ? MONARCH_PHASE_L_OUT : MONARCH_PHASE_L_ROW, st, [&] {
+    launch(final_step ? MONARCH_PHASE_L_OUT : MONARCH_PHASE_L_LSE, st, [&] {
       if (g.d == 128) l_row_simt<T, TO, 128><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
       else l_row_simt<T, TO, 64><<<grid, 32 * kRows, 0, st>>>(q, out, w, g, final_step);
     });
