@@ -281,6 +281,74 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     // are read from TMEM once and kept in registers.
     ok = ptx::mbar_wait(bar_s, 0);
     ptx::tc_fence_after();
+    const int cb = gg * r8;
+    const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
+    const int ch_lo = (wg0 * r8) >> 5, ch_hi = min((wg1 * r8 + g.b2 - 1) >> 5, 3);
+    auto in_tile = [&](int c) { return (unsigned)(c - cb) < (unsigned)g.b2; };
+    uint32_t sv[3][32];
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+      if (ch_lo + j <= ch_hi) ptx::tmem_ld32(tS + lane_off + 32 * (ch_lo + j), sv[j]);
+    ptx::tmem_wait_ld();
+    // Branch-free: columns outside this row's tile become -inf (p = 0).  The
+    // entropy uses sum p s (raw scores, finite everywhere) so that masked
+    // terms are exactly zero; four partial sums shorten the dependency chains.
+    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const bool in = ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i);
+        const float x = in ? __uint_as_float(sv[j][i]) : -INFINITY;
+        sv[j][i] = __float_as_uint(x);
+        mq[i & 3] = fmaxf(mq[i & 3], x);
+      }
+    const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+    const float ms = (m == -INFINITY) ? 0.f : m * g.sl2;   // base-2 units; a row with no column stays 0
+    float lq[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < 3; ++j)
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float x = __uint_as_float(sv[j][i]);
+        const float p = ptx::ex2(fmaf(x, g.sl2, -ms));
+        lq[i & 3] += p;
+        pq[i & 3] = (p > 0.f) ? fmaf(p, x, pq[i & 3]) : pq[i & 3];
+        sv[j][i] = __float_as_uint(p);
+      }
+    const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
+    // sum p (x s2 - ms) with x the raw score
+    const float xe = g.sl2 * ((pq[0] + pq[1]) + (pq[2] + pq[3])) - ms * l;
+    const float inv = 1.f / l;
+    const float2 inv2 = make_float2(inv, inv);
+    // R over S: chunk ch -> columns [32 ch, 32 ch + 16) hi, [32 ch + 16, 32 ch + 32) lo
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      if (ch_lo + j > ch_hi) continue;
+      uint32_t hi[16], lo[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        tc::split2<TQ>(tc::mul2(make_float2(__uint_as_float(sv[j][2 * i]), __uint_as_float(sv[j][2 * i + 1])), inv2),
+                       hi[i], lo[i]);
+      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j), hi);
+      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j) + 16, lo);
+    }
+    {
+      uint32_t zero[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) zero[i] = 0u;
+      for (int ch = 0; ch < 4; ++ch)
+        if (ch < ch_lo || ch > ch_hi) {
+          ptx::tmem_st16(tS + lane_off + 32 * ch, zero);
+          ptx::tmem_st16(tS + lane_off + 32 * ch + 16, zero);
+        }
+    }
+    ptx::tmem_wait_st();
+    ptx::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) ptx::mbar_arrive(bar_r);
+    // h in bits: -sum R log2 R = log2 l - sum R (x - m)
+    if (valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
     if (bf16 && mode != QT_BUFFER) {
       // first step, bf16 input: the L step reads q in f16 (exact for |q| <
       // 65504; larger magnitudes set kErrRange).  Convert the loaded rows into
@@ -320,64 +388,6 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         ptx::bulk_commit();
       }
     }
-    const int cb = gg * r8;
-    const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
-    const int ch_lo = (wg0 * r8) >> 5, ch_hi = min((wg1 * r8 + g.b2 - 1) >> 5, 3);
-    auto in_tile = [&](int c) { return (unsigned)(c - cb) < (unsigned)g.b2; };
-    uint32_t sv[3][32];
-#pragma unroll
-    for (int j = 0; j < 3; ++j)
-      if (ch_lo + j <= ch_hi) ptx::tmem_ld32(tS + lane_off + 32 * (ch_lo + j), sv[j]);
-    ptx::tmem_wait_ld();
-    float m = -INFINITY;
-#pragma unroll
-    for (int j = 0; j < 3; ++j)
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i)) m = fmaxf(m, __uint_as_float(sv[j][i]));
-    const float ms = m * g.sl2;   // base-2 units
-    float l = 0.f, xe = 0.f;
-#pragma unroll
-    for (int j = 0; j < 3; ++j)
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool in = ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i);
-        const float dx = in ? fmaf(__uint_as_float(sv[j][i]), g.sl2, -ms) : 0.f;
-        const float p = in ? ptx::ex2(dx) : 0.f;
-        l += p;
-        xe = fmaf(p, dx, xe);
-        sv[j][i] = __float_as_uint(p);
-      }
-    const float inv = 1.f / l;
-    const float2 inv2 = make_float2(inv, inv);
-    // R over S: chunk ch -> columns [32 ch, 32 ch + 16) hi, [32 ch + 16, 32 ch + 32) lo
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      if (ch_lo + j > ch_hi) continue;
-      uint32_t hi[16], lo[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        tc::split2<TQ>(tc::mul2(make_float2(__uint_as_float(sv[j][2 * i]), __uint_as_float(sv[j][2 * i + 1])), inv2),
-                       hi[i], lo[i]);
-      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j), hi);
-      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j) + 16, lo);
-    }
-    {
-      uint32_t zero[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) zero[i] = 0u;
-      for (int ch = 0; ch < 4; ++ch)
-        if (ch < ch_lo || ch > ch_hi) {
-          ptx::tmem_st16(tS + lane_off + 32 * ch, zero);
-          ptx::tmem_st16(tS + lane_off + 32 * ch + 16, zero);
-        }
-    }
-    ptx::tmem_wait_st();
-    ptx::tc_fence_before();
-    __syncwarp();
-    if (lane == 0) ptx::mbar_arrive(bar_r);
-    // h in bits: -sum R log2 R = log2 l - sum R (x - m)
-    if (valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
 
     // ---- epilogue: a row of k~ (or z) from TMEM, split into hi / lo planes,
     // staged in two swizzled [d half][128 rows][128 B] regions
