@@ -233,6 +233,7 @@ def run_ours(args, rank, world, device):
     roof["peak_source"] = peaks["source"]
 
     call_roof_ms = 1e3 * max(model["flops"] / (peaks["bf16_tflops"] * 1e12), io_bytes / (peaks["hbm_gbs"] * 1e9))
+    dense = dense_context(qd, kd, vd, model, flush if flush_l2 else None, stream, ms)
 
     # End to end through the host-buffer entry point (copies inside the timed region).
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -288,8 +289,39 @@ def run_ours(args, rank, world, device):
                 "d2h_bytes_per_step": q.numel() * 4},
         "gpu_launches": launches,
         "clocks": clocks.summary(),
+        "dense_context": dense,
     }
     return rec, (q, k, v, w)
+
+
+def dense_context(qd, kd, vd, model, flush, stream, monarch_ms):
+    """Context only, not the product: dense softmax attention over the same
+    q, k, v with torch's scaled_dot_product_attention (flash / cuDNN kernels),
+    i.e. the N x N attention that the Monarch factorisation replaces."""
+    import torch.nn.functional as F
+    if qd.dtype == torch.float32:
+        return {"impl": "not timed for f32 inputs"}
+    try:
+        F.scaled_dot_product_attention(qd, kd, vd)
+        torch.cuda.synchronize()
+        n = 3 if model["dense_flops"] > 2e12 else 10
+        times = []
+        for _ in range(n):
+            if flush is not None:
+                flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            F.scaled_dot_product_attention(qd, kd, vd)
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        ms = sorted(times)[len(times) // 2]
+        return {"impl": "torch.nn.functional.scaled_dot_product_attention (backend chosen by torch)",
+                "ms_per_call": ms, "tflops": model["dense_flops"] / (ms * 1e-3) / 1e12,
+                "dense_over_monarch_time": ms / monarch_ms}
+    except Exception as e:  # context only: never fail the bench line over it
+        return {"impl": "unavailable", "error": str(e)[:200]}
 
 
 def cpu_baseline(w, q, k, v, budget_s: float):

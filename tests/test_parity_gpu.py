@@ -118,6 +118,12 @@ EDGE = [
     # largest supported tile (64 positions) and b1 exactly one 128-row block
     _custom("f16", 2, 32, 32, 64, 8, 8, 2),
     _custom("bf16", 8, 16, 16, 128, 4, 2, 2, B=1, heads=2),
+    # positions per tile not a multiple of 8 (padded rows inside each stacked
+    # R-step tile), with and without a KV cache, both head sizes
+    _custom("bf16", 2, 9, 10, 128, 3, 5, 2),
+    _custom("f16", 2, 10, 15, 64, 5, 5, 3),
+    _custom("bf16", 2, 9, 10, 128, 3, 5, 2, Tk=5),
+    _custom("bf16", 3, 12, 21, 64, 3, 7, 1),
 ]
 
 
@@ -215,4 +221,24 @@ def test_invalid_call_returns_an_error_and_leaves_the_context_usable(cuda_lib):
     assert e.value.code == -1
     m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
     torch.cuda.synchronize()
+    assert torch.isfinite(out).all()
+
+
+def test_bf16_queries_beyond_the_f16_range_set_the_range_error(cuda_lib):
+    # The L step computes in f16: a bf16 query of magnitude >= 65520 cannot be
+    # represented, and the call reports it through the device error word
+    # (kErrRange = 3) rather than returning infinities silently.
+    w = _custom("bf16", 2, 12, 20, 128, 4, 4, 1, B=1, heads=1)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    q[0, 0, 17, 5] = 1.0e6
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    m.device_error(reset=True)
+    m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert m.device_error(reset=True) == 3
+    # the context stays usable and an in-range call is clean
+    q[0, 0, 17, 5] = 0.5
+    m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert m.device_error(reset=True) == 0
     assert torch.isfinite(out).all()
