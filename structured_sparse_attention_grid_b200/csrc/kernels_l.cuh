@@ -84,6 +84,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
   constexpr uint32_t kKst = 2 * NH * kBox;   // k~ hi+lo, 64 rows: [d half][plane][64 rows]
   constexpr uint32_t kZst = 2 * NH * kBox;   // z hi+lo, 64 rows:  [plane][d half][64 rows]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
   if (smem_misaligned(smem_raw)) return;
   uint8_t* sQ = smem_raw;                                             // [2 tiles]
   uint8_t* sK = sQ + 2 * kQt;                                         // [kKS]
@@ -138,6 +139,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
   const uint32_t tmem = *sTmem;
   auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
   auto tO = [&](int t) { return tmem + 256 * t + 128; };
@@ -447,6 +449,7 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   constexpr uint32_t kKst = NH * 2 * kBox;   // k~ hi of one block: [d half][128 keys]
   constexpr int kXt = xchg_tile_bytes<0>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
   if (smem_misaligned(smem_raw)) return;
   uint8_t* sQ = smem_raw;                                      // [2 tiles]
   uint8_t* sK = sQ + 2 * kQt;                                  // [kLS]
@@ -486,6 +489,7 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
   const uint32_t tmem = *sTmem;
   auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
 
@@ -663,6 +667,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   constexpr uint32_t kKt = 2 * NH * 2 * kBox;   // k~ hi+lo of one tile: [plane][d half][128 rows]
   constexpr uint32_t kQst = NH * 2 * kBox;      // 128 query rows: [d half][128 rows]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
   if (smem_misaligned(smem_raw)) return;
   uint8_t* sK = smem_raw;                                    // [2 tiles]
   uint8_t* sQ = sK + 2 * kKt;                                // [kQS]
@@ -713,6 +718,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
   const uint32_t tmem = *sTmem;
   auto tS = [&](int t) { return tmem + 256 * t; };
   auto tA = [&](int t) { return tmem + 256 * t + 128; };

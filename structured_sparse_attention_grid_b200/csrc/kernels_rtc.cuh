@@ -72,6 +72,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   constexpr int NH = D / 64;
   constexpr int bf16 = TcType<TQ>::kBf16;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
   if (tc::smem_misaligned(smem_raw)) return;
   uint8_t* sA = smem_raw;                  // [plane][d half] boxes; V in plane 0 later
   uint8_t* sK = sA + 2 * NH * kRBox;       // [d half] boxes
@@ -125,6 +126,8 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // set-up done: from here on global memory of the previous kernel is used
+  ptx::griddep_wait();
   const uint32_t tmem = *sTmem;
   const uint32_t tS = tmem, tAcc = tmem + 128;
 

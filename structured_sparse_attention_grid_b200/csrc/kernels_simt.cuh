@@ -6,6 +6,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace monarch {
 
@@ -21,6 +22,8 @@ template <typename T>
 __global__ void __launch_bounds__(kQbarThreads)
 qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, Geo g) {
   __shared__ float2 part[kQbarThreads];
+  ptx::griddep_launch();
+  ptx::griddep_wait();
   const int a2 = blockIdx.x, bh = blockIdx.y;
   const int npair = g.d / 2, groups = kQbarThreads / npair;
   const int pair = threadIdx.x % npair, grp = threadIdx.x / npair;

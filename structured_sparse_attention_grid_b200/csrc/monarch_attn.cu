@@ -230,6 +230,24 @@ int make_map(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int ran
   return MONARCH_OK;
 }
 
+// Launch with programmatic stream serialization: the kernel may begin its
+// set-up while the previous kernel on the stream finishes; it waits
+// (griddepcontrol.wait) before touching global memory.
+template <typename... KArgs, typename... Args>
+void launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 template <typename K>
 cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
@@ -340,22 +358,25 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     if (it == 0) {
       mode = p.kv ? QT_KVINIT : QT_IDENTITY;
       if (p.kv)
-        launch(MONARCH_PHASE_QBAR, st, [&] { qbar_kernel<TQ><<<dim3(g.b2, g.BH), kQbarThreads, 0, st>>>(q, w.qbar, g); });
+        launch(MONARCH_PHASE_QBAR, st, [&] {
+          launch_pdl(qbar_kernel<TQ>, dim3(g.b2, g.BH), dim3(kQbarThreads), 0, st, q, w.qbar, g);
+        });
     } else {
       launch(MONARCH_PHASE_L_COL, st, [&] {
-        tc::l_col<TQ, D><<<grid_k, tc::kThreads, smem_col, st>>>(maps, w.h, reinterpret_cast<TQ*>(w.qt), g);
+        launch_pdl(tc::l_col<TQ, D>, grid_k, dim3(tc::kThreads), smem_col, st, maps, (const float*)w.h,
+                   reinterpret_cast<TQ*>(w.qt), g);
       });
     }
     launch(MONARCH_PHASE_R_STEP, st, [&] {
-      r_step_tc5<TQ, D><<<grid_r, kRtcThreads, smem_r, st>>>(rmaps, q, w, planes, g, mode, final_step);
+      launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, mode, final_step);
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
-        tc::l_row<__half, TO, D, true><<<grid_q, tc::kThreads, smem_out, st>>>(out, maps, w.lse, g);
+        launch_pdl(tc::l_row<__half, TO, D, true>, grid_q, dim3(tc::kThreads), smem_out, st, out, maps, w.lse, g);
       });
     } else {
       launch(MONARCH_PHASE_L_LSE, st, [&] {
-        tc::l_lse<D><<<grid_q, tc::kThreads, smem_lse, st>>>(maps, w.lse, g);
+        launch_pdl(tc::l_lse<D>, grid_q, dim3(tc::kThreads), smem_lse, st, maps, w.lse, g);
       });
     }
   }

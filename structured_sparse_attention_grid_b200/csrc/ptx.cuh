@@ -227,6 +227,15 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // Waits until every bulk store of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialization may start before the previous kernel on its stream has
+// finished; griddep_wait() blocks until that kernel has completed and its
+// memory is visible, so everything before it must touch no global data the
+// previous kernel reads or writes.  griddep_launch() lets the next kernel start
+// its own set-up early.  Both are no-ops for kernels launched normally.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;" :::); }
+
 // Named barrier `id` (1..15) over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
