@@ -279,10 +279,57 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
       if (lane == 0) ptx::mbar_arrive(bar_a);
     }
 
+    // First step, bf16 input: the L step reads q in f16 (exact for |q| <
+    // 65504; larger finite magnitudes set kErrRange).  The loaded rows are
+    // converted into the A lo plane and stored from there as the block-major
+    // copy of q.
+    auto convert_and_store_q = [&]() {
+      if (valid && exact_q(c1)) {
+        bool over = false;
+#pragma unroll 1
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {
+            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+            uint4 u = *reinterpret_cast<const uint4*>(sA + o);
+            uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              // a finite bf16 of magnitude >= 2^16 (exponent field >= 143) has no f16 value
+              const uint32_t a0 = wv[e] & 0x7FFFu, a1 = (wv[e] >> 16) & 0x7FFFu;
+              over |= (a0 >= 0x4780u && a0 < 0x7F80u) || (a1 >= 0x4780u && a1 < 0x7F80u);
+              const __half2 hv = __floats2half2_rn(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+              wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
+            }
+            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
+          }
+        if (over) atomicExch(&ptx::g_device_error, ptx::kErrRange);
+      }
+      ptx::fence_proxy_async();
+      __syncwarp();
+      if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
+      ptx::named_bar(1, 128);
+      if (tid == 0 && ok) {
+        for (int t = 0; t < Gn; ++t) {
+          if (!exact_q(c1_0 + t)) continue;
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * r8) * 128, hf * 64,
+                              c1_0 + t - g.off, bh * g.b2);
+        }
+        ptx::bulk_commit();
+      }
+    };
+    // Without a KV cache the score MMA does not read the A lo plane: convert
+    // while it runs.  With one, after the score MMA (below).
+    if (bf16 && mode == QT_IDENTITY) {
+      ok = ptx::mbar_wait(bar_ld, 0);
+      convert_and_store_q();
+    }
+
     // ---- R = softmax over this row's tile columns [cb, cb + b2) of S.  The
     // rows of a warp need at most three 32-column chunks, from ch_lo on: they
     // are read from TMEM once and kept in registers.
-    ok = ptx::mbar_wait(bar_s, 0);
+    ok = ptx::mbar_wait(bar_s, 0) && ok;
     ptx::tc_fence_after();
     const int cb = gg * r8;
     const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
@@ -352,46 +399,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     if (lane == 0) ptx::mbar_arrive(bar_r);
     // h in bits: -sum R log2 R = log2 l - sum R (x - m)
     if (valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
-    if (bf16 && mode != QT_BUFFER) {
-      // first step, bf16 input: the L step reads q in f16 (exact for |q| <
-      // 65504; larger magnitudes set kErrRange).  Convert the loaded rows into
-      // the A lo plane, free once S is done, and store them from there.
-      if (valid && exact_q(c1)) {
-        bool over = false;
-#pragma unroll 1
-        for (int hf = 0; hf < NH; ++hf)
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
-            uint4 u = *reinterpret_cast<const uint4*>(sA + o);
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = make_float2(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
-              const __half2 hv = __floats2half2_rn(f.x, f.y);
-              const float2 back = __half22float2(hv);
-              over |= (isinf(back.x) && !isinf(f.x)) || (isinf(back.y) && !isinf(f.y));
-              wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
-          }
-        if (over) atomicExch(&ptx::g_device_error, ptx::kErrRange);
-      }
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
-      ptx::named_bar(1, 128);
-      if (tid == 0 && ok) {
-        for (int t = 0; t < Gn; ++t) {
-          if (!exact_q(c1_0 + t)) continue;
-          for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * r8) * 128, hf * 64,
-                              c1_0 + t - g.off, bh * g.b2);
-        }
-        ptx::bulk_commit();
-      }
-    }
-
+    if (bf16 && mode == QT_KVINIT) convert_and_store_q();
     // ---- epilogue: a row of k~ (or z) from TMEM, split into hi / lo planes,
     // staged in two swizzled [d half][128 rows][128 B] regions
     auto stage_row = [&](uint8_t* shi, uint8_t* slo, auto tag) {
