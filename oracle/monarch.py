@@ -34,6 +34,13 @@ pages give no equations; the reading implemented here is:
   D7  one iteration = one R step then one L step
   D8  output:  z = sum_c2 R v,  y = sum_c1 L z,  out = y scattered back to
                the grid order
+  D9  frame-chunk causal mask (autoregressive training over the whole
+      sequence, chunks of C frames; gist.science explainer §1 "auto-regressive
+      generation"): query tile a1 sees key tile c1 iff
+      frame(c1) // C <= frame(a1) // C, frames counted on the key axis.  The
+      mask restricts the support of L (D6's softmax runs over visible c1 only,
+      D4's sums over the a1 that see c1); R works inside a tile, one frame, so
+      it is unchanged, and the block identity of D3 stays feasible.
 
 D4 and D6 are the exact block maximisers of the variational softmax
 objective F(M) = sum_rows <M_row, S_row> + H(M_row) (whose unconstrained
@@ -61,6 +68,7 @@ class Grid:
     th: int
     tw: int
     Tk: int | None = None
+    chunk_frames: int = 0  # frames per causal chunk (D9); 0 = every key visible
 
     @property
     def Tkey(self) -> int:
@@ -95,6 +103,21 @@ class Grid:
             raise ValueError("tile must divide the frame")
         if self.Tkey < self.T:
             raise ValueError("key frames must include the query chunk")
+        if self.chunk_frames < 0:
+            raise ValueError("chunk_frames must be >= 0")
+
+    def visible(self) -> np.ndarray:
+        """[b1q, b1k] bool: key tile c1 visible to query tile a1 (D9).  The
+        query chunk is the last T frames of the key sequence."""
+        P = self.tiles_per_frame
+        vis = np.ones((self.b1q, self.b1k), dtype=bool)
+        if self.chunk_frames:
+            C = self.chunk_frames
+            for a1 in range(self.b1q):
+                tq = self.Tkey - self.T + a1 // P
+                for c1 in range(self.b1k):
+                    vis[a1, c1] = (c1 // P) // C <= tq // C
+        return vis
 
 
 def block_index(frames: int, H: int, W: int, th: int, tw: int) -> np.ndarray:
@@ -147,7 +170,7 @@ def initial_qtilde(qb: np.ndarray, grid: Grid) -> np.ndarray:
         return qb.copy()
     off = (grid.Tkey - grid.T) * grid.tiles_per_frame
     b1k = grid.b1k
-    visible = np.ones((b1q, b1k), dtype=bool)  # the query chunk sees all keys
+    visible = grid.visible()  # without a mask the query chunk sees all keys
     w = 1.0 / visible.sum(axis=1)  # 1/|visible(a1)|
     qt = np.empty((b1k, b2, d))
     for c1 in range(b1k):
@@ -182,12 +205,15 @@ def _r_step(qt: np.ndarray, kb: np.ndarray, scale: float):
     return R, h
 
 
-def _l_step(qb: np.ndarray, kt: np.ndarray, h: np.ndarray, scale: float):
+def _l_step(qb: np.ndarray, kt: np.ndarray, h: np.ndarray, scale: float, visible=None):
     """D6 for one head: qb [b1q,b2,d], kt [b1k,b2,d], h [b1k,b2] ->
-    L [b2, b1q, b1k], lse [b2, b1q]."""
+    L [b2, b1q, b1k], lse [b2, b1q].  ``visible`` [b1q, b1k] (D9) restricts
+    the softmax to the visible key tiles."""
     qp = np.swapaxes(qb, 0, 1)  # [a2, a1, d]
     kp = np.swapaxes(kt, 0, 1)  # [a2, c1, d]
     s_l = scale * np.matmul(qp, np.swapaxes(kp, 1, 2)) + h.T[:, None, :]
+    if visible is not None:
+        s_l = np.where(visible[None, :, :], s_l, -np.inf)
     return _softmax_last(s_l), _logsumexp_last(s_l)
 
 
@@ -214,6 +240,7 @@ def monarch_head(qb, kb, vb, grid: Grid, iters: int, scale: float,
     if iters < 1:
         raise ValueError("iters must be >= 1")
     qt = initial_qtilde(qb, grid)
+    vis = grid.visible() if grid.chunk_frames else None
     obj = []
     L = None
     for it in range(iters):
@@ -221,7 +248,7 @@ def monarch_head(qb, kb, vb, grid: Grid, iters: int, scale: float,
             qt = _column_qtilde(L, qb)  # L of the previous iteration
         R, h = _r_step(qt, kb, scale)
         kt = np.matmul(R, kb)  # k~[c1, a2] = sum_c2 R k
-        L, lse = _l_step(qb, kt, h, scale)
+        L, lse = _l_step(qb, kt, h, scale, vis)
         if track_objective:
             obj.append(head_objective(L, R, qb, kb, scale))
     z = np.matmul(R, vb)  # [c1, a2, d]
@@ -260,15 +287,27 @@ def monarch_attention(q, k, v, grid: Grid, iters: int, scale: float | None = Non
     return (out, states) if return_states else out
 
 
-def dense_attention(q, k, v, scale: float | None = None):
-    """Textbook softmax(s q k^T) v per (batch, head), fp64."""
+def dense_attention(q, k, v, scale: float | None = None, mask=None):
+    """Textbook softmax(s q k^T) v per (batch, head), fp64.  ``mask``
+    [Nq, Nk] bool keeps only the allowed keys of each query."""
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
     if scale is None:
         scale = 1.0 / np.sqrt(q.shape[-1])
     s = scale * np.matmul(q, np.swapaxes(k, -1, -2))
+    if mask is not None:
+        s = np.where(mask, s, -np.inf)
     return np.matmul(_softmax_last(s), v)
+
+
+def frame_chunk_mask(T: int, Tk: int, H: int, W: int, chunk_frames: int) -> np.ndarray:
+    """Token-level [Nq, Nk] mask of D9: query token of (absolute) frame tq
+    sees key token of frame tk iff tk // C <= tq // C."""
+    hw = H * W
+    tq = (Tk - T) + np.arange(T * hw) // hw
+    tk = np.arange(Tk * hw) // hw
+    return (tk[None, :] // chunk_frames) <= (tq[:, None] // chunk_frames)
 
 
 def monarch_flops(grid: Grid, d: int, iters: int, B: int = 1, heads: int = 1) -> float:

@@ -78,7 +78,7 @@ def test_L_instead_of_L_transpose_is_caught(monkeypatch):
 
 def test_wrong_score_scale_is_caught(monkeypatch):
     orig = om._l_step
-    monkeypatch.setattr(om, "_l_step", lambda qb, kt, h, s: orig(qb, kt, h, s * 1.01))
+    monkeypatch.setattr(om, "_l_step", lambda qb, kt, h, s, vis=None: orig(qb, kt, h, s * 1.01, vis))
     assert not _one_position_is_dense()
 
 
@@ -105,3 +105,47 @@ def test_wrong_position_index_is_caught(monkeypatch):
     from tests.test_oracle_pins import test_block_index_matches_hand_table
     with pytest.raises(AssertionError):
         test_block_index_matches_hand_table()
+
+
+def _masked_separable_is_dense():
+    from tests.test_oracle_pins import _masked_dense
+    g = om.Grid(6, 4, 4, 2, 2, chunk_frames=2)
+    q, k, v = _separable(1, 1, g, 16, seed=13)
+    out = om.monarch_attention(q, k, v, g, 1)
+    return np.abs(out - _masked_dense(q, k, v, g)).max() < 1e-10
+
+
+def test_unmutated_mask_passes():
+    assert _masked_separable_is_dense()
+
+
+def test_mask_that_hides_the_own_chunk_is_caught(monkeypatch):
+    # strict '<' instead of '<=' between chunk indices (own chunk invisible
+    # except through the tile itself, which D3 needs)
+    def strict(self):
+        P = self.tiles_per_frame
+        vis = np.ones((self.b1q, self.b1k), dtype=bool)
+        for a1 in range(self.b1q):
+            for c1 in range(self.b1k):
+                vis[a1, c1] = (c1 // P) // self.chunk_frames < (a1 // P) // self.chunk_frames or c1 == a1
+        return vis
+    monkeypatch.setattr(om.Grid, "visible", strict)
+    assert not _masked_separable_is_dense()
+
+
+def test_mask_over_tiles_instead_of_frames_is_caught(monkeypatch):
+    # chunk index taken from the tile index instead of its frame
+    def by_tile(self):
+        vis = np.ones((self.b1q, self.b1k), dtype=bool)
+        for a1 in range(self.b1q):
+            for c1 in range(self.b1k):
+                vis[a1, c1] = c1 // self.chunk_frames <= a1 // self.chunk_frames
+        return vis
+    monkeypatch.setattr(om.Grid, "visible", by_tile)
+    assert not _masked_separable_is_dense()
+
+
+def test_mask_ignored_by_the_l_step_is_caught(monkeypatch):
+    orig = om._l_step
+    monkeypatch.setattr(om, "_l_step", lambda qb, kt, h, s, vis=None: orig(qb, kt, h, s, None))
+    assert not _masked_separable_is_dense()

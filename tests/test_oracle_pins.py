@@ -262,3 +262,52 @@ def test_flop_counts_match_hand_values():
     assert om.monarch_flops(g, 128, 2, 1, 12) == 12 * (4 * FL + 5 * FR)
     assert abs(om.monarch_flops(g, 128, 2, 1, 12) / 1e9 - 12.94) < 0.01
     assert om.dense_flops(g, 128, 1, 12) == 4 * 12 * 4680 * 4680 * 128
+
+
+# ---- frame-chunk causal mask (D9) -------------------------------------------
+
+def _masked_dense(q, k, v, g: om.Grid):
+    mask = om.frame_chunk_mask(g.T, g.Tkey, g.H, g.W, g.chunk_frames)
+    return om.dense_attention(q, k, v, mask=mask)
+
+
+def test_frame_chunk_mask_matches_hand_table():
+    # 3 frames, chunks of 2: frames {0, 1} | {2}; one token per frame
+    m = om.frame_chunk_mask(3, 3, 1, 1, 2).astype(int)
+    np.testing.assert_array_equal(m, [[1, 1, 0], [1, 1, 0], [1, 1, 1]])
+    # tile-level visibility of a 2-tile-per-frame grid agrees with it
+    g = om.Grid(3, 2, 4, 2, 2, chunk_frames=2)
+    vis = g.visible().astype(int)
+    expect = np.kron(np.array([[1, 1, 0], [1, 1, 0], [1, 1, 1]]), np.ones((2, 2), dtype=int))
+    np.testing.assert_array_equal(vis, expect)
+
+
+@pytest.mark.parametrize("C", [5, 6, 9])
+def test_one_chunk_mask_is_the_bidirectional_result(C):
+    g0 = om.Grid(5, 4, 6, 2, 3)
+    g1 = om.Grid(5, 4, 6, 2, 3, chunk_frames=C)
+    q, k, v = (_rand((1, 2, g0.Nq, 8), s) for s in (31, 32, 33))
+    np.testing.assert_array_equal(om.monarch_attention(q, k, v, g1, 2), om.monarch_attention(q, k, v, g0, 2))
+
+
+@pytest.mark.parametrize("g,iters", [
+    (om.Grid(6, 4, 4, 2, 2, chunk_frames=2), 1),
+    (om.Grid(6, 4, 4, 2, 2, chunk_frames=2), 2),
+    (om.Grid(5, 4, 6, 2, 3, chunk_frames=1), 3),
+    (om.Grid(7, 4, 4, 4, 2, chunk_frames=3), 2),   # ragged last chunk
+])
+def test_separable_scores_with_chunk_mask_give_masked_dense_attention(g, iters):
+    q, k, v = _separable(1, 2, g, 16, seed=13)
+    out = om.monarch_attention(q, k, v, g, iters)
+    np.testing.assert_allclose(out, _masked_dense(q, k, v, g), atol=1e-12, rtol=0)
+
+
+def test_masked_M_is_row_stochastic_and_zero_outside_the_mask():
+    g = om.Grid(4, 4, 4, 2, 2, chunk_frames=2)
+    q, k, v = (_rand((1, 1, g.Nq, 6), s) for s in (41, 42, 43))
+    out, states = om.monarch_attention(q, k, v, g, 2, return_states=True)
+    M = _brute_force_M(states[(0, 0)], g)
+    mask = om.frame_chunk_mask(g.T, g.Tkey, g.H, g.W, g.chunk_frames)
+    assert (M >= 0).all() and (M[~mask] == 0).all()
+    np.testing.assert_allclose(M.sum(axis=1), 1.0, atol=1e-13)
+    np.testing.assert_allclose(out[0, 0], M @ v[0, 0], atol=1e-13)
