@@ -76,6 +76,23 @@ int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out,
                      int tile_h, int tile_w, int iters, long kv_len,
                      int dtype, int out_dtype, cudaStream_t stream);
 
+/* monarch_attn_fwd with the frame-chunk causal mask used when training over
+ * the whole sequence (DEFINITION.md D9; MonarchRT explainers, gist.science §1
+ * "auto-regressive generation"): frames form chunks of chunk_frames from
+ * frame 0, and a query of chunk i attends only to keys of chunks <= i.  In
+ * the Monarch form this restricts the support of the factor L: the R step
+ * (inside one tile, one frame) is unchanged, the L step's softmax runs over
+ * the visible key tiles and the column pass over the queries that see a key
+ * tile.  chunk_frames = 0, or >= T, is the bidirectional call.
+ * Arguments, layout, ownership and errors as monarch_attn_fwd, plus:
+ * MONARCH_EINVAL for chunk_frames < 0; MONARCH_EUNSUPPORTED for
+ * chunk_frames > 0 with a KV cache (kv_len > T*H*W: the query chunk is then
+ * the newest and sees every key, so call monarch_attn_fwd). */
+int monarch_attn_fwd_ex(const void* q, const void* k, const void* v, void* out,
+                        int B, int heads, int T, int H, int W, int d,
+                        int tile_h, int tile_w, int iters, long kv_len, int chunk_frames,
+                        int dtype, int out_dtype, cudaStream_t stream);
+
 /* Bytes of workspace the forward needs for these arguments (0 on invalid
  * arguments, with the reason in monarch_attn_last_error()). */
 size_t monarch_attn_workspace_bytes(int B, int heads, int T, int H, int W, int d,

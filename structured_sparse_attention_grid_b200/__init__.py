@@ -20,6 +20,8 @@ PHASES = ("qbar", "r_step", "l_lse", "l_out", "l_col")
 _SIGS = {
     "monarch_attn_fwd": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                          + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "monarch_attn_fwd_ex": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                            + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_int]),
     "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
@@ -99,15 +101,21 @@ def _check_tensors(*ts):
             raise ValueError("tensors must be contiguous [B, heads, N, d]")
 
 
-def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
+def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None, chunk_frames=0):
     """out <- Monarch attention of (q, k, v); CUDA tensors, contiguous
     [B, heads, N, d]; kv length = k.shape[2]; out is float32 or q's dtype.
-    Asynchronous on ``stream``."""
+    ``chunk_frames`` > 0 applies the frame-chunk causal mask of training
+    over the whole sequence (monarch_attn_fwd_ex).  Asynchronous on ``stream``."""
     lib = load_library()
     _check_tensors(q, k, v, out)
     args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
-    _check(lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
+    if chunk_frames:
+        _check(lib.monarch_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                       *args, int(chunk_frames), _dtype_code(q), _dtype_code(out),
+                                       _stream_ptr(stream)))
+    else:
+        _check(lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                    *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
 
 

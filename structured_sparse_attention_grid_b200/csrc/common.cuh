@@ -28,7 +28,17 @@ struct Geo {
   int b1q_pad;   // row stride of the row LSE
   long long Nq, Nk;
   float sl2;     // s * log2(e), s = 1/sqrt(d)
+  int cq;        // key/query tiles per frame-chunk of the causal mask; 0 = no mask
 };
+
+// Frame-chunk causal mask (self-attention, chunks of C frames, cq = C * P
+// tiles): query tile a1 sees the key tiles [0, key_limit(a1)) and key tile c1
+// is seen by the query tiles [query_start(c1), b1q).  Chunks start at frame
+// 0; the last one may be shorter.
+__device__ __forceinline__ int key_limit(const Geo& g, int a1) {
+  return g.cq ? min(g.b1k, (a1 / g.cq + 1) * g.cq) : g.b1k;
+}
+__device__ __forceinline__ int query_start(const Geo& g, int c1) { return g.cq ? (c1 / g.cq) * g.cq : 0; }
 
 // Token index (within one head) of tile c1, position c2.
 __device__ __forceinline__ long long token_of(const Geo& g, int c1, int c2) {

@@ -109,7 +109,9 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
   const int a1_base = blockIdx.x * 2 * kTile;
   const int zrow = bh * g.b2 + a2;
   const int plane_rows = g.BH * g.b2;
-  const int nkb = (g.b1k + kBlk - 1) / kBlk;
+  // key blocks any row of this CTA sees (all of them without a causal mask)
+  const int kmax = key_limit(g, min(a1_base + 2 * kTile, g.b1q) - 1);
+  const int nkb = (kmax + kBlk - 1) / kBlk;
   const int ntiles = (g.b1q - a1_base > kTile) ? 2 : 1;
 
   if (tid == 0) {
@@ -255,6 +257,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int a1 = a1_base + t * kTile + r;
+    const int rowlim = key_limit(g, min(a1, g.b1q - 1));   // visible key tiles [0, rowlim)
     if (t < ntiles) {
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -293,7 +296,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
           ptx::mbar_arrive(k_free + ks);
           if (!OUT) ptx::mbar_arrive(s_free + 2 * t + b);
         }
-        const int valid = min(kBlk, g.b1k - j * kBlk) - 32 * hf;   // keys of this half (may be <= 0)
+        const int valid = min(kBlk, rowlim - j * kBlk) - 32 * hf;   // keys of this half (may be <= 0)
         if (valid < 32) {  // only the last block of a ragged row
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
@@ -467,7 +470,9 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   const int a2 = blockIdx.y, bh = blockIdx.z;
   const int a1_base = blockIdx.x * 2 * kTile;
   const int zrow = bh * g.b2 + a2;
-  const int nkb = (g.b1k + kLBlk - 1) / kLBlk;
+  // key blocks any row of this CTA sees (all of them without a causal mask)
+  const int kmax = key_limit(g, min(a1_base + 2 * kTile, g.b1q) - 1);
+  const int nkb = (kmax + kLBlk - 1) / kLBlk;
   const int ntiles = (g.b1q - a1_base > kTile) ? 2 : 1;
 
   if (tid == 0) {
@@ -564,6 +569,7 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int a1 = a1_base + t * kTile + r;
+    const int rowlim = key_limit(g, min(a1, g.b1q - 1));   // visible key tiles [0, rowlim)
     if (t < ntiles) {
       float m = -INFINITY, l = 0.f;
       bool ok = true;
@@ -598,7 +604,7 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
               ptx::mbar_arrive(s_free + 2 * t + b);
             }
           }
-          const int valid = min(kLBlk, g.b1k - j * kLBlk) - 64 * hf - 32 * sb;
+          const int valid = min(kLBlk, rowlim - j * kLBlk) - 64 * hf - 32 * sb;
           if (valid < 32) {  // only the last block of a ragged row
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
@@ -689,11 +695,13 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   const int nqb = (g.b1q + kQBlk - 1) / kQBlk;
   const int nchunk = (g.b1k + 2 * kTile - 1) / (2 * kTile);
   const int n_items = g.BH * g.b2 * nchunk;
-  // item -> (row of the [BH][b2] planes, first key tile, tiles in it)
-  auto item_of = [&](int it, int& zrow, int& kb, int& ntiles) {
+  // item -> (row of the [BH][b2] planes, first key tile, tiles in it, first
+  // query block: under a causal mask no earlier query sees these key tiles)
+  auto item_of = [&](int it, int& zrow, int& kb, int& ntiles, int& qb0) {
     zrow = it / nchunk;
     kb = (it - zrow * nchunk) * 2 * kTile;
     ntiles = (g.b1k - kb > kTile) ? 2 : 1;
+    qb0 = query_start(g, kb) / kQBlk;
   };
 
   if (tid == 0) {
@@ -731,8 +739,8 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
       bool ok = true;
       int gq = 0, ni = 0;   // query blocks and items loaded so far
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ni) {
-        int zrow, kb, ntiles;
-        item_of(it, zrow, kb, ntiles);
+        int zrow, kb, ntiles, qb0;
+        item_of(it, zrow, kb, ntiles, qb0);
         if (ni > 0) ok = ptx::mbar_wait(k_empty, (ni - 1) & 1);
         if (!ok) break;
         ptx::mbar_expect_tx(k_full, 2 * kKt);
@@ -742,7 +750,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
               for (int rh = 0; rh < 2; ++rh)
                 ptx::tma_load_3d(sK + t * kKt + (p * NH + hf) * 2 * kBox + rh * kBox, &maps.kt, k_full, hf * 64,
                                  kb + t * kTile + rh * kBlk, p * plane_rows + zrow);
-        for (int blk = 0; blk < nqb && ok; ++blk, ++gq) {
+        for (int blk = qb0; blk < nqb && ok; ++blk, ++gq) {
           const int qs = gq % kQS;
           if (gq >= kQS) ok = ptx::mbar_wait(q_free + qs, ((gq / kQS) - 1) & 1);
           if (!ok) break;
@@ -780,22 +788,22 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
       int gq = 0, ni = 0;
       int cnt0 = 0, cnt1 = 0, icnt0 = 0, icnt1 = 0;   // blocks / items processed per tile
       for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x, ++ni) {
-        int zrow, kb, ntiles;
-        item_of(it, zrow, kb, ntiles);
+        int zrow, kb, ntiles, qb0;
+        item_of(it, zrow, kb, ntiles, qb0);
         ok = ptx::mbar_wait(k_full, ni & 1) && ptx::mbar_wait(q_full + gq % kQS, (gq / kQS) & 1);
         ptx::tc_fence_after();
         if (!ok) break;
         for (int t = 0; t < ntiles; ++t) issue_s(t, gq);
-        if (nqb == 1) ptx::mma_commit(k_empty);
-        for (int i = 0; i < nqb && ok; ++i) {
-          const int qs = (gq + i) % kQS;
+        if (nqb - qb0 == 1) ptx::mma_commit(k_empty);
+        for (int i = qb0; i < nqb && ok; ++i) {
+          const int qs = (gq + i - qb0) % kQS;
           const uint64_t q0 = ptx::sw128_desc(aQ + qs * kQst, 2 * kBox, 1024);
           for (int t = 0; t < ntiles && ok; ++t) {
             const int ct = t ? cnt1 : cnt0, it_t = t ? icnt1 : icnt0;
             ok = ptx::mbar_wait(p_full + t, ct & 1);
             // the first product of an item overwrites the accumulator the
             // previous item's epilogue reads
-            if (ok && i == 0 && it_t > 0) ok = ptx::mbar_wait(acc_free + t, (it_t - 1) & 1);
+            if (ok && i == qb0 && it_t > 0) ok = ptx::mbar_wait(acc_free + t, (it_t - 1) & 1);
             ptx::tc_fence_after();
             if (!ok) break;
             const uint32_t tp = tS(t);
@@ -804,13 +812,14 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
 #pragma unroll
               for (int kk = 0; kk < kQBlk / 16; ++kk)
                 ptx::mma_f16_ts(tA(t), tp + (kk >> 1) * 32 + p * 16 + (kk & 1) * 8, q0 + ((kk * 2048) >> 4), idPQ,
-                                (i | p | kk) != 0);
+                                ((i - qb0) | p | kk) != 0);
             if (t == ntiles - 1) ptx::mma_commit(q_free + qs);
             if (i + 1 < nqb) {
               // S^T(t, i+1) overwrites P^T(t, i): the P^T q product above runs first
-              ok = ptx::mbar_wait(q_full + (gq + i + 1) % kQS, ((gq + i + 1) / kQS) & 1);
+              const int gn = gq + i + 1 - qb0;   // ring index of block i + 1
+              ok = ptx::mbar_wait(q_full + gn % kQS, (gn / kQS) & 1);
               ptx::tc_fence_after();
-              if (ok) issue_s(t, gq + i + 1);
+              if (ok) issue_s(t, gn);
             } else {
               ptx::mma_commit(o_done + t);
             }
@@ -821,7 +830,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
         }
         ++icnt0;
         if (ntiles > 1) ++icnt1;
-        gq += nqb;
+        gq += nqb - qb0;
       }
     }
   } else {
@@ -834,18 +843,21 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
     bool ok = true;
     int gq = 0, cnt = 0, icnt = 0;
     for (int it = blockIdx.x; it < n_items; it += gridDim.x) {
-      int zrow, kb, ntiles;
-      item_of(it, zrow, kb, ntiles);
+      int zrow, kb, ntiles, qb0;
+      item_of(it, zrow, kb, ntiles, qb0);
       if (t < ntiles) {
         const int c1 = kb + t * kTile + r;
+        const int qstart = query_start(g, min(c1, g.b1k - 1));   // queries [qstart, b1q) see this tile
         const float hb = (c1 < g.b1k) ? hbuf[(long long)zrow * g.b1k_pad + c1] + kColShift : 0.f;
         const float2 hb2 = make_float2(hb, hb);
         float2 beta2 = make_float2(0.f, 0.f);
-        for (int i = 0; i < nqb; ++i, ++cnt) {
-          const int qs = (gq + i) % kQS;
-          ok = ok && ptx::mbar_wait(s_full + t, cnt & 1) && ptx::mbar_wait(q_full + qs, ((gq + i) / kQS) & 1);
+        for (int i = qb0; i < nqb; ++i, ++cnt) {
+          const int gi = gq + i - qb0;   // ring index of block i
+          const int qs = gi % kQS;
+          ok = ok && ptx::mbar_wait(s_full + t, cnt & 1) && ptx::mbar_wait(q_full + qs, (gi / kQS) & 1);
           ptx::tc_fence_after();
           const int valid = min(kQBlk, g.b1q - i * kQBlk);
+          const int vlo = qstart - i * kQBlk;   // queries of this block below it are masked
 #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {  // 32 queries at a time
             const int cb = 64 * hf + 32 * hh;   // first S^T column (query) of this chunk
@@ -867,12 +879,12 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
               x1 = sub2(x1, make_float2(l4.z, l4.w));
               float2 p0 = make_float2(ptx::ex2(x0.x), ptx::ex2(x0.y));
               float2 p1 = make_float2(ptx::ex2(x1.x), ptx::ex2(x1.y));
-              if (valid < kQBlk) {  // only the last block of a ragged column
+              if (valid < kQBlk || vlo > 0) {  // a ragged last block, or queries hidden by the mask
                 const int q0 = cb + 4 * e;
-                if (q0 >= valid) p0.x = 0.f;
-                if (q0 + 1 >= valid) p0.y = 0.f;
-                if (q0 + 2 >= valid) p1.x = 0.f;
-                if (q0 + 3 >= valid) p1.y = 0.f;
+                if (q0 >= valid || q0 < vlo) p0.x = 0.f;
+                if (q0 + 1 >= valid || q0 + 1 < vlo) p0.y = 0.f;
+                if (q0 + 2 >= valid || q0 + 2 < vlo) p1.x = 0.f;
+                if (q0 + 3 >= valid || q0 + 3 < vlo) p1.y = 0.f;
               }
               beta2 = add2(beta2, add2(p0, p1));
               split2<__half>(p0, hi[2 * e4], lo[2 * e4]);
@@ -925,7 +937,7 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
         if (lane == 0) ptx::mbar_arrive(acc_free + t);
         ++icnt;
       }
-      gq += nqb;
+      gq += nqb - qb0;
     }
   }
   ptx::tc_fence_before();

@@ -166,6 +166,7 @@ l_row_simt(const T* __restrict__ q, TO* __restrict__ out, Work w, Geo g, int fin
   }
   float m = -INFINITY, l = 0.f;
   const long long base = ((long long)bh * g.b2 + a2) * g.b1k;
+  const int rowlim = key_limit(g, valid ? a1 : 0);   // visible key tiles [0, rowlim)
   for (int c0 = 0; c0 < g.b1k; c0 += KC) {
     const int nk = min(KC, g.b1k - c0);
     __syncthreads();
@@ -177,7 +178,7 @@ l_row_simt(const T* __restrict__ q, TO* __restrict__ out, Work w, Geo g, int fin
     const float* hrow = w.h + ((long long)bh * g.b2 + a2) * g.b1k_pad;
     for (int j = threadIdx.x; j < nk; j += blockDim.x) sH[j] = hrow[c0 + j] * kLog2e;
     __syncthreads();
-    for (int j = 0; j < nk; ++j) {
+    for (int j = 0; j < nk && c0 + j < rowlim; ++j) {
       float p = 0.f;
 #pragma unroll
       for (int i = 0; i < PER; ++i) p = fmaf(qv[i], sK[j][lane + 32 * i], p);
@@ -230,6 +231,7 @@ l_col_simt(const T* __restrict__ q, Work w, Geo g) {
   }
   const float hb = valid ? w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] * kLog2e : 0.f;
   float beta = 0.f, mc = -INFINITY;
+  const int qstart = query_start(g, valid ? c1 : 0);   // queries that see this key tile: [qstart, b1q)
   const T* qh = q + (long long)bh * g.Nq * D;
   const float* lse = w.lse + ((long long)bh * g.b2 + a2) * g.b1q_pad;
   for (int a0 = 0; a0 < g.b1q; a0 += QC) {
@@ -242,6 +244,7 @@ l_col_simt(const T* __restrict__ q, Work w, Geo g) {
     for (int j = threadIdx.x; j < nq; j += blockDim.x) sL[j] = lse[a0 + j];
     __syncthreads();
     for (int j = 0; j < nq; ++j) {
+      if (a0 + j < qstart) continue;
       float p = 0.f;
 #pragma unroll
       for (int i = 0; i < PER; ++i) p = fmaf(kv[i], sQ[j][lane + 32 * i], p);

@@ -136,7 +136,7 @@ struct Plan {
 constexpr int kMaxB2 = 64;
 
 int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int iters,
-              long kv_len, int dtype, int out_dtype, Plan* p) {
+              long kv_len, int dtype, int out_dtype, Plan* p, int chunk_frames = 0) {
   if (B < 1 || heads < 1 || T < 1 || H < 1 || W < 1)
     return fail(MONARCH_EINVAL, "B, heads, T, H, W must be >= 1 (got %d %d %d %d %d)", B, heads, T, H, W);
   if (d != 64 && d != 128) return fail(MONARCH_EINVAL, "head_dim d must be 64 or 128 (got %d)", d);
@@ -177,6 +177,12 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
   g.Nq = nq;
   g.Nk = kv_len;
   g.sl2 = (float)(1.0 / std::sqrt((double)d) * 1.4426950408889634);
+  if (chunk_frames < 0) return fail(MONARCH_EINVAL, "chunk_frames must be >= 0 (got %d)", chunk_frames);
+  if (chunk_frames > 0 && g.Tk != T)
+    return fail(MONARCH_EUNSUPPORTED,
+                "the frame-chunk causal mask is for self-attention (kv_len == T*H*W); with a KV cache the "
+                "query chunk is the newest and sees every key");
+  g.cq = (chunk_frames > 0 && chunk_frames < T) ? chunk_frames * g.P : 0;   // C >= T: one chunk, no mask
   p->dtype = dtype;
   p->out_dtype = out_dtype;
   p->iters = iters;
@@ -570,6 +576,28 @@ int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out, int
   g_err.clear();
   Plan p;
   int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
+  if (rc) return rc;
+  if ((rc = check_io(q, k, v, out))) return rc;
+  void* ws = nullptr;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, p.total, pool, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", p.total, cudaGetErrorString(e));
+  }
+  rc = dispatch(p, q, k, v, out, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+int monarch_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int heads,
+                        int T, int H, int W, int d, int tile_h, int tile_w, int iters, long kv_len,
+                        int chunk_frames, int dtype, int out_dtype, cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p, chunk_frames);
   if (rc) return rc;
   if ((rc = check_io(q, k, v, out))) return rc;
   void* ws = nullptr;

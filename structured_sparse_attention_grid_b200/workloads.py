@@ -60,6 +60,7 @@ class Workload:
     kind: str  # "iid" | "separable" | "pos" | "pos_planted"
     Tk: int = 0  # key frames; 0 means T (self-attention)
     planted: int = 64
+    chunk_frames: int = 0  # frame-chunk causal mask of whole-sequence training; 0 = bidirectional
 
     @property
     def Tkey(self) -> int:
@@ -89,6 +90,9 @@ WORKLOADS = {
         Workload("chunk_4680_bf16", 1, 12, 3, 30, 52, 128, 6, 4, 2, "bf16", 2, "pos"),
         Workload("kvcache_4680x32760_bf16", 1, 12, 3, 30, 52, 128, 6, 4, 2, "bf16", 3, "pos", Tk=21),
         Workload("full_32760_bf16", 2, 12, 21, 30, 52, 128, 6, 4, 3, "bf16", 4, "pos_planted"),
+        # the same sequence in the training regime: 3-frame chunks, chunk-causal
+        Workload("train_32760_bf16_causal", 2, 12, 21, 30, 52, 128, 6, 4, 3, "bf16", 4, "pos_planted",
+                 chunk_frames=3),
         Workload("sweep_2048_f16", 1, 24, 8, 16, 16, 64, 8, 8, 2, "f16", 5, "pos_planted"),
         Workload("sweep_8192_f16", 1, 24, 8, 32, 32, 64, 8, 8, 2, "f16", 5, "pos_planted"),
         Workload("sweep_32768_f16", 1, 24, 8, 64, 64, 64, 8, 8, 2, "f16", 5, "pos_planted"),

@@ -21,13 +21,13 @@ TOL_LOWP = 2e-2
 
 
 def _grid(w):
-    return om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None)
+    return om.Grid(w.T, w.H, w.W, w.th, w.tw, Tk=w.Tkey if w.Tk else None, chunk_frames=w.chunk_frames)
 
 
 def _run_gpu(w, q, k, v, out_dtype=torch.float32):
     qd, kd, vd = (t.cuda() for t in (q, k, v))
     out = torch.empty(qd.shape, dtype=out_dtype, device=qd.device)
-    m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters, chunk_frames=w.chunk_frames)
     torch.cuda.synchronize()
     return out
 
@@ -96,9 +96,9 @@ def test_workload_sampled_heads(name, heads, cuda_lib):
     _compare(w, out, q, k, v, heads=heads)
 
 
-def _custom(dtype, T, H, W, d, th, tw, iters, Tk=0, B=2, heads=3, kind="pos_planted", seed=7):
-    return Workload(f"custom_{dtype}_{T}x{H}x{W}_d{d}_{th}x{tw}_it{iters}_Tk{Tk}", B, heads, T, H, W, d,
-                    th, tw, iters, dtype, seed, kind, Tk=Tk, planted=8)
+def _custom(dtype, T, H, W, d, th, tw, iters, Tk=0, B=2, heads=3, kind="pos_planted", seed=7, C=0):
+    return Workload(f"custom_{dtype}_{T}x{H}x{W}_d{d}_{th}x{tw}_it{iters}_Tk{Tk}_C{C}", B, heads, T, H, W, d,
+                    th, tw, iters, dtype, seed, kind, Tk=Tk, planted=8, chunk_frames=C)
 
 
 EDGE = [
@@ -242,3 +242,57 @@ def test_bf16_queries_beyond_the_f16_range_set_the_range_error(cuda_lib):
     torch.cuda.synchronize()
     assert m.device_error(reset=True) == 0
     assert torch.isfinite(out).all()
+
+
+# ---- frame-chunk causal mask (training over the whole sequence) ----------------
+
+CAUSAL = [
+    # chunk boundaries not aligned to the 64/128-tile blocks, several blocks per row
+    _custom("bf16", 8, 16, 16, 128, 4, 2, 2, C=2, B=1, heads=2),
+    _custom("bf16", 7, 12, 20, 128, 4, 4, 3, C=3),          # ragged last chunk
+    _custom("bf16", 5, 12, 20, 128, 4, 4, 1, C=1),          # one frame per chunk, one iteration
+    _custom("f16", 6, 16, 16, 64, 8, 8, 2, C=2),            # 64-position tiles
+    _custom("bf16", 4, 9, 10, 128, 3, 5, 2, C=2),           # b2 not a multiple of 8
+    _custom("f32", 5, 8, 12, 64, 2, 4, 2, C=2),             # CUDA-core path
+]
+
+
+@pytest.mark.parametrize("w", CAUSAL, ids=[w.name for w in CAUSAL])
+def test_chunk_causal_mask(w, cuda_lib):
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _compare(w, out, q, k, v)
+
+
+def test_chunk_causal_separable_is_masked_dense_attention(cuda_lib):
+    w = _custom("f32", 6, 8, 8, 64, 4, 4, 1, C=2, B=1, heads=2, kind="separable")
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v).double().cpu().numpy()
+    mask = om.frame_chunk_mask(w.T, w.T, w.H, w.W, w.chunk_frames)
+    ref = om.dense_attention(q.double().numpy(), k.double().numpy(), v.double().numpy(), mask=mask)
+    assert np.abs(out - ref).max() <= 1e-4
+
+
+def test_one_chunk_equals_the_bidirectional_call(cuda_lib):
+    w0 = _custom("bf16", 4, 12, 20, 128, 4, 4, 2)
+    q, k, v = make_inputs(w0)
+    a = _run_gpu(w0, q, k, v)
+    b = _run_gpu(_custom("bf16", 4, 12, 20, 128, 4, 4, 2, C=4), q, k, v)
+    assert torch.equal(a, b)
+
+
+def test_training_workload_sampled_heads(cuda_lib):
+    w = WORKLOADS["train_32760_bf16_causal"]
+    q, k, v = make_inputs(w)
+    out = _run_gpu(w, q, k, v)
+    _all_head_properties(out, v)
+    _compare(w, out, q, k, v, heads=[(1, 5)])
+
+
+def test_chunk_mask_with_a_kv_cache_is_unsupported(cuda_lib):
+    w = WORKLOADS["kvcache_4680x32760_bf16"]
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+    with pytest.raises(m.MonarchError) as e:
+        m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters, chunk_frames=1)
+    assert e.value.code == -4
