@@ -287,6 +287,66 @@ def monarch_attention(q, k, v, grid: Grid, iters: int, scale: float | None = Non
     return (out, states) if return_states else out
 
 
+def monarch_head_backward(qb, kb, vb, dyb, grid: Grid, scale: float):
+    """Gradients of one head's output for iters = 1 (the one-step regime of
+    finetuned models, gist.science explainer §2.C), self-attention.
+
+    The forward is D4-D6 + D8 with q~ = q (D3: block identity), optionally
+    under the D9 mask.  The chain rule, step by step (all per head, block order):
+      L step (per position a2):  y = L z, L = softmax_c1(s q.k~ + h)
+        dz = L^T dy;  dL = dy z^T;  dS = L * (dL - rowsum(L * dL))
+        dq += s dS k~;  dk~ = s dS^T q;  dh = colsum(dS)
+      R step (per tile c1):  k~ = R k, z = R v, h = -sum R log R,
+                             R = softmax_c2(s q.k)
+        dR = dk~ k^T + dz v^T - dh (log R + 1)
+        dk = R^T dk~ + s dSr^T q;  dv = R^T dz;  dq += s dSr k,
+        with dSr = R * (dR - rowsum(R * dR)).
+    qb, kb, vb, dyb: [b1, b2, d] in block order -> dq, dk, dv [b1, b2, d]."""
+    if grid.Tkey != grid.T:
+        raise NotImplementedError("the backward covers self-attention")
+    vis = grid.visible() if grid.chunk_frames else None
+    # forward quantities
+    R, h = _r_step(qb, kb, scale)                   # [c1, a2, c2], [c1, a2]
+    kt = np.matmul(R, kb)                           # [c1, a2, d]
+    z = np.matmul(R, vb)
+    L, _ = _l_step(qb, kt, h, scale, vis)           # [a2, a1, c1]
+    sw = lambda x: np.swapaxes(x, 0, 1)
+    # L step backward, positions a2 as the batch axis
+    dy_p, z_p, q_p, kt_p = sw(dyb), sw(z), sw(qb), sw(kt)
+    dz_p = np.matmul(np.swapaxes(L, 1, 2), dy_p)    # [a2, c1, d]
+    dL = np.matmul(dy_p, np.swapaxes(z_p, 1, 2))    # [a2, a1, c1]
+    dS = L * (dL - (L * dL).sum(axis=-1, keepdims=True))
+    dq_p = scale * np.matmul(dS, kt_p)              # [a2, a1, d]
+    dkt_p = scale * np.matmul(np.swapaxes(dS, 1, 2), q_p)
+    dh = dS.sum(axis=1).T                           # [c1, a2]
+    dz, dkt, dq = sw(dz_p), sw(dkt_p), sw(dq_p)
+    # R step backward, tiles c1 as the batch axis
+    dR = (np.matmul(dkt, np.swapaxes(kb, 1, 2)) + np.matmul(dz, np.swapaxes(vb, 1, 2))
+          - dh[..., None] * (np.log(R) + 1.0))      # [c1, a2, c2]
+    dSr = R * (dR - (R * dR).sum(axis=-1, keepdims=True))
+    dk = np.matmul(np.swapaxes(R, 1, 2), dkt) + scale * np.matmul(np.swapaxes(dSr, 1, 2), qb)
+    dv = np.matmul(np.swapaxes(R, 1, 2), dz)
+    dq = dq + scale * np.matmul(dSr, kb)
+    return dq, dk, dv
+
+
+def monarch_attention_backward(q, k, v, dy, grid: Grid, scale: float | None = None, heads=None):
+    """Gradients (dq, dk, dv) of sum(dy * monarch_attention(q, k, v, grid, 1)).
+    Tensors [B, Hh, N, d] in grid order; fp64.  ``heads`` as in
+    monarch_attention (other heads stay NaN)."""
+    grid.check()
+    q, k, v, dy = (np.asarray(x, dtype=np.float64) for x in (q, k, v, dy))
+    B, Hh, N, d = q.shape
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    idx = block_index(grid.T, grid.H, grid.W, grid.th, grid.tw)
+    dq, dk, dv = (np.full(q.shape, np.nan) for _ in range(3))
+    for b, h in (heads if heads is not None else [(b, h) for b in range(B) for h in range(Hh)]):
+        gq, gk, gv = monarch_head_backward(q[b, h][idx], k[b, h][idx], v[b, h][idx], dy[b, h][idx], grid, scale)
+        dq[b, h][idx], dk[b, h][idx], dv[b, h][idx] = gq, gk, gv
+    return dq, dk, dv
+
+
 def dense_attention(q, k, v, scale: float | None = None, mask=None):
     """Textbook softmax(s q k^T) v per (batch, head), fp64.  ``mask``
     [Nq, Nk] bool keeps only the allowed keys of each query."""
