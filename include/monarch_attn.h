@@ -1,5 +1,6 @@
 /*
- * monarch_attn.h -- C ABI of the B200 (sm_100a) Monarch video-attention forward.
+ * monarch_attn.h -- C ABI of the B200 (sm_100a) Monarch video-attention forward
+ * (and the backward of its one-step form).
  *
  * Operation (MonarchRT: Efficient Attention for Real-Time Video Generation;
  * gist.science explainer §2 "Methodology", §2.A "Block Alignment", §2.B "Tiled
@@ -109,6 +110,36 @@ int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
                         int dtype, int out_dtype, void* workspace, size_t workspace_bytes,
                         cudaStream_t stream);
 
+/* Backward of the one-step forward (iters = 1, self-attention: kv_len =
+ * T*H*W), with the frame-chunk causal mask of monarch_attn_fwd_ex when
+ * chunk_frames > 0.  One refinement step after finetuning is the regime the
+ * method trains and runs in (MonarchRT explainers §2.C, "Finetuning and
+ * Efficient Implementation"); the gradients are those of
+ * sum(dy * out) for out = monarch_attn_fwd(q, k, v, ..., iters = 1):
+ *   L step:  dS = L (dy.z - dy.y),  dq = s dS k~,  dk~ = s dS^T q,
+ *            dz = L^T dy,  dh = colsum(dS)
+ *   R step:  dSr = R (dk~ k^T + dz v^T - dh ln R - rowsum(R .)),
+ *            dk = R^T dk~ + s dSr^T q,  dv = R^T dz,  dq += s dSr k.
+ * q, k, v: [B, heads, T*H*W, d] in `dtype`; dy, dq, dk, dv: [B, heads,
+ * T*H*W, d] in `grad_dtype` (MONARCH_F32 or dtype), all caller-owned device
+ * memory, 16-byte aligned; dq, dk, dv are overwritten.  The forward factors
+ * are recomputed (nothing is kept from the forward call).  Arithmetic: fp32
+ * throughout.  Workspace: allocated stream-ordered from the library's pool,
+ * monarch_attn_bwd_workspace_bytes(...) bytes.  Asynchronous on `stream`;
+ * returns MONARCH_OK or a negative status (MONARCH_EINVAL for the checks of
+ * monarch_attn_fwd and a bad grad_dtype, MONARCH_EUNSUPPORTED as there). */
+int monarch_attn_bwd(const void* q, const void* k, const void* v, const void* dy,
+                     void* dq, void* dk, void* dv,
+                     int B, int heads, int T, int H, int W, int d,
+                     int tile_h, int tile_w, int chunk_frames,
+                     int dtype, int grad_dtype, cudaStream_t stream);
+
+/* Bytes of workspace monarch_attn_bwd takes for these arguments (0 on
+ * invalid arguments). */
+size_t monarch_attn_bwd_workspace_bytes(int B, int heads, int T, int H, int W, int d,
+                                        int tile_h, int tile_w, int chunk_frames,
+                                        int dtype, int grad_dtype);
+
 /* End-to-end variant on HOST buffers: copies q, k, v host->device, runs the
  * forward and copies out device->host, all on `stream`, then synchronises
  * `stream` before returning (so `out` is ready).  Device buffers are
@@ -163,7 +194,12 @@ enum {
   MONARCH_PHASE_L_LSE = 2,  /* L step LSE pass of a non-final iteration      */
   MONARCH_PHASE_L_OUT = 3,  /* final L step fused with y = L z and the store  */
   MONARCH_PHASE_L_COL = 4,  /* column pass q~ = L^T q / L^T 1                 */
-  MONARCH_NUM_PHASES = 5
+  /* backward (monarch_attn_bwd; its R-step recompute counts as R_STEP): */
+  MONARCH_PHASE_BWD_PREP = 5, /* row LSE and D = dy . y of the L step          */
+  MONARCH_PHASE_BWD_DQ = 6,   /* L-step part of dq, per query row               */
+  MONARCH_PHASE_BWD_DKV = 7,  /* dk~, dz, dh per key column                      */
+  MONARCH_PHASE_BWD_R = 8,    /* R-step backward per tile: dk, dv, dq finished */
+  MONARCH_NUM_PHASES = 9
 };
 
 /* Number of kernels this process has launched through the library (host

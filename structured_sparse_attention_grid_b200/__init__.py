@@ -1,6 +1,6 @@
 """Python binding of the B200 Monarch video-attention library (C ABI).
 
-Argument marshalling only: every step of the forward runs in the CUDA
+Argument marshalling only: every step of the forward and backward runs in the CUDA
 kernels of ``libmonarch_attn.so``.  PyTorch provides device memory and
 streams.  There is no fallback: if the library is missing, calls fail.
 """
@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmonarch_attn.so")
 
 MONARCH_F32, MONARCH_BF16, MONARCH_F16 = 0, 1, 2
-PHASES = ("qbar", "r_step", "l_lse", "l_out", "l_col")
+PHASES = ("qbar", "r_step", "l_lse", "l_out", "l_col", "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r")
 
 # Every symbol the header declares, with its ctypes signature.
 _SIGS = {
@@ -22,6 +22,8 @@ _SIGS = {
                          + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_fwd_ex": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "monarch_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int] * 11 + [ctypes.c_void_p]),
+    "monarch_attn_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 11),
     "monarch_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_int]),
     "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
@@ -117,6 +119,30 @@ def monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None, 
         _check(lib.monarch_attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                                     *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
+
+
+def monarch_attn_bwd(q, k, v, dy, dq, dk, dv, T, H, W, tile_h, tile_w, stream=None, chunk_frames=0):
+    """dq, dk, dv <- gradients of sum(dy * out) for the one-step forward
+    out = monarch_attn_fwd(q, k, v, ..., iters=1) (self-attention, optional
+    frame-chunk causal mask).  q, k, v in one dtype; dy, dq, dk, dv float32 or
+    q's dtype; all CUDA, contiguous [B, heads, T*H*W, d].  Asynchronous."""
+    lib = load_library()
+    _check_tensors(q, k, v, dy, dq, dk, dv)
+    B, heads, nq, d = q.shape
+    if nq != T * H * W:
+        raise ValueError(f"q has {nq} tokens, grid {T}x{H}x{W} has {T * H * W}")
+    for t in (k, v, dy, dq, dk, dv):
+        if tuple(t.shape) != tuple(q.shape):
+            raise ValueError("k, v, dy, dq, dk, dv must have q's shape (self-attention)")
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share a dtype")
+    g = _dtype_code(dy)
+    if any(_dtype_code(t) != g for t in (dq, dk, dv)):
+        raise TypeError("dy, dq, dk, dv must share a dtype")
+    _check(lib.monarch_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dy.data_ptr(), dq.data_ptr(),
+                                dk.data_ptr(), dv.data_ptr(), B, heads, T, H, W, d, tile_h, tile_w,
+                                int(chunk_frames), _dtype_code(q), g, _stream_ptr(stream)))
+    return dq, dk, dv
 
 
 def workspace_layout(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype_code):

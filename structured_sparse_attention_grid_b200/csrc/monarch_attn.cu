@@ -21,6 +21,7 @@
 #include "kernels_tc.cuh"
 #include "kernels_rtc.cuh"
 #include "kernels_l.cuh"
+#include "kernels_bwd.cuh"
 
 using namespace monarch;
 
@@ -85,7 +86,8 @@ template <typename F>
 void launch(int phase, cudaStream_t st, F&& f) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (debug_sync()) {
-    static const char* names[] = {"qbar", "r_step", "l_lse", "l_out", "l_col"};
+    static const char* names[] = {"qbar", "r_step", "l_lse", "l_out", "l_col",
+                                  "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r"};
     fprintf(stderr, "[monarch] launch %s ...\n", names[phase]);
     auto t0 = std::chrono::steady_clock::now();
     f();
@@ -463,6 +465,103 @@ int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* o
   }
 }
 
+// ---- backward (one-step forward, self-attention) -------------------------
+constexpr int kBwdRegions = 9;  // k~, z, h, lse, D, dqL, dk~, dz, dh
+
+struct BwdPlan {
+  Plan fwd;   // geometry and validation of the forward it differentiates
+  int grad_dtype;
+  size_t off[kBwdRegions];
+  size_t total;
+};
+
+int make_bwd_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int chunk_frames, int dtype,
+                  int grad_dtype, BwdPlan* bp) {
+  const long kv = (long)T * H * W;
+  int rc = make_plan(B, heads, T, H, W, d, th, tw, 1, kv, dtype, dtype, &bp->fwd, chunk_frames);
+  if (rc) return rc;
+  if (grad_dtype != dtype && grad_dtype != MONARCH_F32)
+    return fail(MONARCH_EINVAL, "grad_dtype %d must be MONARCH_F32 or the input dtype %d", grad_dtype, dtype);
+  bp->grad_dtype = grad_dtype;
+  const Geo& g = bp->fwd.g;
+  const size_t big = (size_t)g.BH * g.b2 * g.b1k * d * 4;
+  const size_t col = (size_t)g.BH * g.b2 * g.b1k_pad * 4;
+  const size_t row = (size_t)g.BH * g.b2 * g.b1q_pad * 4;
+  const size_t sizes[kBwdRegions] = {big, big, col, row, row, big, big, big, col};
+  size_t o = 0;
+  for (int i = 0; i < kBwdRegions; ++i) {
+    bp->off[i] = o;
+    o += align256(sizes[i]);
+  }
+  bp->total = o;
+  return MONARCH_OK;
+}
+
+template <typename T, typename TG, int D>
+void launch_l_bwd(const Geo& g, const T* q, const TG* dy, const Work& w, const BwdWork& bw, cudaStream_t st) {
+  constexpr int kRows = 16;
+  const dim3 rgrid((g.b1q + kRows - 1) / kRows, g.b2, g.BH);
+  const dim3 cgrid((g.b1k + kRows - 1) / kRows, g.b2, g.BH);
+  launch(MONARCH_PHASE_BWD_PREP, st, [&] { l_bwd_prep_simt<T, TG, D><<<rgrid, 32 * kRows, 0, st>>>(q, dy, w, bw, g); });
+  launch(MONARCH_PHASE_BWD_DQ, st, [&] { l_bwd_dq_simt<T, TG, D><<<rgrid, 32 * kRows, 0, st>>>(q, dy, w, bw, g); });
+  launch(MONARCH_PHASE_BWD_DKV, st, [&] { l_bwd_dkv_simt<T, TG, D><<<cgrid, 32 * kRows, 0, st>>>(q, dy, w, bw, g); });
+}
+
+// Recomputes the forward's R step (k~, z, h), then runs the L-step backward
+// passes and the per-tile R-step backward, which writes dq, dk, dv.
+template <typename T, typename TG>
+int run_bwd(const BwdPlan& bp, const T* q, const T* k, const T* v, const TG* dy, TG* dq, TG* dk, TG* dv,
+            char* ws, cudaStream_t st) {
+  const Geo& g = bp.fwd.g;
+  Work w = {};
+  w.kt = reinterpret_cast<float*>(ws + bp.off[0]);
+  w.z = reinterpret_cast<float*>(ws + bp.off[1]);
+  w.h = reinterpret_cast<float*>(ws + bp.off[2]);
+  w.lse = reinterpret_cast<float*>(ws + bp.off[3]);
+  BwdWork bw;
+  bw.dd = reinterpret_cast<float*>(ws + bp.off[4]);
+  bw.dqL = reinterpret_cast<float*>(ws + bp.off[5]);
+  bw.dkt = reinterpret_cast<float*>(ws + bp.off[6]);
+  bw.dz = reinterpret_cast<float*>(ws + bp.off[7]);
+  bw.dh = reinterpret_cast<float*>(ws + bp.off[8]);
+
+  const size_t r_smem = (size_t)(3 * g.b2 * g.d + g.b2 * (g.b2 + 1)) * sizeof(float);
+  cudaError_t e = allow_smem(r_step_simt<T>, r_smem);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(r_step)");
+  const size_t rb_smem = (size_t)r_bwd_smem_floats(g.b2, g.d) * sizeof(float);
+  if ((e = allow_smem(r_bwd_simt<T, TG>, rb_smem)) != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(r_bwd)");
+  launch(MONARCH_PHASE_R_STEP, st, [&] {
+    r_step_simt<T><<<dim3(g.b1k, g.BH), 128, r_smem, st>>>(q, k, v, w, g, QT_IDENTITY, 1);
+  });
+  if (g.d == 128) launch_l_bwd<T, TG, 128>(g, q, dy, w, bw, st);
+  else launch_l_bwd<T, TG, 64>(g, q, dy, w, bw, st);
+  launch(MONARCH_PHASE_BWD_R, st, [&] {
+    r_bwd_simt<T, TG><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
+  });
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return MONARCH_OK;
+}
+
+template <typename T>
+int dispatch_bwd_grad(const BwdPlan& bp, const void* q, const void* k, const void* v, const void* dy, void* dq,
+                      void* dk, void* dv, char* ws, cudaStream_t st) {
+  if (bp.grad_dtype == MONARCH_F32)
+    return run_bwd<T, float>(bp, (const T*)q, (const T*)k, (const T*)v, (const float*)dy, (float*)dq, (float*)dk,
+                             (float*)dv, ws, st);
+  return run_bwd<T, T>(bp, (const T*)q, (const T*)k, (const T*)v, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws, st);
+}
+
+int dispatch_bwd(const BwdPlan& bp, const void* q, const void* k, const void* v, const void* dy, void* dq,
+                 void* dk, void* dv, void* ws, cudaStream_t st) {
+  char* w = static_cast<char*>(ws);
+  switch (bp.fwd.dtype) {
+    case MONARCH_F32: return dispatch_bwd_grad<float>(bp, q, k, v, dy, dq, dk, dv, w, st);
+    case MONARCH_BF16: return dispatch_bwd_grad<__nv_bfloat16>(bp, q, k, v, dy, dq, dk, dv, w, st);
+    default: return dispatch_bwd_grad<__half>(bp, q, k, v, dy, dq, dk, dv, w, st);
+  }
+}
+
 // Stream-ordered workspace comes from a per-device pool owned by the library
 // that keeps freed memory (release threshold = max), so repeated calls reuse
 // it without returning memory to the driver between calls.
@@ -609,6 +708,39 @@ int monarch_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, 
     return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", p.total, cudaGetErrorString(e));
   }
   rc = dispatch(p, q, k, v, out, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+size_t monarch_attn_bwd_workspace_bytes(int B, int heads, int T, int H, int W, int d, int tile_h, int tile_w,
+                                        int chunk_frames, int dtype, int grad_dtype) {
+  BwdPlan bp;
+  if (make_bwd_plan(B, heads, T, H, W, d, tile_h, tile_w, chunk_frames, dtype, grad_dtype, &bp) != MONARCH_OK)
+    return 0;
+  return bp.total;
+}
+
+int monarch_attn_bwd(const void* q, const void* k, const void* v, const void* dy, void* dq, void* dk, void* dv,
+                     int B, int heads, int T, int H, int W, int d, int tile_h, int tile_w, int chunk_frames,
+                     int dtype, int grad_dtype, cudaStream_t stream) {
+  g_err.clear();
+  BwdPlan bp;
+  int rc = make_bwd_plan(B, heads, T, H, W, d, tile_h, tile_w, chunk_frames, dtype, grad_dtype, &bp);
+  if (rc) return rc;
+  if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v")) ||
+      (rc = check_ptr(dy, "dy")) || (rc = check_ptr(dq, "dq")) || (rc = check_ptr(dk, "dk")) ||
+      (rc = check_ptr(dv, "dv")))
+    return rc;
+  void* ws = nullptr;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bp.total, pool, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", bp.total, cudaGetErrorString(e));
+  }
+  rc = dispatch_bwd(bp, q, k, v, dy, dq, dk, dv, ws, stream);
   e = cudaFreeAsync(ws, stream);
   if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
   return rc;

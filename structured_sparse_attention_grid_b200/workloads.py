@@ -187,3 +187,14 @@ def make_inputs(w: Workload):
             k[b, h] = _round(kk, w.dtype)
             noise_q[b][h] = noise_k[b][h] = None
     return q, k, v
+
+
+def make_cotangent(w: Workload, dtype: str = "f32"):
+    """Seeded output gradient dy for the backward: [B, heads, Nq, d] standard
+    normal entries rounded to `dtype` (CPU torch tensor)."""
+    rng = np.random.default_rng(w.seed + 1_000_003)
+    dy = torch.empty((w.B, w.heads, w.Nq, w.d), dtype=DTYPES[dtype])
+    for b in range(w.B):
+        for h in range(w.heads):
+            dy[b, h] = _round(rng.standard_normal((w.Nq, w.d)), dtype)
+    return dy

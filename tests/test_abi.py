@@ -116,3 +116,36 @@ def test_product_path_does_not_import_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(import|from)\s+oracle\b", src, flags=re.M), f
                 assert not any("oracle" in inc for inc in re.findall(r"#include.*", src)), f
+
+
+def _bwd(lib, ptrs=(0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0x6000, 0x7000), **kw):
+    c = dict(B=1, heads=2, T=3, H=8, W=12, d=64, th=2, tw=4, C=0, dt=1, gdt=0)
+    c.update(kw)
+    return lib.monarch_attn_bwd(*ptrs, c["B"], c["heads"], c["T"], c["H"], c["W"], c["d"], c["th"], c["tw"],
+                                c["C"], c["dt"], c["gdt"], None)
+
+
+@pytest.mark.parametrize("bad,needle", [
+    (dict(H=9), "tile"),
+    (dict(d=80), "head_dim"),
+    (dict(gdt=2), "grad_dtype"),     # f16 gradients of bf16 inputs
+    (dict(dt=5), "dtype"),
+    (dict(C=-1), "chunk_frames"),
+])
+def test_backward_validates_on_the_host(lib, bad, needle):
+    assert _bwd(lib, **bad) == -1
+    assert needle in lib.monarch_attn_last_error().decode()
+
+
+def test_backward_rejects_null_and_misaligned_pointers(lib):
+    assert _bwd(lib, ptrs=(0x1000, 0x2000, 0x3000, None, 0x5000, 0x6000, 0x7000)) == -1
+    assert "dy is null" in lib.monarch_attn_last_error().decode()
+    assert _bwd(lib, ptrs=(0x1000, 0x2000, 0x3000, 0x4000, 0x5004, 0x6000, 0x7000)) == -1
+    assert "dq is not 16-byte aligned" in lib.monarch_attn_last_error().decode()
+
+
+def test_backward_workspace_holds_the_gradient_intermediates(lib):
+    n = lib.monarch_attn_bwd_workspace_bytes(1, 12, 3, 30, 52, 128, 6, 4, 0, 1, 0)
+    big = 12 * 24 * 195 * 128 * 4   # fp32 k~, z, dqL, dk~, dz
+    assert n >= 5 * big + 4 * 12 * 24 * 195 * 4
+    assert lib.monarch_attn_bwd_workspace_bytes(1, 12, 3, 30, 52, 128, 6, 4, 0, 1, 2) == 0

@@ -112,3 +112,15 @@ def test_entropy_plus_one_cancels_in_softmax_backward(monkeypatch):
     monkeypatch.setattr(om, "monarch_head_backward",
                         _mutant("- dh[..., None] * (np.log(R) + 1.0)", "- dh[..., None] * np.log(R)"))
     assert _fd_ok()
+
+
+@pytest.mark.parametrize("g", [om.Grid(4, 6, 8, 2, 4), om.Grid(6, 4, 4, 2, 2, chunk_frames=2)],
+                         ids=["bidirectional", "chunk_causal"])
+def test_gradient_invariants_of_a_row_stochastic_operator(g):
+    """Rows of M sum to 1, so sum_tokens dv = sum_tokens dy; one shift of every
+    key leaves R and every visible row of L unchanged, so sum_tokens dk = 0."""
+    q, k, v, dy = _inputs(g, 16, seed=11)
+    dq, dk, dv = om.monarch_attention_backward(q, k, v, dy, g)
+    assert np.allclose(dv.sum(axis=2), dy.sum(axis=2), rtol=0, atol=1e-10)
+    assert np.abs(dk.sum(axis=2)).max() <= 1e-10 * np.abs(dk).sum(axis=2).max()
+    assert np.isfinite(dq).all()
