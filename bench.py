@@ -32,11 +32,13 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
-from structured_sparse_attention_grid_b200.workloads import WORKLOADS, make_inputs  # noqa: E402
+from structured_sparse_attention_grid_b200.workloads import WORKLOADS, make_cotangent, make_inputs  # noqa: E402
 
 METRIC = "Monarch-attn ms/call & effective TFLOP/s, bf16, N=4680–32760; % roofline"
 DEFAULT_WORKLOAD = "chunk_4680_bf16"
 L2_BYTES = 126 * 2**20
+# FP32 FMA ceiling of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
+ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 
 def load_peaks():
@@ -89,6 +91,18 @@ def work_model(w):
     }
     return dict(flops=flops_total, io_bytes=nq + 2 * nk + no, dense_flops=4.0 * BH * w.Nq * w.Nk * w.d * fv,
                 phases=phases, FL=FL, FR=FR, visible_fraction=fv)
+
+
+def backward_work_model(w):
+    """Algorithmic FLOPs of the backward of the one-step forward (gradient
+    contractions only, the forward recompute not counted): L step dL, dq, dk~,
+    dz (4 F_L); R step dR (2 F_R), dk (2 F_R), dv and dq (2 F_R).  Per kernel,
+    the dot-product work it performs (recompute included), for its roofline."""
+    m = work_model(w)
+    FL, FR, BH = m["FL"], m["FR"], w.B * w.heads
+    return dict(flops=BH * (4 * FL + 6 * FR),
+                phases={"bwd_prep": BH * 2 * FL, "bwd_dq": BH * 3 * FL, "bwd_dkv": BH * 4 * FL,
+                        "bwd_r": BH * 5 * FR, "r_step": BH * 3 * FR})
 
 
 # ---------------------------------------------------------------------------
@@ -247,6 +261,7 @@ def run_ours(args, rank, world, device):
 
     call_roof_ms = 1e3 * max(model["flops"] / (peaks["bf16_tflops"] * 1e12), io_bytes / (peaks["hbm_gbs"] * 1e9))
     dense = dense_context(qd, kd, vd, model, flush if flush_l2 else None, stream, ms)
+    backward = backward_line(m, w, qd, kd, vd, flush if flush_l2 else None, stream)
 
     # End to end (copies inside the timed region): the host-buffer entry point,
     # or, with the causal mask (not an argument of that entry point), pinned
@@ -318,8 +333,60 @@ def run_ours(args, rank, world, device):
         "gpu_launches": launches,
         "clocks": clocks.summary(),
         "dense_context": dense,
+        "backward": backward,
     }
     return rec, (q, k, v, w)
+
+
+def backward_line(m, w, qd, kd, vd, flush, stream):
+    """The backward of the one-step forward (the finetuned regime) on the same
+    q, k, v with a seeded cotangent and f32 gradients: ms per call, effective
+    TFLOP/s of its algorithmic FLOPs and the roofline of its dominant kernel,
+    all from CUDA events on the launching stream."""
+    if w.Tkey != w.T:
+        return {"impl": "not defined: the backward is for self-attention"}
+    bm = backward_work_model(w)
+    dy = make_cotangent(w, "f32").to(qd.device)
+    dq, dk, dv = (torch.empty_like(dy) for _ in range(3))
+
+    def call():
+        m.monarch_attn_bwd(qd, kd, vd, dy, dq, dk, dv, w.T, w.H, w.W, w.th, w.tw, stream=stream,
+                           chunk_frames=w.chunk_frames)
+
+    for _ in range(3):
+        call()
+    torch.cuda.synchronize()
+    n = 3 if bm["flops"] > 2e11 else 10
+    times = []
+    for _ in range(n):
+        if flush is not None:
+            flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        call()
+        b.record(stream)
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    m.profile_enable(True)
+    m.profile_read(reset=True)
+    if flush is not None:
+        flush.zero_()
+    call()
+    torch.cuda.synchronize()
+    prof = m.profile_read(reset=True)
+    m.profile_enable(False)
+    kernels = {p: prof[p][0] / prof[p][1] for p in prof if prof[p][1] > 0}
+    dom = max(kernels, key=kernels.get)
+    achieved = bm["phases"][dom] / (kernels[dom] * 1e-3) / 1e12
+    return {"workload": w.name, "iters": 1, "grad_dtype": "f32", "ms_per_call": ms,
+            "value": bm["flops"] / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "gflop_per_call": bm["flops"] / 1e9,
+            "kernels_ms": kernels,
+            "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": ALU_F32_TFLOPS,
+                         "unit": "TFLOP/s", "frac": achieved / ALU_F32_TFLOPS, "traffic": None,
+                         "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
 
 
 def dense_context(qd, kd, vd, model, flush, stream, monarch_ms):
