@@ -37,6 +37,13 @@ from structured_sparse_attention_grid_b200.workloads import WORKLOADS, make_cota
 METRIC = "Monarch-attn ms/call & effective TFLOP/s, bf16, N=4680–32760; % roofline"
 DEFAULT_WORKLOAD = "chunk_4680_bf16"
 L2_BYTES = 126 * 2**20
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) of a
+# workload's dominant kernel from an ncu capture of the current kernel code,
+# scaled to the workload's heads where the capture used fewer (profiles/);
+# a kernel without a capture of its current code reports null.
+NCU_TRAFFIC = {
+    ("full_32760_bf16", "l_col"): 879.8e6,   # 293.3 MB at 8 heads x 3
+}
 # FP32 FMA ceiling of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
@@ -254,7 +261,8 @@ def run_ours(args, rank, world, device):
         roof = {"bound": "hbm", "achieved": ph["bytes"] / (dom_ms * 1e-3) / 1e9,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = NCU_TRAFFIC.get((w.name, dom))
+    roof["traffic_unit"] = "bytes per launch (ncu DRAM read + write)"
     roof["kernel"] = dom
     roof["launch_ms"] = dom_ms
     roof["peak_source"] = peaks["source"]
@@ -497,16 +505,24 @@ def run_reference(args, rank, world):
 
 
 def profile_calls(args):
-    """A bare run of the workload for profiler captures: no timing, no bench line."""
+    """A bare run of the workload for profiler captures: no timing, no bench
+    line.  --profile-pass bwd runs the backward (f32 gradients) instead."""
     import structured_sparse_attention_grid_b200 as m
     w = WORKLOADS[args.workload]
     q, k, v = (t.cuda() for t in make_inputs(w))
-    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
-    for _ in range(args.profile_calls):
-        m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    if args.profile_pass == "bwd":
+        dy = make_cotangent(w, "f32").cuda()
+        dq, dk, dv = (torch.empty_like(dy) for _ in range(3))
+        for _ in range(args.profile_calls):
+            m.monarch_attn_bwd(q, k, v, dy, dq, dk, dv, w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
+    else:
+        out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+        for _ in range(args.profile_calls):
+            m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters, chunk_frames=w.chunk_frames)
     torch.cuda.synchronize()
     err = m.device_error()
-    print(f"profile case {w.name} B={w.B} heads={w.heads} calls={args.profile_calls} device_error={err}")
+    print(f"profile case {w.name} ({args.profile_pass}) B={w.B} heads={w.heads} calls={args.profile_calls} "
+          f"device_error={err}")
     if err:
         raise SystemExit(1)
 
@@ -523,6 +539,8 @@ def main():
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiler cases)")
     ap.add_argument("--profile-calls", type=int, default=0,
                     help="run this many forward calls of the workload and exit (for ncu); no timing")
+    ap.add_argument("--profile-pass", default="fwd", choices=["fwd", "bwd"],
+                    help="which pass --profile-calls runs")
     args = ap.parse_args()
     if args.batch or args.heads:
         import dataclasses
