@@ -1,0 +1,529 @@
+// tcgen05 kernels of the L-step backward for bf16 / f16 inputs (one-step
+// forward, self-attention, optional frame-chunk causal mask).  Per position
+// a2 the L step is a softmax attention of the queries q over the key tiles k~
+// with values z and a per-key bias h, so its backward is
+//   P = 2^(s log2(e) q.k~ + h - lse),  dS = P (dy.z - D),  D = dy.y,
+//   dq = s dS k~,  dk~ = s dS^T q,  dz = P^T dy,  dh = colsum(dS).
+//
+// Two kernels, each with 128 rows on the TMEM lanes and 128-wide blocks of
+// the other side streamed through shared memory:
+//   l_bwd_kv: rows = key tiles c1, blocks of queries.
+//     X = S^T = k~ q^T,  Y = dP^T = z dy^T        (shared-memory operands)
+//     P^T, dS^T written over X, Y as f16 hi/lo    (A operands in TMEM)
+//     dz += P^T dy,  dk~ += dS^T q                (accumulators in TMEM)
+//   l_bwd_q:  rows = queries a1, blocks of key tiles.
+//     X = S = q k~^T,  Y = dP = dy z^T;  dS over Y;  dq += dS k~.
+//
+// Precision: dS = P (dP - D) cancels where P is peaked, so a relative error e
+// of dP becomes e |z| / |z - y| in dS.  Every operand of every product is
+// therefore carried as f16 hi + lo planes where it is not exact: k~, z (from
+// the R step), dy (scaled by a power of two sigma per head so that
+// max |sigma dy| lies in [1/2, 1)), P and dS; q is exact in f16.  A product
+// of two split operands takes three MMAs (hi hi, lo hi, hi lo).  dS is scaled
+// by 2^kDsShift before its split; fp32 accumulation throughout.
+//
+// TMEM (512 columns): X [0, 128), Y [128, 256), accumulators from 256.  A
+// 32-column chunk of X or Y that held 32 scores holds, after the softmax,
+// the hi values of those 32 entries in its first 16 columns and the lo values
+// in the last 16 (two f16 per column), the layout of an A operand in TMEM.
+// Each block's products that read P or dS are issued before the next block's
+// score products, and one thread's MMAs run in issue order, so the next
+// scores never overwrite an operand still in use.
+#pragma once
+
+#include "tc_common.cuh"
+
+namespace monarch {
+namespace tcb {
+
+using tc::kBox;
+constexpr int kSoftWarps = 8;                  // 4 lane quadrants x 2 column halves
+constexpr int kThreads = 32 * (kSoftWarps + 2);
+constexpr int kMmaWarp = kSoftWarps;
+constexpr int kLoadWarp = kSoftWarps + 1;
+constexpr int kSoftThreads = 32 * kSoftWarps;
+constexpr int kBlk = 128;                      // rows per tile and columns per streamed block
+constexpr float kDsShift = 16.f;               // dS is split as 16 dS (range and subnormals)
+
+struct BwdMaps {
+  CUtensorMap dy;   // sigma dy planes  {d, b1q, 2*BH*b2}  box {64, 64, 1}  (f16)
+  CUtensorMap dd;   // sigma D          {b1q_pad, BH*b2}   box {64, 1}      (f32)
+};
+
+// Power-of-two scale that maps the largest |dy| of a head into [1/2, 1).
+__device__ __forceinline__ float dy_sigma(float amax) {
+  if (!(amax > 0.f) || !(amax < INFINITY)) return 1.f;
+  int e;
+  frexpf(amax, &e);
+  e = max(-120, min(120, e));
+  return ldexpf(1.f, -e);
+}
+
+template <int D>
+constexpr size_t kv_smem() {
+  constexpr int NH = D / 64;
+  return (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + (size_t)NH * 2 * kBox /* q */ +
+         (size_t)2 * NH * 2 * kBox /* dy planes */ + 2 * kBlk * 4 /* lse, D */ + 2 * kBlk * 4 /* dh halves */ +
+         16 * 8;
+}
+
+template <int D>
+constexpr size_t q_smem() {
+  constexpr int NH = D / 64;
+  return (size_t)NH * 2 * kBox /* q */ + (size_t)2 * NH * 2 * kBox /* dy planes */ +
+         (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + kBlk * 4 /* h */ + 16 * 8;
+}
+
+// One 32-column chunk of the softmax: reads 32 scores X and 32 values Y of
+// this thread's row, forms P and dS, and writes their hi/lo f16 planes over
+// the chunk (P over X when WRITE_P, dS over Y).  Column j of the chunk has
+// base-2 offset off[j] (h - lse, per column or per row) and D value dd[j];
+// keep(j) masks it.  Accumulates dS into dsum; tracks max |2^shift dS|.
+template <bool WRITE_P, typename Off, typename Dv, typename Keep>
+__device__ __forceinline__ void softmax_chunk(uint32_t tx, uint32_t ty, float sl2, Off off, Dv dd, Keep keep,
+                                              float& dsum, float& dmax) {
+  uint32_t xr[32], yr[32];
+  ptx::tmem_ld32(tx, xr);
+  ptx::tmem_ld32(ty, yr);
+  ptx::tmem_wait_ld();
+#pragma unroll
+  for (int h16 = 0; h16 < 2; ++h16) {
+    uint32_t phi[8], plo[8], shi[8], slo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int j = 16 * h16 + 2 * e;
+      float p0 = ptx::ex2(fmaf(__uint_as_float(xr[j]), sl2, off(j)));
+      float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
+      if (!keep(j)) p0 = 0.f;
+      if (!keep(j + 1)) p1 = 0.f;
+      const float d0 = p0 * (__uint_as_float(yr[j]) - dd(j));
+      const float d1 = p1 * (__uint_as_float(yr[j + 1]) - dd(j + 1));
+      dsum += d0 + d1;
+      const float2 ds = make_float2(d0 * kDsShift, d1 * kDsShift);
+      dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
+      tc::split2<__half>(ds, shi[e], slo[e]);
+      if (WRITE_P) tc::split2<__half>(make_float2(p0, p1), phi[e], plo[e]);
+    }
+    if (WRITE_P) {
+      ptx::tmem_st8(tx + 8 * h16, phi);
+      ptx::tmem_st8(tx + 16 + 8 * h16, plo);
+    }
+    ptx::tmem_st8(ty + 8 * h16, shi);
+    ptx::tmem_st8(ty + 16 + 8 * h16, slo);
+  }
+}
+
+// Writes 16 accumulator columns of this thread's row, times `scale`, as f32.
+__device__ __forceinline__ void store_acc16(uint32_t taddr, float scale, float* dst, bool ok) {
+  uint32_t o[16];
+  ptx::tmem_ld16(taddr, o);
+  ptx::tmem_wait_ld();
+  if (!ok) return;
+  float4* p = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    p[v] = make_float4(__uint_as_float(o[4 * v]) * scale, __uint_as_float(o[4 * v + 1]) * scale,
+                       __uint_as_float(o[4 * v + 2]) * scale, __uint_as_float(o[4 * v + 3]) * scale);
+}
+
+// ===========================================================================
+// dk~, dz, dh for 128 key tiles of one (head, position a2).
+// grid (ceil(b1k/128), b2, BH), block kThreads, dynamic smem kv_smem<D>().
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps bmaps, const float* __restrict__ hbuf,
+         const unsigned* __restrict__ amax, float* __restrict__ dkt, float* __restrict__ dz, float* __restrict__ dh,
+         Geo g) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t kPl = NH * 2 * kBox;   // one 128-row operand plane: [d half][row half][64 rows][128 B]
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
+  if (tc::smem_misaligned(smem_raw)) return;
+  uint8_t* sK = smem_raw;               // k~ [plane]
+  uint8_t* sZ = sK + 2 * kPl;           // z  [plane]
+  uint8_t* sQ = sZ + 2 * kPl;           // q
+  uint8_t* sY = sQ + kPl;               // sigma dy [plane]
+  float* sL = reinterpret_cast<float*>(sY + 2 * kPl);   // lse of the block's queries
+  float* sD = sL + kBlk;                                // sigma D
+  float* sX = sD + kBlk;                                // dh of the two column halves
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * kBlk);
+  uint64_t* k_full = bar + 0;
+  uint64_t* q_full = bar + 1;
+  uint64_t* q_free = bar + 2;
+  uint64_t* s_full = bar + 3;
+  uint64_t* p_full = bar + 4;
+  uint64_t* o_done = bar + 5;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 6);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int a2 = blockIdx.y, bh = blockIdx.z;
+  const int kb = blockIdx.x * kBlk;
+  const int zrow = bh * g.b2 + a2;
+  const int rows = g.BH * g.b2;
+  const int nqb = (g.b1q + kBlk - 1) / kBlk;
+  const int qb0 = query_start(g, kb) / kBlk;   // earlier query blocks see none of these key tiles
+  const int nblk = nqb - qb0;
+
+  if (tid == 0) {
+    ptx::mbar_init(k_full, 1);
+    ptx::mbar_init(q_full, 1);
+    ptx::mbar_init(q_free, 1);
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(p_full, kSoftWarps);
+    ptx::mbar_init(o_done, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  ptx::griddep_wait();
+  const uint32_t tmem = *sTmem;
+  const uint32_t tX = tmem, tY = tmem + 128, tZ = tmem + 256, tK = tmem + 256 + D;
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      ptx::mbar_expect_tx(k_full, 4 * kPl);
+      for (int p = 0; p < 2; ++p)
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh) {
+            const int off = p * kPl + hf * 2 * kBox + rh * kBox;
+            ptx::tma_load_3d(sK + off, &maps.kt, k_full, hf * 64, kb + rh * 64, p * rows + zrow);
+            ptx::tma_load_3d(sZ + off, &maps.z, k_full, hf * 64, kb + rh * 64, p * rows + zrow);
+          }
+      bool ok = true;
+      for (int j = 0; j < nblk && ok; ++j) {
+        const int q0 = (qb0 + j) * kBlk;
+        if (j > 0) ok = ptx::mbar_wait(q_free, (j - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(q_full, 3 * kPl + 2 * kBlk * 4);
+        for (int hf = 0; hf < NH; ++hf)
+          for (int rh = 0; rh < 2; ++rh) {
+            ptx::tma_load_3d(sQ + hf * 2 * kBox + rh * kBox, &maps.qb, q_full, hf * 64, q0 + rh * 64, zrow);
+            for (int p = 0; p < 2; ++p)
+              ptx::tma_load_3d(sY + p * kPl + hf * 2 * kBox + rh * kBox, &bmaps.dy, q_full, hf * 64, q0 + rh * 64,
+                               p * rows + zrow);
+          }
+        for (int rh = 0; rh < 2; ++rh) {
+          tc::tma_load_2d(sL + rh * 64, &maps.lse, q_full, q0 + rh * 64, zrow);
+          tc::tma_load_2d(sD + rh * 64, &bmaps.dd, q_full, q0 + rh * 64, zrow);
+        }
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idS = ptx::idesc_f16(128, kBlk, 0, 0, 0);
+      constexpr uint32_t idA = ptx::idesc_f16(128, D, 0, 0, 1);
+      const uint32_t aK = ptx::smem_u32(sK), aZ = ptx::smem_u32(sZ), aQ = ptx::smem_u32(sQ), aY = ptx::smem_u32(sY);
+      // score-like product: rows x 128 columns over K = d
+      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) {
+        const uint64_t da = ptx::sw128_desc(a, 16, 1024), db = ptx::sw128_desc(b, 16, 1024);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ptx::mma_f16_ss(td, da + ((hf * 2 * kBox + k4 * 32) >> 4), db + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
+                            !(first && hf == 0 && k4 == 0));
+      };
+      // accumulation: acc += A (TMEM, planes pa over 128 K columns) * B (MN-major, K = 128 rows, N = d)
+      auto accum = [&](uint32_t tacc, uint32_t ta, int pa, uint32_t b, bool first) {
+        const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          ptx::mma_f16_ts(tacc, ta + (kk >> 1) * 32 + pa * 16 + (kk & 1) * 8, db + ((kk * 2048) >> 4), idA,
+                          !(first && kk == 0));
+      };
+      bool ok = ptx::mbar_wait(k_full, 0);
+      for (int j = 0; j < nblk && ok; ++j) {
+        ok = ptx::mbar_wait(q_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
+        scores(tX, aK, aQ, true);              // S^T = k~_hi q^T + k~_lo q^T
+        scores(tX, aK + kPl, aQ, false);
+        scores(tY, aZ, aY, true);              // dP^T = z dy^T (hi hi, lo hi, hi lo)
+        scores(tY, aZ + kPl, aY, false);
+        scores(tY, aZ, aY + kPl, false);
+        ptx::mma_commit(s_full);
+        ok = ptx::mbar_wait(p_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
+        accum(tZ, tX, 0, aY, j == 0);          // dz += P^T dy
+        accum(tZ, tX, 1, aY, false);
+        accum(tZ, tX, 0, aY + kPl, false);
+        accum(tK, tY, 0, aQ, j == 0);          // dk~ += dS^T q
+        accum(tK, tY, 1, aQ, false);
+        ptx::mma_commit(q_free);
+      }
+      ptx::mma_commit(o_done);
+    }
+  } else {
+    const int qd = warp & 3, hf = warp >> 2;
+    const int r = 32 * qd + lane;
+    const int c1 = kb + r;
+    const bool row_ok = c1 < g.b1k;
+    const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+    const int qstart = query_start(g, row_ok ? c1 : g.b1k - 1);
+    const float hb = row_ok ? hbuf[(long long)zrow * g.b1k_pad + c1] : 0.f;
+    float dsum = 0.f, dmax = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const int q0 = (qb0 + j) * kBlk;
+      ok = ok && ptx::mbar_wait(s_full, j & 1) && ptx::mbar_wait(q_full, j & 1);
+      ptx::tc_fence_after();
+      const int lim = min(kBlk, g.b1q - q0);   // valid queries of the block
+      const int lo = qstart - q0;              // queries below this one do not see the key tile
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int cb = 64 * hf + 32 * hh;
+        const float* l = sL + cb;
+        const float* dv = sD + cb;
+        softmax_chunk<true>(
+            tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hb - l[jj]; },
+            [&](int jj) { return dv[jj]; }, [&](int jj) { return cb + jj < lim && cb + jj >= lo; }, dsum, dmax);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(p_full);
+    }
+    if (dmax >= 65504.f) atomicExch(&ptx::g_device_error, ptx::kErrRange);
+    sX[hf * kBlk + r] = dsum;
+    ptx::named_bar(1, kSoftThreads);
+    ok = ok && ptx::mbar_wait(o_done, 0);
+    ptx::tc_fence_after();
+    const float inv = 1.f / dy_sigma(__uint_as_float(amax[bh]));
+    const float s = g.sl2 * (1.f / kLog2e);
+    const long long o = ((long long)zrow * g.b1k + (row_ok ? c1 : 0)) * D + hf * (D / 2);
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc) {
+      store_acc16(tZ + lane_off + hf * (D / 2) + 16 * cc, inv, dz + o + 16 * cc, row_ok && ok);
+      store_acc16(tK + lane_off + hf * (D / 2) + 16 * cc, inv * s / kDsShift, dkt + o + 16 * cc, row_ok && ok);
+    }
+    if (hf == 0 && row_ok && ok) dh[(long long)zrow * g.b1k_pad + c1] = (dsum + sX[kBlk + r]) * inv;
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ===========================================================================
+// L-step dq for 128 queries of one (head, position a2).
+// grid (ceil(b1q/128), b2, BH), block kThreads, dynamic smem q_smem<D>().
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps bmaps, const float* __restrict__ lse,
+        const float* __restrict__ ddv, const unsigned* __restrict__ amax, float* __restrict__ dq, Geo g) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t kPl = NH * 2 * kBox;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  ptx::griddep_launch();
+  if (tc::smem_misaligned(smem_raw)) return;
+  uint8_t* sQ = smem_raw;               // q
+  uint8_t* sY = sQ + kPl;               // sigma dy [plane]
+  uint8_t* sK = sY + 2 * kPl;           // k~ [plane]
+  uint8_t* sZ = sK + 2 * kPl;           // z  [plane]
+  float* sH = reinterpret_cast<float*>(sZ + 2 * kPl);   // h of the block's key tiles (bits)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sH + kBlk);
+  uint64_t* c_full = bar + 0;
+  uint64_t* k_full = bar + 1;
+  uint64_t* k_free = bar + 2;
+  uint64_t* s_full = bar + 3;
+  uint64_t* p_full = bar + 4;
+  uint64_t* o_done = bar + 5;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 6);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int a2 = blockIdx.y, bh = blockIdx.z;
+  const int ab = blockIdx.x * kBlk;
+  const int zrow = bh * g.b2 + a2;
+  const int rows = g.BH * g.b2;
+  const int kmax = key_limit(g, min(ab + kBlk, g.b1q) - 1);   // key tiles any row of this CTA sees
+  const int nblk = (kmax + kBlk - 1) / kBlk;
+
+  if (tid == 0) {
+    ptx::mbar_init(c_full, 1);
+    ptx::mbar_init(k_full, 1);
+    ptx::mbar_init(k_free, 1);
+    ptx::mbar_init(s_full, 1);
+    ptx::mbar_init(p_full, kSoftWarps);
+    ptx::mbar_init(o_done, 1);
+    ptx::fence_mbar_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  ptx::griddep_wait();
+  const uint32_t tmem = *sTmem;
+  const uint32_t tX = tmem, tY = tmem + 128, tA = tmem + 256;
+
+  if (warp == kLoadWarp) {
+    if (lane == 0) {
+      ptx::mbar_expect_tx(c_full, 3 * kPl);
+      for (int hf = 0; hf < NH; ++hf)
+        for (int rh = 0; rh < 2; ++rh) {
+          ptx::tma_load_3d(sQ + hf * 2 * kBox + rh * kBox, &maps.qb, c_full, hf * 64, ab + rh * 64, zrow);
+          for (int p = 0; p < 2; ++p)
+            ptx::tma_load_3d(sY + p * kPl + hf * 2 * kBox + rh * kBox, &bmaps.dy, c_full, hf * 64, ab + rh * 64,
+                             p * rows + zrow);
+        }
+      bool ok = true;
+      for (int j = 0; j < nblk && ok; ++j) {
+        if (j > 0) ok = ptx::mbar_wait(k_free, (j - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(k_full, 4 * kPl + kBlk * 4);
+        for (int p = 0; p < 2; ++p)
+          for (int hf = 0; hf < NH; ++hf)
+            for (int rh = 0; rh < 2; ++rh) {
+              const int off = p * kPl + hf * 2 * kBox + rh * kBox;
+              ptx::tma_load_3d(sK + off, &maps.kt, k_full, hf * 64, j * kBlk + rh * 64, p * rows + zrow);
+              ptx::tma_load_3d(sZ + off, &maps.z, k_full, hf * 64, j * kBlk + rh * 64, p * rows + zrow);
+            }
+        for (int rh = 0; rh < 2; ++rh) tc::tma_load_2d(sH + rh * 64, &maps.h, k_full, j * kBlk + rh * 64, zrow);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      constexpr uint32_t idS = ptx::idesc_f16(128, kBlk, 0, 0, 0);
+      constexpr uint32_t idA = ptx::idesc_f16(128, D, 0, 0, 1);
+      const uint32_t aK = ptx::smem_u32(sK), aZ = ptx::smem_u32(sZ), aQ = ptx::smem_u32(sQ), aY = ptx::smem_u32(sY);
+      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) {
+        const uint64_t da = ptx::sw128_desc(a, 16, 1024), db = ptx::sw128_desc(b, 16, 1024);
+#pragma unroll
+        for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4)
+            ptx::mma_f16_ss(td, da + ((hf * 2 * kBox + k4 * 32) >> 4), db + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
+                            !(first && hf == 0 && k4 == 0));
+      };
+      auto accum = [&](uint32_t tacc, uint32_t ta, int pa, uint32_t b, bool first) {
+        const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk)
+          ptx::mma_f16_ts(tacc, ta + (kk >> 1) * 32 + pa * 16 + (kk & 1) * 8, db + ((kk * 2048) >> 4), idA,
+                          !(first && kk == 0));
+      };
+      bool ok = ptx::mbar_wait(c_full, 0);
+      for (int j = 0; j < nblk && ok; ++j) {
+        ok = ptx::mbar_wait(k_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
+        scores(tX, aQ, aK, true);              // S = q k~_hi^T + q k~_lo^T
+        scores(tX, aQ, aK + kPl, false);
+        scores(tY, aY, aZ, true);              // dP = dy z^T (hi hi, lo hi, hi lo)
+        scores(tY, aY + kPl, aZ, false);
+        scores(tY, aY, aZ + kPl, false);
+        ptx::mma_commit(s_full);
+        ok = ptx::mbar_wait(p_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
+        accum(tA, tY, 0, aK, j == 0);          // dq += dS k~ (hi hi, lo hi, hi lo)
+        accum(tA, tY, 1, aK, false);
+        accum(tA, tY, 0, aK + kPl, false);
+        ptx::mma_commit(k_free);
+      }
+      ptx::mma_commit(o_done);
+    }
+  } else {
+    const int qd = warp & 3, hf = warp >> 2;
+    const int r = 32 * qd + lane;
+    const int a1 = ab + r;
+    const bool row_ok = a1 < g.b1q;
+    const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
+    const long long lr = (long long)zrow * g.b1q_pad + (row_ok ? a1 : 0);
+    const float l = lse[lr], dd = ddv[lr];
+    const int climit = key_limit(g, row_ok ? a1 : g.b1q - 1);   // visible key tiles [0, climit)
+    float dsum = 0.f, dmax = 0.f;
+    bool ok = true;
+    for (int j = 0; j < nblk; ++j) {
+      const int k0 = j * kBlk;
+      ok = ok && ptx::mbar_wait(s_full, j & 1) && ptx::mbar_wait(k_full, j & 1);
+      ptx::tc_fence_after();
+      const int lim = climit - k0;
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int cb = 64 * hf + 32 * hh;
+        const float* hv = sH + cb;
+        softmax_chunk<false>(
+            tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; },
+            [&](int jj) { return dd; }, [&](int jj) { return cb + jj < lim; }, dsum, dmax);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(p_full);
+    }
+    if (dmax >= 65504.f) atomicExch(&ptx::g_device_error, ptx::kErrRange);
+    ok = ok && ptx::mbar_wait(o_done, 0);
+    ptx::tc_fence_after();
+    const float scale = g.sl2 * (1.f / kLog2e) / (kDsShift * dy_sigma(__uint_as_float(amax[bh])));
+    const long long o = ((long long)zrow * g.b1q + (row_ok ? a1 : 0)) * D + hf * (D / 2);
+#pragma unroll 1
+    for (int cc = 0; cc < D / 32; ++cc)
+      store_acc16(tA + lane_off + hf * (D / 2) + 16 * cc, scale, dq + o + 16 * cc, row_ok && ok);
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+}
+
+// ===========================================================================
+// Largest |dy| per head (as the bits of a non-negative float, which order like
+// unsigned integers).  grid (ceil(Nq*d / (256*8)), BH), block 256.
+template <typename TG>
+__global__ void __launch_bounds__(256) dy_amax(const TG* __restrict__ dy, unsigned* __restrict__ amax, Geo g) {
+  const long long n = g.Nq * g.d;
+  const TG* p = dy + (long long)blockIdx.y * n;
+  float m = 0.f;
+  for (long long i = (long long)blockIdx.x * 256 * 8 + threadIdx.x; i < n && i < (long long)(blockIdx.x + 1) * 2048;
+       i += 256)
+    m = fmaxf(m, fabsf(to_f(p[i])));
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(amax + blockIdx.y, __float_as_uint(m));
+}
+
+// One warp per query token: sigma dy as f16 hi/lo planes in block order
+// ([plane][BH*b2][b1q][d]) and sigma D = sigma dy . y, y the forward output
+// (f32, grid order).  grid (ceil(Nq/8), BH), block 256.
+template <typename TG, int D>
+__global__ void __launch_bounds__(256)
+dy_planes(const TG* __restrict__ dy, const float* __restrict__ y, const unsigned* __restrict__ amax,
+          __half* __restrict__ dyp, float* __restrict__ ddv, Geo g) {
+  constexpr int PER = D / 32;
+  const int bh = blockIdx.y;
+  const long long n = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (n >= g.Nq) return;
+  const float sig = dy_sigma(__uint_as_float(amax[bh]));
+  // grid token -> (tile a1, position a2)
+  const int hw = g.H * g.W;
+  const int t = (int)(n / hw), rem = (int)(n - (long long)t * hw);
+  const int yy = rem / g.W, xx = rem - yy * g.W;
+  const int a1 = (t * (g.H / g.th) + yy / g.th) * g.ntx + xx / g.tw;
+  const int a2 = (yy % g.th) * g.tw + xx % g.tw;
+  const long long src = ((long long)bh * g.Nq + n) * D;
+  const long long zrow = (long long)bh * g.b2 + a2;
+  const long long plane = (long long)g.BH * g.b2 * g.b1q * D;
+  __half* hi = dyp + (zrow * g.b1q + a1) * D;
+  float dot = 0.f;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int c = lane + 32 * i;
+    const float v = to_f(dy[src + c]) * sig;
+    dot = fmaf(v, y[src + c], dot);
+    const __half h = __float2half_rn(v);
+    hi[c] = h;
+    hi[plane + c] = __float2half_rn(v - __half2float(h));
+  }
+  dot = warp_sum(dot);
+  if (lane == 0) ddv[zrow * g.b1q_pad + a1] = dot;
+}
+
+}  // namespace tcb
+}  // namespace monarch

@@ -71,12 +71,13 @@ constexpr size_t row_smem() {
 
 // ===========================================================================
 // Row pass over 64-key blocks for one (head, position a2, 256 query rows).
-//   OUT:  out[token(a1,a2)] = sum_c1 L z     (inverse permutation in the store)
+//   OUT:  out[token(a1,a2)] = sum_c1 L z     (inverse permutation in the store);
+//         with LSE_OUT also lse[a1] (base 2) of the same scores
 //   !OUT: lse[a1] = log2 sum_c1 2^(s q.k~ + h)
 // TMEM, tile t at column 256 t.  OUT: S [0, 128) (q.k~_hi in [0, 64), q.k~_lo
 // in [64, 128); P over [0, 32)), O [128, 128 + D).  !OUT: S buffers [0, 128),
 // [128, 256).
-template <typename TQ, typename TO, int D, bool OUT>
+template <typename TQ, typename TO, int D, bool OUT, bool LSE_OUT = false>
 __global__ void __launch_bounds__(kThreads, 1)
 l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   constexpr int NH = D / 64;
@@ -260,6 +261,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     const int rowlim = key_limit(g, min(a1, g.b1q - 1));   // visible key tiles [0, rowlim)
     if (t < ntiles) {
       float m = -INFINITY, l = 0.f;
+      float lx = 0.f;   // LSE_OUT: the row sum of the unrounded exponentials
       bool ok = true;
       const float2 sl2 = make_float2(g.sl2, g.sl2);
       for (int j = 0; j < nkb; ++j) {
@@ -342,13 +344,17 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
             }
           }
           uint32_t pk[16];
+          float2 accx = make_float2(0.f, 0.f);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 d = add2(x[i], nm);
-            const __half2 hp = __floats2half2_rn(ptx::ex2(d.x), ptx::ex2(d.y));
+            const float2 e = make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
+            const __half2 hp = __floats2half2_rn(e.x, e.y);
             acc2 = add2(acc2, __half22float2(hp));
+            if constexpr (LSE_OUT) accx = add2(accx, e);
             pk[i] = *reinterpret_cast<const uint32_t*>(&hp);
           }
+          if constexpr (LSE_OUT) lx = fmaf(lx, corr, accx.x + accx.y);
           // P: keys 2c, 2c + 1 in column c of the first 32 columns of S
           ptx::tmem_st16(tS(t, 0) + lane_off + 16 * hf, pk);
           ptx::tmem_wait_st();
@@ -375,6 +381,14 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
         xs[hf * kTile + r] = l;
         ptx::named_bar(1 + t, kTileThreads);
         const float lt = l + xs[(hf ^ 1) * kTile + r];
+        if constexpr (LSE_OUT) {
+          // the row's base-2 log-sum-exp of the same scores, from the
+          // unrounded exponentials (the backward's P sums to 1 with it)
+          ptx::named_bar(1 + t, kTileThreads);
+          xs[hf * kTile + r] = lx;
+          ptx::named_bar(1 + t, kTileThreads);
+          if (hf == 0 && a1 < g.b1q) lse[(long long)zrow * g.b1q_pad + a1] = m + log2f(lx + xs[kTile + r]);
+        }
         ok = ok && ptx::mbar_wait(o_done + t, 0);
         ptx::tc_fence_after();
         const float inv = 1.f / lt;

@@ -22,6 +22,7 @@
 #include "kernels_rtc.cuh"
 #include "kernels_l.cuh"
 #include "kernels_bwd.cuh"
+#include "kernels_bwd_tc.cuh"
 
 using namespace monarch;
 
@@ -261,25 +262,16 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-template <typename TQ, typename TO, int D>
-int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* ws, cudaStream_t st) {
-  const Geo& g = p.g;
-  Work w;
-  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
-  w.z = reinterpret_cast<float*>(ws + p.off[1]);
-  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
-  w.h = reinterpret_cast<float*>(ws + p.off[3]);
-  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
-  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
-  w.qb = ws + p.off[6];
-  TcPlanes<TQ> planes;
+// Workspace views and tensor maps of the tensor-core forward (shared by the
+// forward and the backward's recompute).
+template <typename TQ, int D>
+int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& w, TcPlanes<TQ>& planes,
+               tc::Maps& maps, RtcMaps& rmaps) {
   planes.kt_hi = reinterpret_cast<__half*>(w.kt);
   planes.z_hi = reinterpret_cast<__half*>(w.z);
   planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
-
   const CUtensorMapDataType dq =
       TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
-  tc::Maps maps;
   int rc;
   {
     const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
@@ -307,7 +299,6 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   }
   // R-step maps: the key / value / query grids as (d, W, H, frames) with one
   // tile per box, and the q~ planes as (d, b1k, 2*BH*b2) with one key tile per box
-  RtcMaps rmaps;
   {
     cuuint32_t box4[4] = {64, (cuuint32_t)g.tw, (cuuint32_t)g.th, 1};
     cuuint64_t dk4[4] = {(cuuint64_t)D, (cuuint64_t)g.W, (cuuint64_t)g.H, (cuuint64_t)g.BH * g.Tk};
@@ -331,6 +322,25 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
                        CU_TENSOR_MAP_SWIZZLE_128B)))
       return rc;
   }
+  return MONARCH_OK;
+}
+
+template <typename TQ, typename TO, int D>
+int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* ws, cudaStream_t st) {
+  const Geo& g = p.g;
+  Work w;
+  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
+  w.z = reinterpret_cast<float*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
+  w.h = reinterpret_cast<float*>(ws + p.off[3]);
+  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
+  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  w.qb = ws + p.off[6];
+  TcPlanes<TQ> planes;
+  tc::Maps maps;
+  RtcMaps rmaps;
+  int rc;
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
 
   constexpr size_t smem_lse = tc::lse_smem<D>();
   constexpr size_t smem_out = tc::row_smem<D, true>();
@@ -466,12 +476,15 @@ int dispatch(const Plan& p, const void* q, const void* k, const void* v, void* o
 }
 
 // ---- backward (one-step forward, self-attention) -------------------------
-constexpr int kBwdRegions = 9;  // k~, z, h, lse, D, dqL, dk~, dz, dh
+constexpr int kBwdRegions = 9;  // f32 path: k~, z, h, lse, D, dqL, dk~, dz, dh
+constexpr int kBwdTcRegions = 8;  // tensor-core path, after the forward's regions: y, dy planes, D, amax, dqL, dk~, dz, dh
 
 struct BwdPlan {
   Plan fwd;   // geometry and validation of the forward it differentiates
   int grad_dtype;
+  bool tc;    // bf16 / f16 inputs: tensor-core L-step backward
   size_t off[kBwdRegions];
+  size_t toff[kBwdTcRegions];
   size_t total;
 };
 
@@ -483,15 +496,26 @@ int make_bwd_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, 
   if (grad_dtype != dtype && grad_dtype != MONARCH_F32)
     return fail(MONARCH_EINVAL, "grad_dtype %d must be MONARCH_F32 or the input dtype %d", grad_dtype, dtype);
   bp->grad_dtype = grad_dtype;
+  bp->tc = dtype != MONARCH_F32;
   const Geo& g = bp->fwd.g;
   const size_t big = (size_t)g.BH * g.b2 * g.b1k * d * 4;
   const size_t col = (size_t)g.BH * g.b2 * g.b1k_pad * 4;
   const size_t row = (size_t)g.BH * g.b2 * g.b1q_pad * 4;
-  const size_t sizes[kBwdRegions] = {big, big, col, row, row, big, big, big, col};
   size_t o = 0;
-  for (int i = 0; i < kBwdRegions; ++i) {
-    bp->off[i] = o;
-    o += align256(sizes[i]);
+  if (bp->tc) {
+    const size_t sizes[kBwdTcRegions] = {(size_t)g.BH * g.Nq * d * 4, (size_t)2 * g.BH * g.b2 * g.b1q * d * 2, row,
+                                         (size_t)g.BH * 4, big, big, big, col};
+    o = bp->fwd.total;
+    for (int i = 0; i < kBwdTcRegions; ++i) {
+      bp->toff[i] = o;
+      o += align256(sizes[i]);
+    }
+  } else {
+    const size_t sizes[kBwdRegions] = {big, big, col, row, row, big, big, big, col};
+    for (int i = 0; i < kBwdRegions; ++i) {
+      bp->off[i] = o;
+      o += align256(sizes[i]);
+    }
   }
   bp->total = o;
   return MONARCH_OK;
@@ -543,13 +567,128 @@ int run_bwd(const BwdPlan& bp, const T* q, const T* k, const T* v, const TG* dy,
   return MONARCH_OK;
 }
 
+// Tensor-core backward (bf16 / f16 inputs): the forward's R step and output
+// pass recompute k~, z, h, y and the row LSE; dy becomes scaled f16
+// hi/lo planes with D = sigma dy . y; the two tensor-core L-step kernels give
+// dk~, dz, dh and the L-step dq; the per-tile R-step backward finishes.
+template <typename TQ, typename TG, int D>
+int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const TG* dy, TG* dq, TG* dk, TG* dv,
+               char* ws, cudaStream_t st) {
+  const Plan& p = bp.fwd;
+  const Geo& g = p.g;
+  Work w;
+  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
+  w.z = reinterpret_cast<float*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
+  w.h = reinterpret_cast<float*>(ws + p.off[3]);
+  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
+  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  w.qb = ws + p.off[6];
+  float* y = reinterpret_cast<float*>(ws + bp.toff[0]);
+  __half* dyp = reinterpret_cast<__half*>(ws + bp.toff[1]);
+  float* ddv = reinterpret_cast<float*>(ws + bp.toff[2]);
+  unsigned* amax = reinterpret_cast<unsigned*>(ws + bp.toff[3]);
+  BwdWork bw;
+  bw.dd = ddv;
+  bw.dqL = reinterpret_cast<float*>(ws + bp.toff[4]);
+  bw.dkt = reinterpret_cast<float*>(ws + bp.toff[5]);
+  bw.dz = reinterpret_cast<float*>(ws + bp.toff[6]);
+  bw.dh = reinterpret_cast<float*>(ws + bp.toff[7]);
+
+  TcPlanes<TQ> planes;
+  tc::Maps maps;
+  RtcMaps rmaps;
+  int rc;
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
+  tcb::BwdMaps bmaps;
+  {
+    const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
+    cuuint32_t box3[3] = {64, 64, 1};
+    cuuint64_t dy3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, 2 * rows};
+    cuuint64_t sy3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1q * D * 2};
+    cuuint32_t box2[2] = {64, 1};
+    cuuint64_t dd2[2] = {(cuuint64_t)g.b1q_pad, rows};
+    cuuint64_t sd2[1] = {(cuuint64_t)g.b1q_pad * 4};
+    if ((rc = make_map(&bmaps.dy, dyp, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dy3, sy3, box3,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&bmaps.dd, ddv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dd2, sd2, box2,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)))
+      return rc;
+  }
+  constexpr size_t smem_out = tc::row_smem<D, true>();
+  constexpr size_t smem_r = rtc_smem<D>();
+  constexpr size_t smem_kv = tcb::kv_smem<D>();
+  constexpr size_t smem_q = tcb::q_smem<D>();
+  static_assert(smem_kv <= (size_t)tc::kMaxSmem && smem_q <= (size_t)tc::kMaxSmem, "backward shared memory");
+  const size_t rb_smem = (size_t)r_bwd_smem_floats(g.b2, g.d) * sizeof(float);
+  static bool attrs_set = false;
+  if (!attrs_set) {
+    cudaError_t e;
+    if ((e = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
+        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess ||
+        (e = allow_smem(tcb::l_bwd_kv<D>, smem_kv)) != cudaSuccess ||
+        (e = allow_smem(tcb::l_bwd_q<D>, smem_q)) != cudaSuccess ||
+        (e = allow_smem(r_bwd_simt<TQ, TG>, (size_t)r_bwd_smem_floats(kMaxB2, 128) * sizeof(float))) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncSetAttribute");
+    attrs_set = true;
+  }
+  const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
+  const int r_group = kRtcRows / ((g.b2 + 7) & ~7);
+  const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
+  launch(MONARCH_PHASE_R_STEP, st, [&] {
+    launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1);
+  });
+  // the output pass gives y and the row LSE of the same (hi + lo) scores
+  launch(MONARCH_PHASE_L_OUT, st, [&] {
+    launch_pdl(tc::l_row<__half, float, D, true, true>, grid_q, dim3(tc::kThreads), smem_out, st, y, maps, w.lse, g);
+  });
+  cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)g.BH * 4, st);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
+  launch(MONARCH_PHASE_BWD_PREP, st, [&] {
+    const long long n = g.Nq * D;
+    tcb::dy_amax<TG><<<dim3((unsigned)((n + 2047) / 2048), g.BH), 256, 0, st>>>(dy, amax, g);
+  });
+  launch(MONARCH_PHASE_BWD_PREP, st, [&] {
+    tcb::dy_planes<TG, D><<<dim3((unsigned)((g.Nq + 7) / 8), g.BH), 256, 0, st>>>(dy, y, amax, dyp, ddv, g);
+  });
+  launch(MONARCH_PHASE_BWD_DKV, st, [&] {
+    launch_pdl(tcb::l_bwd_kv<D>, dim3((g.b1k + tcb::kBlk - 1) / tcb::kBlk, g.b2, g.BH), dim3(tcb::kThreads), smem_kv,
+               st, maps, bmaps, (const float*)w.h, (const unsigned*)amax, bw.dkt, bw.dz, bw.dh, g);
+  });
+  launch(MONARCH_PHASE_BWD_DQ, st, [&] {
+    launch_pdl(tcb::l_bwd_q<D>, dim3((g.b1q + tcb::kBlk - 1) / tcb::kBlk, g.b2, g.BH), dim3(tcb::kThreads), smem_q,
+               st, maps, bmaps, (const float*)w.lse, (const float*)ddv, (const unsigned*)amax, bw.dqL, g);
+  });
+  launch(MONARCH_PHASE_BWD_R, st, [&] {
+    r_bwd_simt<TQ, TG><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
+  });
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return MONARCH_OK;
+}
+
 template <typename T>
 int dispatch_bwd_grad(const BwdPlan& bp, const void* q, const void* k, const void* v, const void* dy, void* dq,
                       void* dk, void* dv, char* ws, cudaStream_t st) {
-  if (bp.grad_dtype == MONARCH_F32)
-    return run_bwd<T, float>(bp, (const T*)q, (const T*)k, (const T*)v, (const float*)dy, (float*)dq, (float*)dk,
-                             (float*)dv, ws, st);
-  return run_bwd<T, T>(bp, (const T*)q, (const T*)k, (const T*)v, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws, st);
+  if constexpr (sizeof(T) == 2) {
+    if (bp.fwd.g.d == 128) {
+      if (bp.grad_dtype == MONARCH_F32)
+        return run_bwd_tc<T, float, 128>(bp, (const T*)q, (const T*)k, (const T*)v, (const float*)dy, (float*)dq,
+                                         (float*)dk, (float*)dv, ws, st);
+      return run_bwd_tc<T, T, 128>(bp, (const T*)q, (const T*)k, (const T*)v, (const T*)dy, (T*)dq, (T*)dk, (T*)dv,
+                                   ws, st);
+    }
+    if (bp.grad_dtype == MONARCH_F32)
+      return run_bwd_tc<T, float, 64>(bp, (const T*)q, (const T*)k, (const T*)v, (const float*)dy, (float*)dq,
+                                      (float*)dk, (float*)dv, ws, st);
+    return run_bwd_tc<T, T, 64>(bp, (const T*)q, (const T*)k, (const T*)v, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws,
+                                st);
+  } else {
+    if (bp.grad_dtype == MONARCH_F32)
+      return run_bwd<T, float>(bp, (const T*)q, (const T*)k, (const T*)v, (const float*)dy, (float*)dq, (float*)dk,
+                               (float*)dv, ws, st);
+    return run_bwd<T, T>(bp, (const T*)q, (const T*)k, (const T*)v, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws, st);
+  }
 }
 
 int dispatch_bwd(const BwdPlan& bp, const void* q, const void* k, const void* v, const void* dy, void* dq,

@@ -2,10 +2,15 @@
 frame-chunk causal mask): dq, dk, dv from the C ABI against the fp64 oracle
 backward on the same seeded inputs and cotangent.
 
-Tolerance, per gradient, per head and element: |got - ref| <= 1e-3 *
-RMS(ref) + (u/2) |ref|.  The first term is the fp32 arithmetic: dS = L (dy.z
-- D) subtracts two rounded dot products of length d whose difference is small
-where L is peaked, so the relative error of dS, not of the output, sets it.
+Tolerance, per gradient, per head and element: |got - ref| <= tol *
+RMS(ref) + (u/2) |ref|.  f32 inputs run the fp32 CUDA-core backward, tol =
+1e-3: dS = L (dy.z - D) subtracts two rounded dot products of length d whose
+difference is small where L is peaked, so the relative error of dS, not of
+the output, sets it.  bf16/f16 inputs run the tensor-core backward, tol =
+2e-2, the bar of every bf16/f16 result of this library: its own products
+carry every operand as f16 hi/lo planes, and the rest is the precision of the
+forward it recomputes (R rounded to the input type in k~ = R k and z = R v, P
+a single f16 in y = P z).
 The second is the one rounding of the stored gradient (u/2 = 2^-8 for bf16,
 2^-11 for f16, 0 for f32), which on peaked rows' entries of many times the RMS
 is larger than any fixed fraction of the RMS.  Full-size workloads compare
@@ -23,7 +28,7 @@ from structured_sparse_attention_grid_b200.workloads import (DTYPES, WORKLOADS, 
 
 pytestmark = pytest.mark.gpu
 
-TOL_GRAD = 1e-3
+TOL_GRAD = {"f32": 1e-3, "bf16": 2e-2, "f16": 2e-2}   # by input dtype
 # largest relative error of one round-to-nearest store in the gradient type,
 # 2^-p for p significand bits (8 for bf16, 11 for f16)
 HALF_ULP = {torch.float32: 0.0, torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}
@@ -51,6 +56,7 @@ def _compare(w, got, q, k, v, dy, heads=None):
     qn, kn, vn, dyn = (t.double().numpy() for t in (q, k, v, dy))
     ref = om.monarch_attention_backward(qn, kn, vn, dyn, _grid(w), heads=heads)
     half_ulp = HALF_ULP[got[0].dtype]
+    tol = TOL_GRAD[w.dtype]
     hs = heads or [(b, h) for b in range(w.B) for h in range(w.heads)]
     worst = 0.0
     for name, g, r in zip(("dq", "dk", "dv"), got, ref):
@@ -59,7 +65,7 @@ def _compare(w, got, q, k, v, dy, heads=None):
             rms = float(np.sqrt((r[b, h] ** 2).mean()))
             excess = np.abs(g[b, h] - r[b, h]) - half_ulp * np.abs(r[b, h])
             err = float(excess.max())
-            assert err <= TOL_GRAD * rms, f"{w.name} {name} head {(b, h)}: max excess {err:.3e} > {TOL_GRAD} * rms {rms:.3e}"
+            assert err <= tol * rms, f"{w.name} {name} head {(b, h)}: max excess {err:.3e} > {tol} * rms {rms:.3e}"
             worst = max(worst, err / rms)
     return worst
 
@@ -90,6 +96,10 @@ CASES = [
     ("f32", _wl("f32", 1, 6, 8, 128, 6, 8)),                # b1 = 1: one tile
     ("f32", _wl("f32", 2, 16, 16, 128, 8, 8, B=1)),         # b2 = 64, the largest tile
     ("f32", _wl("bf16", 3, 30, 52, 128, 6, 4, B=1, heads=2)),   # the 4680-token chunk grid
+    ("f32", _wl("f16", 2, 16, 16, 64, 8, 8, B=1)),          # tensor cores: b2 = 64, d = 64
+    ("f32", _wl("bf16", 2, 6, 8, 128, 1, 1)),               # tensor cores: b2 = 1
+    ("f32", _wl("bf16", 1, 6, 8, 128, 6, 8)),               # tensor cores: b1 = 1
+    ("f32", _wl("bf16", 9, 16, 16, 128, 4, 4, C=4, B=1)),   # tensor cores: several 128-tile blocks, masked
 ]
 
 
