@@ -104,12 +104,22 @@ def backward_work_model(w):
     """Algorithmic FLOPs of the backward of the one-step forward (gradient
     contractions only, the forward recompute not counted): L step dL, dq, dk~,
     dz (4 F_L); R step dR (2 F_R), dk (2 F_R), dv and dq (2 F_R).  Per kernel,
-    the dot-product work it performs (recompute included), for its roofline."""
+    the algorithmic work of what it computes (recompute included) and its
+    bound: tensor-core kernels against the bf16 tensor peak, CUDA-core ones
+    against the FP32 FMA ceiling."""
     m = work_model(w)
     FL, FR, BH = m["FL"], m["FR"], w.B * w.heads
-    return dict(flops=BH * (4 * FL + 6 * FR),
-                phases={"bwd_prep": BH * 2 * FL, "bwd_dq": BH * 3 * FL, "bwd_dkv": BH * 4 * FL,
-                        "bwd_r": BH * 5 * FR, "r_step": BH * 3 * FR})
+    if w.dtype == "f32":
+        phases = {"bwd_prep": (BH * 2 * FL, "alu"), "bwd_dq": (BH * 3 * FL, "alu"), "bwd_dkv": (BH * 4 * FL, "alu"),
+                  "bwd_r": (BH * 5 * FR, "alu"), "r_step": (BH * 3 * FR, "alu")}
+    else:
+        phases = {"bwd_dq": (BH * 3 * FL, "tensor"),        # S, dP, dq
+                  "bwd_dkv": (BH * 4 * FL, "tensor"),       # S^T, dP^T, dz, dk~
+                  "l_out": (BH * 2 * FL, "tensor"),         # recompute: S, y
+                  "r_step": (BH * 3 * FR, "tensor"),        # recompute: scores, k~, z
+                  "bwd_r": (BH * 5 * FR, "alu"),            # R-step backward (CUDA cores)
+                  "bwd_prep": (0.0, "hbm")}
+    return dict(flops=BH * (4 * FL + 6 * FR), phases=phases)
 
 
 # ---------------------------------------------------------------------------
@@ -386,15 +396,24 @@ def backward_line(m, w, qd, kd, vd, flush, stream):
     prof = m.profile_read(reset=True)
     m.profile_enable(False)
     kernels = {p: prof[p][0] / prof[p][1] for p in prof if prof[p][1] > 0}
-    dom = max(kernels, key=kernels.get)
-    achieved = bm["phases"][dom] / (kernels[dom] * 1e-3) / 1e12
+    totals = {p: prof[p][0] for p in prof if prof[p][1] > 0}
+    dom = max(totals, key=totals.get)
+    flops, bound = bm["phases"][dom]
+    achieved = flops / (totals[dom] * 1e-3) / 1e12
+    peaks = load_peaks()
+    if bound == "tensor":
+        roof = {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": peaks["source"]}
+    else:
+        roof = {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": ALU_F32_TFLOPS,
+                "unit": "TFLOP/s", "frac": achieved / ALU_F32_TFLOPS, "traffic": None,
+                "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}
     return {"workload": w.name, "iters": 1, "grad_dtype": "f32", "ms_per_call": ms,
             "value": bm["flops"] / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
             "gflop_per_call": bm["flops"] / 1e9,
-            "kernels_ms": kernels,
-            "roofline": {"bound": "alu", "kernel": dom, "achieved": achieved, "peak": ALU_F32_TFLOPS,
-                         "unit": "TFLOP/s", "frac": achieved / ALU_F32_TFLOPS, "traffic": None,
-                         "peak_source": "FP32 FMA: 148 SMs x 128 lanes x 2 x 1.965 GHz"}}
+            "kernels_ms": kernels, "launches": {p: prof[p][1] for p in prof if prof[p][1] > 0},
+            "roofline": roof}
 
 
 def dense_context(qd, kd, vd, model, flush, stream, monarch_ms):

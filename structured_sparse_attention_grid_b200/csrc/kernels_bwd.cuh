@@ -241,56 +241,123 @@ l_bwd_dkv_simt(const T* __restrict__ q, const TG* __restrict__ dy, Work w, BwdWo
 // ---------------------------------------------------------------------------
 // R-step backward for one key tile c1 of one head (all positions at once):
 // recomputes R from q and k, forms dSr, and writes dk, dv and the finished dq
-// of the tile's tokens in grid order.  Shared rows are padded to d+1 floats
-// so that the column-wise dot products hit distinct banks.
-// grid (b1k, BH), block 256, dynamic smem r_bwd_smem_floats(b2, d) floats.
-__host__ __device__ constexpr int r_bwd_smem_floats(int b2, int d) { return 5 * b2 * (d + 1) + 2 * b2 * (b2 + 1) + b2; }
+// of the tile's tokens in grid order.  Shared rows hold D + 4 floats (16-byte
+// aligned for float4 access); the position count is padded to even with zero
+// rows so that the score and G products run in 2 x 2 register blocks.
+// grid (b1k, BH), block 256, dynamic smem r_bwd_smem_bytes(b2, D).
+__host__ __device__ constexpr size_t r_bwd_smem_bytes(int b2, int d) {
+  return ((size_t)5 * ((b2 + 1) & ~1) * (d + 4) + 2 * (size_t)b2 * (b2 + 1) + ((b2 + 1) & ~1)) * 4 +
+         (size_t)b2 * 8;
+}
 
-template <typename T, typename TG>
-__global__ void __launch_bounds__(256)
+template <typename T> __device__ __forceinline__ float4 load4(const T* p);
+template <> __device__ __forceinline__ float4 load4<float>(const float* p) { return *reinterpret_cast<const float4*>(p); }
+template <> __device__ __forceinline__ float4 load4<__nv_bfloat16>(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xFFFF0000u), __uint_as_float(u.y << 16),
+                     __uint_as_float(u.y & 0xFFFF0000u));
+}
+template <> __device__ __forceinline__ float4 load4<__half>(const __half* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&u.x));
+  const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&u.y));
+  return make_float4(a.x, a.y, b.x, b.y);
+}
+template <typename T> __device__ __forceinline__ void store4(T* p, float4 v);
+template <> __device__ __forceinline__ void store4<float>(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+template <> __device__ __forceinline__ void store4<__nv_bfloat16>(__nv_bfloat16* p, float4 v) {
+  __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
+template <> __device__ __forceinline__ void store4<__half>(__half* p, float4 v) {
+  __half2 a = __floats2half2_rn(v.x, v.y), b = __floats2half2_rn(v.z, v.w);
+  *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
+__device__ __forceinline__ float dot4(float4 a, float4 b, float acc) {
+  return fmaf(a.x, b.x, fmaf(a.y, b.y, fmaf(a.z, b.z, fmaf(a.w, b.w, acc))));
+}
+__device__ __forceinline__ float4 axpy4(float a, float4 x, float4 y) {
+  return make_float4(fmaf(a, x.x, y.x), fmaf(a, x.y, y.y), fmaf(a, x.z, y.z), fmaf(a, x.w, y.w));
+}
+
+template <typename T, typename TG, int D>
+__global__ void __launch_bounds__(256, 3)
 r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v, TG* __restrict__ dq,
            TG* __restrict__ dk, TG* __restrict__ dv, BwdWork bw, Geo g) {
-  extern __shared__ float smem[];
+  extern __shared__ float4 smem4[];
+  constexpr int DP = D + 4, C4 = D / 4;
   const int c1 = blockIdx.x, bh = blockIdx.y;
-  const int d = g.d, b2 = g.b2, dp = d + 1, sp = b2 + 1;
-  float* sK = smem;
-  float* sV = sK + b2 * dp;
-  float* sQ = sV + b2 * dp;
-  float* sDK = sQ + b2 * dp;
-  float* sDZ = sDK + b2 * dp;
-  float* sR = sDZ + b2 * dp;   // [a2][c2]: scores, then R
-  float* sG = sR + b2 * sp;    // [a2][c2]: G, then dSr
-  float* sDH = sG + b2 * sp;
-  const long long hq = (long long)bh * g.Nq * d;
-  const long long hk = (long long)bh * g.Nk * d;
-  for (int i = threadIdx.x; i < b2 * d; i += blockDim.x) {
-    const int r = i / d, c = i - r * d;
-    const long long tk = token_of(g, c1, r) * d + c;
-    sK[r * dp + c] = to_f(k[hk + tk]);
-    sV[r * dp + c] = to_f(v[hk + tk]);
-    sQ[r * dp + c] = to_f(q[hq + tk]);
-    const long long o = (((long long)bh * b2 + r) * g.b1k + c1) * d + c;
-    sDK[r * dp + c] = bw.dkt[o];
-    sDZ[r * dp + c] = bw.dz[o];
+  const int b2 = g.b2, b2e = (b2 + 1) & ~1, sp = b2 + 1;
+  float* sK = reinterpret_cast<float*>(smem4);
+  float* sV = sK + b2e * DP;
+  float* sQ = sV + b2e * DP;
+  float* sDK = sQ + b2e * DP;
+  float* sDZ = sDK + b2e * DP;
+  float* sR = sDZ + b2e * DP;   // [a2][c2]: scores, then R
+  float* sG = sR + b2 * sp;     // [a2][c2]: G, then dSr
+  float* sDH = sG + b2 * sp;    // [b2e]
+  long long* sTok = reinterpret_cast<long long*>(sDH + b2e);
+  const long long hq = (long long)bh * g.Nq * D;
+  const long long hk = (long long)bh * g.Nk * D;
+  for (int r = threadIdx.x; r < b2; r += blockDim.x) {
+    sTok[r] = token_of(g, c1, r) * D;
+    sDH[r] = bw.dh[((long long)bh * b2 + r) * g.b1k_pad + c1];
   }
-  for (int r = threadIdx.x; r < b2; r += blockDim.x) sDH[r] = bw.dh[((long long)bh * b2 + r) * g.b1k_pad + c1];
+  __syncthreads();
+  for (int i = threadIdx.x; i < b2e * C4; i += blockDim.x) {
+    const int r = i / C4, c = (i - r * C4) * 4;
+    float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), vv = kk, qq = kk, dkk = kk, dzz = kk;
+    if (r < b2) {
+      const long long t = sTok[r] + c;
+      kk = load4(k + hk + t);
+      vv = load4(v + hk + t);
+      qq = load4(q + hq + t);
+      const long long o = (((long long)bh * b2 + r) * g.b1k + c1) * D + c;
+      dkk = *reinterpret_cast<const float4*>(bw.dkt + o);
+      dzz = *reinterpret_cast<const float4*>(bw.dz + o);
+    }
+    *reinterpret_cast<float4*>(sK + r * DP + c) = kk;
+    *reinterpret_cast<float4*>(sV + r * DP + c) = vv;
+    *reinterpret_cast<float4*>(sQ + r * DP + c) = qq;
+    *reinterpret_cast<float4*>(sDK + r * DP + c) = dkk;
+    *reinterpret_cast<float4*>(sDZ + r * DP + c) = dzz;
+  }
   __syncthreads();
 
-  // scores (base 2) and G = dk~ k^T + dz v^T
-  for (int i = threadIdx.x; i < b2 * b2; i += blockDim.x) {
-    const int a2 = i / b2, c2 = i - a2 * b2;
-    const float* qa = sQ + a2 * dp;
-    const float* ka = sDK + a2 * dp;
-    const float* za = sDZ + a2 * dp;
-    const float* kc = sK + c2 * dp;
-    const float* vc = sV + c2 * dp;
-    float sc = 0.f, gg = 0.f;
-    for (int c = 0; c < d; ++c) {
-      sc = fmaf(qa[c], kc[c], sc);
-      gg = fmaf(ka[c], kc[c], fmaf(za[c], vc[c], gg));
+  // scores (base 2) and G = dk~ k^T + dz v^T in 2 x 2 blocks of (a2, c2):
+  // rows {a, a + nb} and columns {c, c + nb}, so that neighbouring threads read
+  // neighbouring rows (D + 4 floats apart: distinct banks for float4 loads)
+  const int nb = b2e / 2;
+  for (int blk = threadIdx.x; blk < nb * nb; blk += blockDim.x) {
+    const int a = blk / nb, c = blk % nb;
+    float sc[2][2] = {}, gg[2][2] = {};
+#pragma unroll 4
+    for (int cc = 0; cc < D; cc += 4) {
+      float4 qa[2], ka[2], za[2], kc[2], vc[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        qa[i] = *reinterpret_cast<const float4*>(sQ + (a + i * nb) * DP + cc);
+        ka[i] = *reinterpret_cast<const float4*>(sDK + (a + i * nb) * DP + cc);
+        za[i] = *reinterpret_cast<const float4*>(sDZ + (a + i * nb) * DP + cc);
+        kc[i] = *reinterpret_cast<const float4*>(sK + (c + i * nb) * DP + cc);
+        vc[i] = *reinterpret_cast<const float4*>(sV + (c + i * nb) * DP + cc);
+      }
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          sc[i][j] = dot4(qa[i], kc[j], sc[i][j]);
+          gg[i][j] = dot4(za[i], vc[j], dot4(ka[i], kc[j], gg[i][j]));
+        }
     }
-    sR[a2 * sp + c2] = sc * g.sl2;
-    sG[a2 * sp + c2] = gg;
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+        if (a + i * nb < b2 && c + j * nb < b2) {
+          sR[(a + i * nb) * sp + c + j * nb] = sc[i][j] * g.sl2;
+          sG[(a + i * nb) * sp + c + j * nb] = gg[i][j];
+        }
   }
   __syncthreads();
 
@@ -324,26 +391,27 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 
   const float s = g.sl2 * (1.f / kLog2e);
   // dk[c2] = sum_a2 R dk~[a2] + s dSr q[a2];  dv[c2] = sum_a2 R dz[a2]
-  for (int i = threadIdx.x; i < b2 * d; i += blockDim.x) {
-    const int c2 = i / d, c = i - c2 * d;
-    float ak = 0.f, aq = 0.f, av = 0.f;
+  for (int i = threadIdx.x; i < b2 * C4; i += blockDim.x) {
+    const int c2 = i / C4, c = (i - c2 * C4) * 4;
+    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak, av = ak;
     for (int a2 = 0; a2 < b2; ++a2) {
       const float R = sR[a2 * sp + c2], ds = sG[a2 * sp + c2];
-      ak = fmaf(R, sDK[a2 * dp + c], ak);
-      aq = fmaf(ds, sQ[a2 * dp + c], aq);
-      av = fmaf(R, sDZ[a2 * dp + c], av);
+      ak = axpy4(R, *reinterpret_cast<const float4*>(sDK + a2 * DP + c), ak);
+      aq = axpy4(ds, *reinterpret_cast<const float4*>(sQ + a2 * DP + c), aq);
+      av = axpy4(R, *reinterpret_cast<const float4*>(sDZ + a2 * DP + c), av);
     }
-    const long long t = token_of(g, c1, c2) * d + c;
-    dk[hk + t] = from_f<TG>(fmaf(s, aq, ak));
-    dv[hk + t] = from_f<TG>(av);
+    const long long t = hk + sTok[c2] + c;
+    store4(dk + t, make_float4(fmaf(s, aq.x, ak.x), fmaf(s, aq.y, ak.y), fmaf(s, aq.z, ak.z), fmaf(s, aq.w, ak.w)));
+    store4(dv + t, av);
   }
   // dq[a2] = dqL[c1, a2] + s sum_c2 dSr k[c2]   (query tile c1 = key tile c1)
-  for (int i = threadIdx.x; i < b2 * d; i += blockDim.x) {
-    const int a2 = i / d, c = i - a2 * d;
-    float a = 0.f;
-    for (int c2 = 0; c2 < b2; ++c2) a = fmaf(sG[a2 * sp + c2], sK[c2 * dp + c], a);
-    const float base = bw.dqL[(((long long)bh * b2 + a2) * g.b1q + c1) * d + c];
-    dq[hq + token_of(g, c1, a2) * d + c] = from_f<TG>(fmaf(s, a, base));
+  for (int i = threadIdx.x; i < b2 * C4; i += blockDim.x) {
+    const int a2 = i / C4, c = (i - a2 * C4) * 4;
+    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c2 = 0; c2 < b2; ++c2) a = axpy4(sG[a2 * sp + c2], *reinterpret_cast<const float4*>(sK + c2 * DP + c), a);
+    const float4 base = *reinterpret_cast<const float4*>(bw.dqL + (((long long)bh * b2 + a2) * g.b1q + c1) * D + c);
+    store4(dq + hq + sTok[a2] + c,
+           make_float4(fmaf(s, a.x, base.x), fmaf(s, a.y, base.y), fmaf(s, a.z, base.z), fmaf(s, a.w, base.w)));
   }
 }
 

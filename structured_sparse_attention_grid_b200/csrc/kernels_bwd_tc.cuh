@@ -32,6 +32,7 @@
 #pragma once
 
 #include "tc_common.cuh"
+#include "kernels_bwd.cuh"
 
 namespace monarch {
 namespace tcb {
@@ -64,7 +65,7 @@ constexpr size_t kv_smem() {
   constexpr int NH = D / 64;
   return (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + (size_t)NH * 2 * kBox /* q */ +
          (size_t)2 * NH * 2 * kBox /* dy planes */ + 2 * kBlk * 4 /* lse, D */ + 2 * kBlk * 4 /* dh halves */ +
-         16 * 8;
+         16 * 8 /* 8 barriers, TMEM address */;
 }
 
 template <int D>
@@ -148,12 +149,14 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
   float* sX = sD + kBlk;                                // dh of the two column halves
   uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * kBlk);
   uint64_t* k_full = bar + 0;
-  uint64_t* q_full = bar + 1;
+  uint64_t* q_full = bar + 1;    // q, lse, D of a query block
   uint64_t* q_free = bar + 2;
   uint64_t* s_full = bar + 3;
   uint64_t* p_full = bar + 4;
   uint64_t* o_done = bar + 5;
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* y_full = bar + 6;    // dy planes of a query block
+  uint64_t* y_free = bar + 7;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a2 = blockIdx.y, bh = blockIdx.z;
@@ -171,6 +174,8 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(p_full, kSoftWarps);
     ptx::mbar_init(o_done, 1);
+    ptx::mbar_init(y_full, 1);
+    ptx::mbar_init(y_free, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -194,23 +199,29 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
             ptx::tma_load_3d(sK + off, &maps.kt, k_full, hf * 64, kb + rh * 64, p * rows + zrow);
             ptx::tma_load_3d(sZ + off, &maps.z, k_full, hf * 64, kb + rh * 64, p * rows + zrow);
           }
+      // q (with lse, D) and dy are refilled separately: the products of a
+      // block release q before dy, so the next q arrives while dz is summed
       bool ok = true;
       for (int j = 0; j < nblk && ok; ++j) {
         const int q0 = (qb0 + j) * kBlk;
         if (j > 0) ok = ptx::mbar_wait(q_free, (j - 1) & 1);
         if (!ok) break;
-        ptx::mbar_expect_tx(q_full, 3 * kPl + 2 * kBlk * 4);
+        ptx::mbar_expect_tx(q_full, kPl + 2 * kBlk * 4);
         for (int hf = 0; hf < NH; ++hf)
-          for (int rh = 0; rh < 2; ++rh) {
+          for (int rh = 0; rh < 2; ++rh)
             ptx::tma_load_3d(sQ + hf * 2 * kBox + rh * kBox, &maps.qb, q_full, hf * 64, q0 + rh * 64, zrow);
-            for (int p = 0; p < 2; ++p)
-              ptx::tma_load_3d(sY + p * kPl + hf * 2 * kBox + rh * kBox, &bmaps.dy, q_full, hf * 64, q0 + rh * 64,
-                               p * rows + zrow);
-          }
         for (int rh = 0; rh < 2; ++rh) {
           tc::tma_load_2d(sL + rh * 64, &maps.lse, q_full, q0 + rh * 64, zrow);
           tc::tma_load_2d(sD + rh * 64, &bmaps.dd, q_full, q0 + rh * 64, zrow);
         }
+        if (j > 0) ok = ptx::mbar_wait(y_free, (j - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(y_full, 2 * kPl);
+        for (int p = 0; p < 2; ++p)
+          for (int hf = 0; hf < NH; ++hf)
+            for (int rh = 0; rh < 2; ++rh)
+              ptx::tma_load_3d(sY + p * kPl + hf * 2 * kBox + rh * kBox, &bmaps.dy, y_full, hf * 64, q0 + rh * 64,
+                               p * rows + zrow);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -243,6 +254,9 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
         if (!ok) break;
         scores(tX, aK, aQ, true);              // S^T = k~_hi q^T + k~_lo q^T
         scores(tX, aK + kPl, aQ, false);
+        ok = ptx::mbar_wait(y_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
         scores(tY, aZ, aY, true);              // dP^T = z dy^T (hi hi, lo hi, hi lo)
         scores(tY, aZ + kPl, aY, false);
         scores(tY, aZ, aY + kPl, false);
@@ -250,12 +264,13 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
         ok = ptx::mbar_wait(p_full, j & 1);
         ptx::tc_fence_after();
         if (!ok) break;
-        accum(tZ, tX, 0, aY, j == 0);          // dz += P^T dy
-        accum(tZ, tX, 1, aY, false);
-        accum(tZ, tX, 0, aY + kPl, false);
         accum(tK, tY, 0, aQ, j == 0);          // dk~ += dS^T q
         accum(tK, tY, 1, aQ, false);
         ptx::mma_commit(q_free);
+        accum(tZ, tX, 0, aY, j == 0);          // dz += P^T dy
+        accum(tZ, tX, 1, aY, false);
+        accum(tZ, tX, 0, aY + kPl, false);
+        ptx::mma_commit(y_free);
       }
       ptx::mma_commit(o_done);
     }
@@ -328,12 +343,14 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
   float* sH = reinterpret_cast<float*>(sZ + 2 * kPl);   // h of the block's key tiles (bits)
   uint64_t* bar = reinterpret_cast<uint64_t*>(sH + kBlk);
   uint64_t* c_full = bar + 0;
-  uint64_t* k_full = bar + 1;
+  uint64_t* k_full = bar + 1;    // k~ planes and h of a key block
   uint64_t* k_free = bar + 2;
   uint64_t* s_full = bar + 3;
   uint64_t* p_full = bar + 4;
   uint64_t* o_done = bar + 5;
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* z_full = bar + 6;    // z planes of a key block
+  uint64_t* z_free = bar + 7;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a2 = blockIdx.y, bh = blockIdx.z;
@@ -350,6 +367,8 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
     ptx::mbar_init(s_full, 1);
     ptx::mbar_init(p_full, kSoftWarps);
     ptx::mbar_init(o_done, 1);
+    ptx::mbar_init(z_full, 1);
+    ptx::mbar_init(z_free, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -373,18 +392,26 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
             ptx::tma_load_3d(sY + p * kPl + hf * 2 * kBox + rh * kBox, &bmaps.dy, c_full, hf * 64, ab + rh * 64,
                              p * rows + zrow);
         }
+      // z is released right after the dP products, k~ (with h) after the dq
+      // products: the next z arrives during the softmax
       bool ok = true;
       for (int j = 0; j < nblk && ok; ++j) {
-        if (j > 0) ok = ptx::mbar_wait(k_free, (j - 1) & 1);
+        if (j > 0) ok = ptx::mbar_wait(z_free, (j - 1) & 1);
         if (!ok) break;
-        ptx::mbar_expect_tx(k_full, 4 * kPl + kBlk * 4);
+        ptx::mbar_expect_tx(z_full, 2 * kPl);
         for (int p = 0; p < 2; ++p)
           for (int hf = 0; hf < NH; ++hf)
-            for (int rh = 0; rh < 2; ++rh) {
-              const int off = p * kPl + hf * 2 * kBox + rh * kBox;
-              ptx::tma_load_3d(sK + off, &maps.kt, k_full, hf * 64, j * kBlk + rh * 64, p * rows + zrow);
-              ptx::tma_load_3d(sZ + off, &maps.z, k_full, hf * 64, j * kBlk + rh * 64, p * rows + zrow);
-            }
+            for (int rh = 0; rh < 2; ++rh)
+              ptx::tma_load_3d(sZ + p * kPl + hf * 2 * kBox + rh * kBox, &maps.z, z_full, hf * 64, j * kBlk + rh * 64,
+                               p * rows + zrow);
+        if (j > 0) ok = ptx::mbar_wait(k_free, (j - 1) & 1);
+        if (!ok) break;
+        ptx::mbar_expect_tx(k_full, 2 * kPl + kBlk * 4);
+        for (int p = 0; p < 2; ++p)
+          for (int hf = 0; hf < NH; ++hf)
+            for (int rh = 0; rh < 2; ++rh)
+              ptx::tma_load_3d(sK + p * kPl + hf * 2 * kBox + rh * kBox, &maps.kt, k_full, hf * 64, j * kBlk + rh * 64,
+                               p * rows + zrow);
         for (int rh = 0; rh < 2; ++rh) tc::tma_load_2d(sH + rh * 64, &maps.h, k_full, j * kBlk + rh * 64, zrow);
       }
     }
@@ -416,10 +443,14 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
         if (!ok) break;
         scores(tX, aQ, aK, true);              // S = q k~_hi^T + q k~_lo^T
         scores(tX, aQ, aK + kPl, false);
+        ok = ptx::mbar_wait(z_full, j & 1);
+        ptx::tc_fence_after();
+        if (!ok) break;
         scores(tY, aY, aZ, true);              // dP = dy z^T (hi hi, lo hi, hi lo)
         scores(tY, aY + kPl, aZ, false);
         scores(tY, aY, aZ + kPl, false);
         ptx::mma_commit(s_full);
+        ptx::mma_commit(z_free);
         ok = ptx::mbar_wait(p_full, j & 1);
         ptx::tc_fence_after();
         if (!ok) break;
@@ -475,15 +506,21 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
 
 // ===========================================================================
 // Largest |dy| per head (as the bits of a non-negative float, which order like
-// unsigned integers).  grid (ceil(Nq*d / (256*8)), BH), block 256.
+// unsigned integers).  Each thread reads 16 consecutive elements (four 16-byte
+// or 8-byte loads in flight).  grid (ceil(Nq*d / 4096), BH), block 256.
 template <typename TG>
 __global__ void __launch_bounds__(256) dy_amax(const TG* __restrict__ dy, unsigned* __restrict__ amax, Geo g) {
-  const long long n = g.Nq * g.d;
+  const long long n = g.Nq * g.d;   // a multiple of 64
   const TG* p = dy + (long long)blockIdx.y * n;
+  const long long base = ((long long)blockIdx.x * 256 + threadIdx.x) * 16;
   float m = 0.f;
-  for (long long i = (long long)blockIdx.x * 256 * 8 + threadIdx.x; i < n && i < (long long)(blockIdx.x + 1) * 2048;
-       i += 256)
-    m = fmaxf(m, fabsf(to_f(p[i])));
+  if (base < n) {
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) v[i] = load4(p + base + 4 * i);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m = fmaxf(m, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
   m = warp_max(m);
   if ((threadIdx.x & 31) == 0 && m > 0.f) atomicMax(amax + blockIdx.y, __float_as_uint(m));
 }

@@ -552,15 +552,18 @@ int run_bwd(const BwdPlan& bp, const T* q, const T* k, const T* v, const TG* dy,
   const size_t r_smem = (size_t)(3 * g.b2 * g.d + g.b2 * (g.b2 + 1)) * sizeof(float);
   cudaError_t e = allow_smem(r_step_simt<T>, r_smem);
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(r_step)");
-  const size_t rb_smem = (size_t)r_bwd_smem_floats(g.b2, g.d) * sizeof(float);
-  if ((e = allow_smem(r_bwd_simt<T, TG>, rb_smem)) != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(r_bwd)");
+  const size_t rb_smem = r_bwd_smem_bytes(g.b2, g.d);
+  if ((e = allow_smem(r_bwd_simt<T, TG, 128>, r_bwd_smem_bytes(kMaxB2, 128))) != cudaSuccess ||
+      (e = allow_smem(r_bwd_simt<T, TG, 64>, r_bwd_smem_bytes(kMaxB2, 64))) != cudaSuccess)
+    return cuda_fail(e, "cudaFuncSetAttribute(r_bwd)");
   launch(MONARCH_PHASE_R_STEP, st, [&] {
     r_step_simt<T><<<dim3(g.b1k, g.BH), 128, r_smem, st>>>(q, k, v, w, g, QT_IDENTITY, 1);
   });
   if (g.d == 128) launch_l_bwd<T, TG, 128>(g, q, dy, w, bw, st);
   else launch_l_bwd<T, TG, 64>(g, q, dy, w, bw, st);
   launch(MONARCH_PHASE_BWD_R, st, [&] {
-    r_bwd_simt<T, TG><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
+    if (g.d == 128) r_bwd_simt<T, TG, 128><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
+    else r_bwd_simt<T, TG, 64><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
   });
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
@@ -620,7 +623,7 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   constexpr size_t smem_kv = tcb::kv_smem<D>();
   constexpr size_t smem_q = tcb::q_smem<D>();
   static_assert(smem_kv <= (size_t)tc::kMaxSmem && smem_q <= (size_t)tc::kMaxSmem, "backward shared memory");
-  const size_t rb_smem = (size_t)r_bwd_smem_floats(g.b2, g.d) * sizeof(float);
+  const size_t rb_smem = r_bwd_smem_bytes(g.b2, D);
   static bool attrs_set = false;
   if (!attrs_set) {
     cudaError_t e;
@@ -628,7 +631,7 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
         (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess ||
         (e = allow_smem(tcb::l_bwd_kv<D>, smem_kv)) != cudaSuccess ||
         (e = allow_smem(tcb::l_bwd_q<D>, smem_q)) != cudaSuccess ||
-        (e = allow_smem(r_bwd_simt<TQ, TG>, (size_t)r_bwd_smem_floats(kMaxB2, 128) * sizeof(float))) != cudaSuccess)
+        (e = allow_smem(r_bwd_simt<TQ, TG, D>, r_bwd_smem_bytes(kMaxB2, D))) != cudaSuccess)
       return cuda_fail(e, "cudaFuncSetAttribute");
     attrs_set = true;
   }
@@ -646,7 +649,7 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   launch(MONARCH_PHASE_BWD_PREP, st, [&] {
     const long long n = g.Nq * D;
-    tcb::dy_amax<TG><<<dim3((unsigned)((n + 2047) / 2048), g.BH), 256, 0, st>>>(dy, amax, g);
+    tcb::dy_amax<TG><<<dim3((unsigned)((n + 4095) / 4096), g.BH), 256, 0, st>>>(dy, amax, g);
   });
   launch(MONARCH_PHASE_BWD_PREP, st, [&] {
     tcb::dy_planes<TG, D><<<dim3((unsigned)((g.Nq + 7) / 8), g.BH), 256, 0, st>>>(dy, y, amax, dyp, ddv, g);
@@ -660,7 +663,7 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
                st, maps, bmaps, (const float*)w.lse, (const float*)ddv, (const unsigned*)amax, bw.dqL, g);
   });
   launch(MONARCH_PHASE_BWD_R, st, [&] {
-    r_bwd_simt<TQ, TG><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
+    r_bwd_simt<TQ, TG, D><<<dim3(g.b1k, g.BH), 256, rb_smem, st>>>(q, k, v, dq, dk, dv, bw, g);
   });
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
