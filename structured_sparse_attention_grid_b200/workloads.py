@@ -93,6 +93,9 @@ WORKLOADS = {
         # the same sequence in the training regime: 3-frame chunks, chunk-causal
         Workload("train_32760_bf16_causal", 2, 12, 21, 30, 52, 128, 6, 4, 3, "bf16", 4, "pos_planted",
                  chunk_frames=3),
+        # the one-step regime of finetuned models (a single refinement step)
+        Workload("chunk_4680_bf16_1step", 1, 12, 3, 30, 52, 128, 6, 4, 1, "bf16", 2, "pos"),
+        Workload("full_32760_bf16_1step", 2, 12, 21, 30, 52, 128, 6, 4, 1, "bf16", 4, "pos_planted"),
         Workload("sweep_2048_f16", 1, 24, 8, 16, 16, 64, 8, 8, 2, "f16", 5, "pos_planted"),
         Workload("sweep_8192_f16", 1, 24, 8, 32, 32, 64, 8, 8, 2, "f16", 5, "pos_planted"),
         Workload("sweep_32768_f16", 1, 24, 8, 64, 64, 64, 8, 8, 2, "f16", 5, "pos_planted"),
