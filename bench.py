@@ -187,6 +187,17 @@ class ClockSampler:
                 "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value over the ranks (for a time: the slowest rank); the
+    value itself on one rank.  device: where the reduction tensor lives (the
+    rank's GPU under NCCL, None = host under gloo)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ---------------------------------------------------------------------------
 def run_ours(args, rank, world, device):
     import structured_sparse_attention_grid_b200 as m
@@ -243,10 +254,7 @@ def run_ours(args, rank, world, device):
         clocks.end()
     clocks.stop()
 
-    if world > 1:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, world, device)
 
     # Per-kernel times: the same step, with CUDA events around every launch.
     m.profile_enable(True)
@@ -313,10 +321,7 @@ def run_ours(args, rank, world, device):
     e1.record(stream)
     torch.cuda.synchronize(device)
     e2e_ms = e0.elapsed_time(e1) / e2e_n
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, device)
 
     es = q.element_size()
     rec = {

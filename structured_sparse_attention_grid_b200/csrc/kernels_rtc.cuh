@@ -64,11 +64,11 @@ constexpr size_t rtc_smem() {
   return need > 80 * 1024 ? need : 80 * 1024;
 }
 
-// grid (ceil(b1k / G), BH), block kRtcThreads.
+// grid (ceil(b1k / G), BH), block kRtcThreads; 1 <= G <= floor(128 / r8).
 template <typename TQ, int D>
 __global__ void __launch_bounds__(kRtcThreads, 2)
 r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work w, TcPlanes<TQ> out, Geo g,
-           int mode, int final_step) {
+           int mode, int final_step, int G) {
   constexpr int NH = D / 64;
   constexpr int bf16 = TcType<TQ>::kBf16;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -89,8 +89,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
-  const int r8 = (g.b2 + 7) & ~7;
-  const int G = kRtcRows / r8;
+  const int r8 = (g.b2 + 7) & ~7;   // G * r8 <= 128 (the host's choice of G)
   const int c1_0 = blockIdx.x * G;
   const int Gn = min(G, g.b1k - c1_0);
 

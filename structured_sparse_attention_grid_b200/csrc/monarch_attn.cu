@@ -262,6 +262,42 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Key tiles per R-step CTA.  At most floor(128 / r8) fit the 128 MMA rows;
+// fewer give more, shorter CTAs.  Two CTAs run per SM, so the launch takes
+// ceil(CTAs / (2 * SMs)) rounds of CTAs whose time grows with G plus a fixed
+// part (loads, the MMA and softmax chain, the epilogue).  The group size with
+// the fewest rounds x (G + kRFixed) is taken.  Measured on B200 with 6 x 4
+// tiles, a CTA takes about (G + 3.7) times the time of one tile's share.
+int r_step_group(const Geo& g, int sm_count) {
+  constexpr double kRFixed = 3.5;   // fixed part of a CTA's time, in tiles
+  const int gmax = kRtcRows / ((g.b2 + 7) & ~7);
+  int best = gmax;
+  double best_t = 1e300;
+  for (int G = gmax; G >= 1; --G) {
+    const long long ctas = (long long)((g.b1k + G - 1) / G) * g.BH;
+    const long long rounds = (ctas + 2LL * sm_count - 1) / (2LL * sm_count);
+    const double t = (double)rounds * (G + kRFixed);
+    if (t < best_t - 1e-9) {
+      best_t = t;
+      best = G;
+    }
+  }
+  return best;
+}
+
+int sm_count_of_device() {
+  static int n[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) return 148;
+  if (!n[dev]) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    n[dev] = v > 0 ? v : 1;
+  }
+  return n[dev];
+}
+
 // Workspace views and tensor maps of the tensor-core forward (shared by the
 // forward and the backward's recompute).
 template <typename TQ, int D>
@@ -368,7 +404,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   }
   const long long col_items = (long long)g.BH * g.b2 * ((g.b1k + 2 * kTile - 1) / (2 * kTile));
   const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
-  const int r_group = kRtcRows / ((g.b2 + 7) & ~7);   // key tiles per R-step CTA
+  const int r_group = r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
@@ -386,7 +422,8 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
       });
     }
     launch(MONARCH_PHASE_R_STEP, st, [&] {
-      launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, mode, final_step);
+      launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, mode, final_step,
+                 r_group);
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
@@ -636,10 +673,11 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
     attrs_set = true;
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
-  const int r_group = kRtcRows / ((g.b2 + 7) & ~7);
+  const int r_group = r_step_group(g, sm_count_of_device());
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   launch(MONARCH_PHASE_R_STEP, st, [&] {
-    launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1);
+    launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1,
+               r_group);
   });
   // the output pass gives y and the row LSE of the same (hi + lo) scores
   launch(MONARCH_PHASE_L_OUT, st, [&] {
