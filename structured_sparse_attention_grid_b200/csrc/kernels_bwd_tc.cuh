@@ -23,9 +23,14 @@
 // by 2^kDsShift before its split; fp32 accumulation throughout.
 //
 // TMEM (512 columns): X [0, 128), Y [128, 256), accumulators from 256.  A
-// 32-column chunk of X or Y that held 32 scores holds, after the softmax,
-// the hi values of those 32 entries in its first 16 columns and the lo values
-// in the last 16 (two f16 per column), the layout of an A operand in TMEM.
+// 16-column group of X or Y that held 16 scores holds, after the softmax, the
+// hi values of those 16 entries in its first 8 columns and the lo values in
+// the last 8 (two f16 per column): per 16 entries of K, the A operand of one
+// MMA for each plane.
+//
+// Warps 0-15 run the softmax: warp w owns TMEM lanes 32 (w mod 4) .. + 31 and
+// the 32 columns 32 (w / 4) .. + 31 of each block (later a quarter of d in the
+// epilogue).  Warp 16 issues the MMAs, warp 17 the TMA loads.
 // Each block's products that read P or dS are issued before the next block's
 // score products, and one thread's MMAs run in issue order, so the next
 // scores never overwrite an operand still in use.
@@ -38,7 +43,7 @@ namespace monarch {
 namespace tcb {
 
 using tc::kBox;
-constexpr int kSoftWarps = 8;                  // 4 lane quadrants x 2 column halves
+constexpr int kSoftWarps = 16;                 // 4 lane quadrants x 4 column quarters
 constexpr int kThreads = 32 * (kSoftWarps + 2);
 constexpr int kMmaWarp = kSoftWarps;
 constexpr int kLoadWarp = kSoftWarps + 1;
@@ -64,7 +69,7 @@ template <int D>
 constexpr size_t kv_smem() {
   constexpr int NH = D / 64;
   return (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + (size_t)NH * 2 * kBox /* q */ +
-         (size_t)2 * NH * 2 * kBox /* dy planes */ + 2 * kBlk * 4 /* lse, D */ + 2 * kBlk * 4 /* dh halves */ +
+         (size_t)2 * NH * 2 * kBox /* dy planes */ + 2 * kBlk * 4 /* lse, D */ + 2 * kBlk * 4 /* dh partial sums */ +
          16 * 8 /* 8 barriers, TMEM address */;
 }
 
@@ -75,43 +80,41 @@ constexpr size_t q_smem() {
          (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + kBlk * 4 /* h */ + 16 * 8;
 }
 
-// One 32-column chunk of the softmax: reads 32 scores X and 32 values Y of
+// One 16-column group of the softmax: reads 16 scores X and 16 values Y of
 // this thread's row, forms P and dS, and writes their hi/lo f16 planes over
-// the chunk (P over X when WRITE_P, dS over Y).  Column j of the chunk has
-// base-2 offset off[j] (h - lse, per column or per row) and D value dd[j];
-// keep(j) masks it.  Accumulates dS into dsum; tracks max |2^shift dS|.
+// the group (P over X when WRITE_P, dS over Y): hi in the first 8 columns, lo
+// in the last 8.  Column j has base-2 offset off(j) (h - lse, per column or
+// per row) and D value dd(j); keep(j) masks it.  Accumulates dS into dsum;
+// tracks max |2^shift dS|.
 template <bool WRITE_P, typename Off, typename Dv, typename Keep>
-__device__ __forceinline__ void softmax_chunk(uint32_t tx, uint32_t ty, float sl2, Off off, Dv dd, Keep keep,
+__device__ __forceinline__ void softmax_group(uint32_t tx, uint32_t ty, float sl2, Off off, Dv dd, Keep keep,
                                               float& dsum, float& dmax) {
-  uint32_t xr[32], yr[32];
-  ptx::tmem_ld32(tx, xr);
-  ptx::tmem_ld32(ty, yr);
+  uint32_t xr[16], yr[16];
+  ptx::tmem_ld16(tx, xr);
+  ptx::tmem_ld16(ty, yr);
   ptx::tmem_wait_ld();
+  uint32_t phi[8], plo[8], shi[8], slo[8];
 #pragma unroll
-  for (int h16 = 0; h16 < 2; ++h16) {
-    uint32_t phi[8], plo[8], shi[8], slo[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const int j = 16 * h16 + 2 * e;
-      float p0 = ptx::ex2(fmaf(__uint_as_float(xr[j]), sl2, off(j)));
-      float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
-      if (!keep(j)) p0 = 0.f;
-      if (!keep(j + 1)) p1 = 0.f;
-      const float d0 = p0 * (__uint_as_float(yr[j]) - dd(j));
-      const float d1 = p1 * (__uint_as_float(yr[j + 1]) - dd(j + 1));
-      dsum += d0 + d1;
-      const float2 ds = make_float2(d0 * kDsShift, d1 * kDsShift);
-      dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
-      tc::split2<__half>(ds, shi[e], slo[e]);
-      if (WRITE_P) tc::split2<__half>(make_float2(p0, p1), phi[e], plo[e]);
-    }
-    if (WRITE_P) {
-      ptx::tmem_st8(tx + 8 * h16, phi);
-      ptx::tmem_st8(tx + 16 + 8 * h16, plo);
-    }
-    ptx::tmem_st8(ty + 8 * h16, shi);
-    ptx::tmem_st8(ty + 16 + 8 * h16, slo);
+  for (int e = 0; e < 8; ++e) {
+    const int j = 2 * e;
+    float p0 = ptx::ex2(fmaf(__uint_as_float(xr[j]), sl2, off(j)));
+    float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
+    if (!keep(j)) p0 = 0.f;
+    if (!keep(j + 1)) p1 = 0.f;
+    const float d0 = p0 * (__uint_as_float(yr[j]) - dd(j));
+    const float d1 = p1 * (__uint_as_float(yr[j + 1]) - dd(j + 1));
+    dsum += d0 + d1;
+    const float2 ds = make_float2(d0 * kDsShift, d1 * kDsShift);
+    dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
+    tc::split2<__half>(ds, shi[e], slo[e]);
+    if (WRITE_P) tc::split2<__half>(make_float2(p0, p1), phi[e], plo[e]);
   }
+  if (WRITE_P) {
+    ptx::tmem_st8(tx, phi);
+    ptx::tmem_st8(tx + 8, plo);
+  }
+  ptx::tmem_st8(ty, shi);
+  ptx::tmem_st8(ty + 8, slo);
 }
 
 // Writes 16 accumulator columns of this thread's row, times `scale`, as f32.
@@ -146,7 +149,7 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
   uint8_t* sY = sQ + kPl;               // sigma dy [plane]
   float* sL = reinterpret_cast<float*>(sY + 2 * kPl);   // lse of the block's queries
   float* sD = sL + kBlk;                                // sigma D
-  float* sX = sD + kBlk;                                // dh of the two column halves
+  float* sX = sD + kBlk;                                // dh partial sums of the column quarters
   uint64_t* bar = reinterpret_cast<uint64_t*>(sX + 2 * kBlk);
   uint64_t* k_full = bar + 0;
   uint64_t* q_full = bar + 1;    // q, lse, D of a query block
@@ -244,8 +247,7 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
         const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          ptx::mma_f16_ts(tacc, ta + (kk >> 1) * 32 + pa * 16 + (kk & 1) * 8, db + ((kk * 2048) >> 4), idA,
-                          !(first && kk == 0));
+          ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
       };
       bool ok = ptx::mbar_wait(k_full, 0);
       for (int j = 0; j < nblk && ok; ++j) {
@@ -275,7 +277,7 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
       ptx::mma_commit(o_done);
     }
   } else {
-    const int qd = warp & 3, hf = warp >> 2;
+    const int qd = warp & 3, cq = warp >> 2;   // lane quadrant, column quarter
     const int r = 32 * qd + lane;
     const int c1 = kb + r;
     const bool row_ok = c1 < g.b1k;
@@ -291,11 +293,11 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
       const int lim = min(kBlk, g.b1q - q0);   // valid queries of the block
       const int lo = qstart - q0;              // queries below this one do not see the key tile
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int cb = 64 * hf + 32 * hh;
+      for (int g16 = 0; g16 < 2; ++g16) {
+        const int cb = 32 * cq + 16 * g16;
         const float* l = sL + cb;
         const float* dv = sD + cb;
-        softmax_chunk<true>(
+        softmax_group<true>(
             tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hb - l[jj]; },
             [&](int jj) { return dv[jj]; }, [&](int jj) { return cb + jj < lim && cb + jj >= lo; }, dsum, dmax);
       }
@@ -305,19 +307,24 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
       if (lane == 0) ptx::mbar_arrive(p_full);
     }
     if (dmax >= 65504.f) atomicExch(&ptx::g_device_error, ptx::kErrRange);
-    sX[hf * kBlk + r] = dsum;
+    // dh = the four quarters' sums: 1 -> 0 and 3 -> 2, then 2 -> 0
+    if (cq & 1) sX[(cq >> 1) * kBlk + r] = dsum;
+    ptx::named_bar(1, kSoftThreads);
+    if (!(cq & 1)) dsum += sX[(cq >> 1) * kBlk + r];
+    ptx::named_bar(1, kSoftThreads);
+    if (cq == 2) sX[r] = dsum;
     ptx::named_bar(1, kSoftThreads);
     ok = ok && ptx::mbar_wait(o_done, 0);
     ptx::tc_fence_after();
     const float inv = 1.f / dy_sigma(__uint_as_float(amax[bh]));
     const float s = g.sl2 * (1.f / kLog2e);
-    const long long o = ((long long)zrow * g.b1k + (row_ok ? c1 : 0)) * D + hf * (D / 2);
+    const long long o = ((long long)zrow * g.b1k + (row_ok ? c1 : 0)) * D + cq * (D / 4);
 #pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc) {
-      store_acc16(tZ + lane_off + hf * (D / 2) + 16 * cc, inv, dz + o + 16 * cc, row_ok && ok);
-      store_acc16(tK + lane_off + hf * (D / 2) + 16 * cc, inv * s / kDsShift, dkt + o + 16 * cc, row_ok && ok);
+    for (int cc = 0; cc < D / 64; ++cc) {
+      store_acc16(tZ + lane_off + cq * (D / 4) + 16 * cc, inv, dz + o + 16 * cc, row_ok && ok);
+      store_acc16(tK + lane_off + cq * (D / 4) + 16 * cc, inv * s / kDsShift, dkt + o + 16 * cc, row_ok && ok);
     }
-    if (hf == 0 && row_ok && ok) dh[(long long)zrow * g.b1k_pad + c1] = (dsum + sX[kBlk + r]) * inv;
+    if (cq == 0 && row_ok && ok) dh[(long long)zrow * g.b1k_pad + c1] = (dsum + sX[r]) * inv;
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -433,8 +440,7 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
         const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk)
-          ptx::mma_f16_ts(tacc, ta + (kk >> 1) * 32 + pa * 16 + (kk & 1) * 8, db + ((kk * 2048) >> 4), idA,
-                          !(first && kk == 0));
+          ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
       };
       bool ok = ptx::mbar_wait(c_full, 0);
       for (int j = 0; j < nblk && ok; ++j) {
@@ -462,7 +468,7 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
       ptx::mma_commit(o_done);
     }
   } else {
-    const int qd = warp & 3, hf = warp >> 2;
+    const int qd = warp & 3, cq = warp >> 2;   // lane quadrant, column quarter
     const int r = 32 * qd + lane;
     const int a1 = ab + r;
     const bool row_ok = a1 < g.b1q;
@@ -478,10 +484,10 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
       ptx::tc_fence_after();
       const int lim = climit - k0;
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int cb = 64 * hf + 32 * hh;
+      for (int g16 = 0; g16 < 2; ++g16) {
+        const int cb = 32 * cq + 16 * g16;
         const float* hv = sH + cb;
-        softmax_chunk<false>(
+        softmax_group<false>(
             tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; },
             [&](int jj) { return dd; }, [&](int jj) { return cb + jj < lim; }, dsum, dmax);
       }
@@ -494,10 +500,10 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
     ok = ok && ptx::mbar_wait(o_done, 0);
     ptx::tc_fence_after();
     const float scale = g.sl2 * (1.f / kLog2e) / (kDsShift * dy_sigma(__uint_as_float(amax[bh])));
-    const long long o = ((long long)zrow * g.b1q + (row_ok ? a1 : 0)) * D + hf * (D / 2);
+    const long long o = ((long long)zrow * g.b1q + (row_ok ? a1 : 0)) * D + cq * (D / 4);
 #pragma unroll 1
-    for (int cc = 0; cc < D / 32; ++cc)
-      store_acc16(tA + lane_off + hf * (D / 2) + 16 * cc, scale, dq + o + 16 * cc, row_ok && ok);
+    for (int cc = 0; cc < D / 64; ++cc)
+      store_acc16(tA + lane_off + cq * (D / 4) + 16 * cc, scale, dq + o + 16 * cc, row_ok && ok);
   }
   ptx::tc_fence_before();
   __syncthreads();

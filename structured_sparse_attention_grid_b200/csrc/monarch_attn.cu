@@ -769,6 +769,48 @@ int workspace_pool(cudaMemPool_t* out) {
   return MONARCH_OK;
 }
 
+// Copy streams of the host-buffer entry point, one pair per device, created
+// on first use (non-blocking) and kept for the life of the process.
+constexpr int kHostGroups = 8;   // most groups one host-buffer call splits its units into
+
+struct HostStreams {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev[2 * kHostGroups + 3] = {};   // per group: inputs landed, forward done; + 3
+};
+
+// One host-buffer call at a time per device: the call holds this lock until
+// its copies are done, since the events above are shared.
+std::mutex g_host_call_mu[64];
+
+int host_streams(HostStreams* hs, int* dev_out) {
+  static std::mutex mu;
+  static HostStreams per_dev[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(mu);
+  HostStreams& s = per_dev[dev];
+  if (!s.in) {
+    HostStreams n;
+    bool good = cudaStreamCreateWithFlags(&n.in, cudaStreamNonBlocking) == cudaSuccess &&
+                cudaStreamCreateWithFlags(&n.out, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto& x : n.ev) good = good && cudaEventCreateWithFlags(&x, cudaEventDisableTiming) == cudaSuccess;
+    if (!good) {
+      e = cudaGetLastError();
+      if (n.in) cudaStreamDestroy(n.in);
+      if (n.out) cudaStreamDestroy(n.out);
+      for (auto& x : n.ev)
+        if (x) cudaEventDestroy(x);
+      return cuda_fail(e, "creating the copy streams");
+    }
+    s = n;
+  }
+  *hs = s;
+  *dev_out = dev;
+  return MONARCH_OK;
+}
+
 int check_io(const void* q, const void* k, const void* v, const void* out) {
   int rc;
   if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v")) ||
@@ -935,28 +977,69 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
   int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
   if (rc) return rc;
   if (!q_host || !k_host || !v_host || !out_host) return fail(MONARCH_EINVAL, "null host pointer");
-  const size_t es = elem_size(dtype);
-  const size_t qb = (size_t)p.g.BH * p.g.Nq * d * es;
-  const size_t kb = (size_t)p.g.BH * p.g.Nk * d * es;
-  const size_t ob = (size_t)p.g.BH * p.g.Nq * d * elem_size(out_dtype);
-  const size_t oq = 0, ok = align256(qb), ov = ok + align256(kb), oo = ov + align256(kb);
-  const size_t ow = oo + align256(ob);
+  HostStreams hs;
+  int dev = 0;
+  if ((rc = host_streams(&hs, &dev))) return rc;
+  std::lock_guard<std::mutex> call_lock(g_host_call_mu[dev]);
+  // (batch, head) units are independent: split them into groups whose copies
+  // in, compute and copies out overlap (copies in on hs.in, the forward on
+  // `stream`, copies out on hs.out, ordered by events per group)
+  const long long U = p.g.BH;
+  const size_t es = elem_size(dtype), eo = elem_size(out_dtype);
+  const size_t qu = (size_t)p.g.Nq * d * es, ku = (size_t)p.g.Nk * d * es, ou = (size_t)p.g.Nq * d * eo;
+  const long long in_bytes = (long long)(U * (qu + 2 * ku));
+  int ng = (int)std::max<long long>(1, std::min<long long>({in_bytes / (4LL << 20), U, (long long)kHostGroups}));
+  const long long gs = (U + ng - 1) / ng;
+  ng = (int)((U + gs - 1) / gs);
+  Plan pg;   // one group of gs units (B = 1, heads = gs); the last group may be smaller
+  if ((rc = make_plan(1, (int)gs, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pg))) return rc;
+  const size_t oq = 0, ok = align256(U * qu), ov = ok + align256(U * ku), oo = ov + align256(U * ku);
+  const size_t ow = oo + align256(U * ou);
   char* buf = nullptr;
   cudaMemPool_t pool;
   if ((rc = workspace_pool(&pool))) return rc;
-  cudaError_t e = cudaMallocFromPoolAsync((void**)&buf, ow + p.total, pool, stream);
+  cudaError_t e = cudaMallocFromPoolAsync((void**)&buf, ow + pg.total, pool, stream);
   if (e != cudaSuccess) {
     cudaGetLastError();
-    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", ow + p.total, cudaGetErrorString(e));
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", ow + pg.total, cudaGetErrorString(e));
   }
-  if ((e = cudaMemcpyAsync(buf + oq, q_host, qb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(buf + ok, k_host, kb, cudaMemcpyHostToDevice, stream)) != cudaSuccess ||
-      (e = cudaMemcpyAsync(buf + ov, v_host, kb, cudaMemcpyHostToDevice, stream)) != cudaSuccess) {
-    rc = cuda_fail(e, "cudaMemcpyAsync(host->device)");
+  cudaEvent_t* ev = hs.ev;   // the device's events (this call holds its lock)
+  cudaEvent_t ev_alloc = ev[2 * kHostGroups], ev_in_done = ev[2 * kHostGroups + 1], ev_out_done = ev[2 * kHostGroups + 2];
+  {
+    cudaEventRecord(ev_alloc, stream);
+    cudaStreamWaitEvent(hs.in, ev_alloc, 0);
+    for (int gi = 0; gi < ng && rc == MONARCH_OK; ++gi) {
+      const long long u0 = gi * gs, n = std::min<long long>(gs, U - u0);
+      const char* qh = static_cast<const char*>(q_host);
+      const char* kh = static_cast<const char*>(k_host);
+      const char* vh = static_cast<const char*>(v_host);
+      if ((e = cudaMemcpyAsync(buf + oq + u0 * qu, qh + u0 * qu, n * qu, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(buf + ok + u0 * ku, kh + u0 * ku, n * ku, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(buf + ov + u0 * ku, vh + u0 * ku, n * ku, cudaMemcpyHostToDevice, hs.in)) != cudaSuccess)
+        rc = cuda_fail(e, "cudaMemcpyAsync(host->device)");
+      cudaEventRecord(ev[gi], hs.in);
+    }
+    for (int gi = 0; gi < ng && rc == MONARCH_OK; ++gi) {
+      const long long u0 = gi * gs, n = std::min<long long>(gs, U - u0);
+      Plan pn = pg;
+      if (n != gs && (rc = make_plan(1, (int)n, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pn)))
+        break;
+      cudaStreamWaitEvent(stream, ev[gi], 0);
+      rc = dispatch(pn, buf + oq + u0 * qu, buf + ok + u0 * ku, buf + ov + u0 * ku, buf + oo + u0 * ou, buf + ow,
+                    stream);
+      cudaEventRecord(ev[ng + gi], stream);
+      cudaStreamWaitEvent(hs.out, ev[ng + gi], 0);
+      if (rc == MONARCH_OK &&
+          (e = cudaMemcpyAsync(static_cast<char*>(out_host) + u0 * ou, buf + oo + u0 * ou, n * ou,
+                               cudaMemcpyDeviceToHost, hs.out)) != cudaSuccess)
+        rc = cuda_fail(e, "cudaMemcpyAsync(device->host)");
+    }
+    // the caller's stream waits for every copy, then frees the buffers
+    cudaEventRecord(ev_in_done, hs.in);
+    cudaStreamWaitEvent(stream, ev_in_done, 0);
+    cudaEventRecord(ev_out_done, hs.out);
+    cudaStreamWaitEvent(stream, ev_out_done, 0);
   }
-  if (rc == MONARCH_OK) rc = dispatch(p, buf + oq, buf + ok, buf + ov, buf + oo, buf + ow, stream);
-  if (rc == MONARCH_OK && (e = cudaMemcpyAsync(out_host, buf + oo, ob, cudaMemcpyDeviceToHost, stream)) != cudaSuccess)
-    rc = cuda_fail(e, "cudaMemcpyAsync(device->host)");
   cudaFreeAsync(buf, stream);
   e = cudaStreamSynchronize(stream);
   if (rc == MONARCH_OK && e != cudaSuccess) rc = cuda_fail(e, "cudaStreamSynchronize");

@@ -188,6 +188,20 @@ def test_host_buffer_entry_point(cuda_lib):
     _compare(w, out, q, k, v)
 
 
+@pytest.mark.parametrize("name", ["chunk_4680_bf16", "kvcache_4680x32760_bf16"])
+def test_host_buffer_groups_match_the_device_call(name, cuda_lib):
+    """The host entry point pipelines groups of (batch, head) units (4 and 6
+    groups here, the last one shorter for the KV cache); every row is computed
+    by the same arithmetic as in one device call over all units."""
+    w = WORKLOADS[name]
+    q, k, v = make_inputs(w)
+    out = torch.empty(q.shape, dtype=torch.float32).pin_memory()
+    m.monarch_attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), out, w.T, w.H, w.W, w.th,
+                            w.tw, w.iters)
+    dev = _run_gpu(w, q, k, v).cpu()
+    assert torch.equal(out, dev)
+
+
 def test_workspace_entry_point_matches_allocating_call(cuda_lib):
     w = WORKLOADS["chunk_4680_bf16"]
     q, k, v = (t.cuda() for t in make_inputs(w))
