@@ -241,12 +241,15 @@ l_bwd_dkv_simt(const T* __restrict__ q, const TG* __restrict__ dy, Work w, BwdWo
 // ---------------------------------------------------------------------------
 // R-step backward for one key tile c1 of one head (all positions at once):
 // recomputes R from q and k, forms dSr, and writes dk, dv and the finished dq
-// of the tile's tokens in grid order.  Shared rows hold D + 4 floats (16-byte
-// aligned for float4 access); the position count is padded to even with zero
-// rows so that the score and G products run in 2 x 2 register blocks.
+// of the tile's tokens in grid order.  Positions are padded with zero rows to
+// P4 = b2 rounded up to 4; shared rows of k, v, q, dk~, dz hold D + 4 floats
+// and rows of R and dSr P4 floats, so that every shared access is a float4.
+// The contractions run in register blocks: 2 x 2 (a2, c2) for the scores and
+// G, 4 positions x 4 channels for dk/dv and for dq.
 // grid (b1k, BH), block 256, dynamic smem r_bwd_smem_bytes(b2, D).
+__host__ __device__ constexpr int r_bwd_p4(int b2) { return (b2 + 3) & ~3; }
 __host__ __device__ constexpr size_t r_bwd_smem_bytes(int b2, int d) {
-  return ((size_t)5 * ((b2 + 1) & ~1) * (d + 4) + 2 * (size_t)b2 * (b2 + 1) + ((b2 + 1) & ~1)) * 4 +
+  return ((size_t)5 * r_bwd_p4(b2) * (d + 4) + 2 * (size_t)r_bwd_p4(b2) * r_bwd_p4(b2) + r_bwd_p4(b2)) * 4 +
          (size_t)b2 * 8;
 }
 
@@ -287,24 +290,29 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   extern __shared__ float4 smem4[];
   constexpr int DP = D + 4, C4 = D / 4;
   const int c1 = blockIdx.x, bh = blockIdx.y;
-  const int b2 = g.b2, b2e = (b2 + 1) & ~1, sp = b2 + 1;
+  const int b2 = g.b2, P4 = r_bwd_p4(b2);
   float* sK = reinterpret_cast<float*>(smem4);
-  float* sV = sK + b2e * DP;
-  float* sQ = sV + b2e * DP;
-  float* sDK = sQ + b2e * DP;
-  float* sDZ = sDK + b2e * DP;
-  float* sR = sDZ + b2e * DP;   // [a2][c2]: scores, then R
-  float* sG = sR + b2 * sp;     // [a2][c2]: G, then dSr
-  float* sDH = sG + b2 * sp;    // [b2e]
-  long long* sTok = reinterpret_cast<long long*>(sDH + b2e);
+  float* sV = sK + P4 * DP;
+  float* sQ = sV + P4 * DP;
+  float* sDK = sQ + P4 * DP;
+  float* sDZ = sDK + P4 * DP;
+  float* sR = sDZ + P4 * DP;   // [a2][c2], stride P4: scores, then R
+  float* sG = sR + P4 * P4;    // [a2][c2], stride P4: G, then dSr
+  float* sDH = sG + P4 * P4;   // [P4]
+  long long* sTok = reinterpret_cast<long long*>(sDH + P4);
   const long long hq = (long long)bh * g.Nq * D;
   const long long hk = (long long)bh * g.Nk * D;
   for (int r = threadIdx.x; r < b2; r += blockDim.x) {
     sTok[r] = token_of(g, c1, r) * D;
     sDH[r] = bw.dh[((long long)bh * b2 + r) * g.b1k_pad + c1];
   }
+  // zero the padding of R and dSr (rows and columns >= b2); the rest is written below
+  for (int i = threadIdx.x; i < P4 * P4; i += blockDim.x) {
+    const int r = i / P4, c = i - r * P4;
+    if (r >= b2 || c >= b2) sR[i] = sG[i] = 0.f;
+  }
   __syncthreads();
-  for (int i = threadIdx.x; i < b2e * C4; i += blockDim.x) {
+  for (int i = threadIdx.x; i < P4 * C4; i += blockDim.x) {
     const int r = i / C4, c = (i - r * C4) * 4;
     float4 kk = make_float4(0.f, 0.f, 0.f, 0.f), vv = kk, qq = kk, dkk = kk, dzz = kk;
     if (r < b2) {
@@ -327,7 +335,7 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   // scores (base 2) and G = dk~ k^T + dz v^T in 2 x 2 blocks of (a2, c2):
   // rows {a, a + nb} and columns {c, c + nb}, so that neighbouring threads read
   // neighbouring rows (D + 4 floats apart: distinct banks for float4 loads)
-  const int nb = b2e / 2;
+  const int nb = P4 / 2;
   for (int blk = threadIdx.x; blk < nb * nb; blk += blockDim.x) {
     const int a = blk / nb, c = blk % nb;
     float sc[2][2] = {}, gg[2][2] = {};
@@ -355,8 +363,8 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
 #pragma unroll
       for (int j = 0; j < 2; ++j)
         if (a + i * nb < b2 && c + j * nb < b2) {
-          sR[(a + i * nb) * sp + c + j * nb] = sc[i][j] * g.sl2;
-          sG[(a + i * nb) * sp + c + j * nb] = gg[i][j];
+          sR[(a + i * nb) * P4 + c + j * nb] = sc[i][j] * g.sl2;
+          sG[(a + i * nb) * P4 + c + j * nb] = gg[i][j];
         }
   }
   __syncthreads();
@@ -366,8 +374,8 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   constexpr float kLn2 = 0.6931471805599453f;
   for (int a2 = warp; a2 < b2; a2 += blockDim.x >> 5) {
-    float* xr = sR + a2 * sp;
-    float* gr = sG + a2 * sp;
+    float* xr = sR + a2 * P4;
+    float* gr = sG + a2 * P4;
     float m = -INFINITY;
     for (int c2 = lane; c2 < b2; c2 += 32) m = fmaxf(m, xr[c2]);
     m = warp_max(m);
@@ -390,28 +398,64 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   __syncthreads();
 
   const float s = g.sl2 * (1.f / kLog2e);
+  const int n4 = P4 / 4;
   // dk[c2] = sum_a2 R dk~[a2] + s dSr q[a2];  dv[c2] = sum_a2 R dz[a2]
-  for (int i = threadIdx.x; i < b2 * C4; i += blockDim.x) {
-    const int c2 = i / C4, c = (i - c2 * C4) * 4;
-    float4 ak = make_float4(0.f, 0.f, 0.f, 0.f), aq = ak, av = ak;
+  // (4 positions c2 x 4 channels per thread)
+  for (int i = threadIdx.x; i < n4 * C4; i += blockDim.x) {
+    const int cg = i / C4, c = (i - cg * C4) * 4, c2b = 4 * cg;
+    float4 ak[4], av[4];   // dk and dv of positions c2b .. c2b + 3
+#pragma unroll
+    for (int j = 0; j < 4; ++j) ak[j] = av[j] = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int a2 = 0; a2 < b2; ++a2) {
-      const float R = sR[a2 * sp + c2], ds = sG[a2 * sp + c2];
-      ak = axpy4(R, *reinterpret_cast<const float4*>(sDK + a2 * DP + c), ak);
-      aq = axpy4(ds, *reinterpret_cast<const float4*>(sQ + a2 * DP + c), aq);
-      av = axpy4(R, *reinterpret_cast<const float4*>(sDZ + a2 * DP + c), av);
+      const float4 r4 = *reinterpret_cast<const float4*>(sR + a2 * P4 + c2b);
+      const float4 d4 = *reinterpret_cast<const float4*>(sG + a2 * P4 + c2b);
+      const float4 k4 = *reinterpret_cast<const float4*>(sDK + a2 * DP + c);
+      const float4 q4 = *reinterpret_cast<const float4*>(sQ + a2 * DP + c);
+      const float4 z4 = *reinterpret_cast<const float4*>(sDZ + a2 * DP + c);
+      const float rr[4] = {r4.x, r4.y, r4.z, r4.w}, dd[4] = {s * d4.x, s * d4.y, s * d4.z, s * d4.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        ak[j] = axpy4(dd[j], q4, axpy4(rr[j], k4, ak[j]));
+        av[j] = axpy4(rr[j], z4, av[j]);
+      }
     }
-    const long long t = hk + sTok[c2] + c;
-    store4(dk + t, make_float4(fmaf(s, aq.x, ak.x), fmaf(s, aq.y, ak.y), fmaf(s, aq.z, ak.z), fmaf(s, aq.w, ak.w)));
-    store4(dv + t, av);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c2 = c2b + j;
+      if (c2 >= b2) break;
+      const long long t = hk + sTok[c2] + c;
+      store4(dk + t, ak[j]);
+      store4(dv + t, av[j]);
+    }
   }
-  // dq[a2] = dqL[c1, a2] + s sum_c2 dSr k[c2]   (query tile c1 = key tile c1)
-  for (int i = threadIdx.x; i < b2 * C4; i += blockDim.x) {
-    const int a2 = i / C4, c = (i - a2 * C4) * 4;
-    float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c2 = 0; c2 < b2; ++c2) a = axpy4(sG[a2 * sp + c2], *reinterpret_cast<const float4*>(sK + c2 * DP + c), a);
-    const float4 base = *reinterpret_cast<const float4*>(bw.dqL + (((long long)bh * b2 + a2) * g.b1q + c1) * D + c);
-    store4(dq + hq + sTok[a2] + c,
-           make_float4(fmaf(s, a.x, base.x), fmaf(s, a.y, base.y), fmaf(s, a.z, base.z), fmaf(s, a.w, base.w)));
+  // dq[a2] = dqL[c1, a2] + s sum_c2 dSr k[c2]   (query tile c1 = key tile c1;
+  // 4 positions a2 x 4 channels per thread; padded c2 rows are zero)
+  for (int i = threadIdx.x; i < n4 * C4; i += blockDim.x) {
+    const int ag = i / C4, c = (i - ag * C4) * 4, a2b = 4 * ag;
+    float4 acc[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c2 = 0; c2 < P4; c2 += 4) {
+      float4 kr[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) kr[u] = *reinterpret_cast<const float4*>(sK + (c2 + u) * DP + c);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float4 d4 = *reinterpret_cast<const float4*>(sG + (a2b + j) * P4 + c2);
+        acc[j] = axpy4(d4.x, kr[0], acc[j]);
+        acc[j] = axpy4(d4.y, kr[1], acc[j]);
+        acc[j] = axpy4(d4.z, kr[2], acc[j]);
+        acc[j] = axpy4(d4.w, kr[3], acc[j]);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int a2 = a2b + j;
+      if (a2 >= b2) break;
+      const float4 base = *reinterpret_cast<const float4*>(bw.dqL + (((long long)bh * b2 + a2) * g.b1q + c1) * D + c);
+      store4(dq + hq + sTok[a2] + c, make_float4(fmaf(s, acc[j].x, base.x), fmaf(s, acc[j].y, base.y),
+                                                 fmaf(s, acc[j].z, base.z), fmaf(s, acc[j].w, base.w)));
+    }
   }
 }
 
