@@ -70,7 +70,7 @@ constexpr size_t kv_smem() {
   constexpr int NH = D / 64;
   return (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + (size_t)NH * 2 * kBox /* q */ +
          (size_t)2 * NH * 2 * kBox /* dy planes */ + 2 * kBlk * 4 /* lse, D */ + 2 * kBlk * 4 /* dh partial sums */ +
-         16 * 8 /* 8 barriers, TMEM address */;
+         16 * 8 /* 9 barriers, TMEM address */;
 }
 
 template <int D>
@@ -80,20 +80,22 @@ constexpr size_t q_smem() {
          (size_t)2 * (2 * NH * 2 * kBox) /* k~, z planes */ + kBlk * 4 /* h */ + 16 * 8;
 }
 
-// One 16-column group of the softmax: reads 16 scores X and 16 values Y of
-// this thread's row, forms P and dS, and writes their hi/lo f16 planes over
-// the group (P over X when WRITE_P, dS over Y): hi in the first 8 columns, lo
-// in the last 8.  Column j has base-2 offset off(j) (h - lse, per column or
-// per row) and D value dd(j); keep(j) masks it.  Accumulates dS into dsum;
-// tracks max |2^shift dS|.
-template <bool WRITE_P, typename Off, typename Dv, typename Keep>
-__device__ __forceinline__ void softmax_group(uint32_t tx, uint32_t ty, float sl2, Off off, Dv dd, Keep keep,
-                                              float& dsum, float& dmax) {
-  uint32_t xr[16], yr[16];
+// The softmax of one 16-column group, in two phases so that the first runs
+// while the dP products are still being computed:
+//   softmax_p:  reads 16 scores X of this thread's row, forms P = 2^(x sl2 +
+//               off(j)) (0 where keep(j) is false) and writes its f16 hi/lo
+//               planes over the group (hi in the first 8 columns, lo in the
+//               last 8);
+//   softmax_ds: reads P back (hi + lo, about 22 bits) and 16 values Y, forms
+//               dS = P (y - dd(j)) and writes the hi/lo planes of 2^shift dS
+//               over the group of Y.  Accumulates dS into dsum; tracks
+//               max |2^shift dS|.
+template <typename Off, typename Keep>
+__device__ __forceinline__ void softmax_p(uint32_t tx, float sl2, Off off, Keep keep) {
+  uint32_t xr[16];
   ptx::tmem_ld16(tx, xr);
-  ptx::tmem_ld16(ty, yr);
   ptx::tmem_wait_ld();
-  uint32_t phi[8], plo[8], shi[8], slo[8];
+  uint32_t phi[8], plo[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const int j = 2 * e;
@@ -101,17 +103,57 @@ __device__ __forceinline__ void softmax_group(uint32_t tx, uint32_t ty, float sl
     float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
     if (!keep(j)) p0 = 0.f;
     if (!keep(j + 1)) p1 = 0.f;
-    const float d0 = p0 * (__uint_as_float(yr[j]) - dd(j));
-    const float d1 = p1 * (__uint_as_float(yr[j + 1]) - dd(j + 1));
+    tc::split2<__half>(make_float2(p0, p1), phi[e], plo[e]);
+  }
+  ptx::tmem_st8(tx, phi);
+  ptx::tmem_st8(tx + 8, plo);
+}
+
+template <typename Dv>
+__device__ __forceinline__ void softmax_ds(uint32_t tx, uint32_t ty, Dv dd, float& dsum, float& dmax) {
+  uint32_t pr[16], yr[16];
+  ptx::tmem_ld16(tx, pr);
+  ptx::tmem_ld16(ty, yr);
+  ptx::tmem_wait_ld();
+  uint32_t shi[8], slo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int j = 2 * e;
+    const float2 ph = __half22float2(*reinterpret_cast<const __half2*>(&pr[e]));
+    const float2 pl = __half22float2(*reinterpret_cast<const __half2*>(&pr[8 + e]));
+    const float d0 = (ph.x + pl.x) * (__uint_as_float(yr[j]) - dd(j));
+    const float d1 = (ph.y + pl.y) * (__uint_as_float(yr[j + 1]) - dd(j + 1));
     dsum += d0 + d1;
     const float2 ds = make_float2(d0 * kDsShift, d1 * kDsShift);
     dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
     tc::split2<__half>(ds, shi[e], slo[e]);
-    if (WRITE_P) tc::split2<__half>(make_float2(p0, p1), phi[e], plo[e]);
   }
-  if (WRITE_P) {
-    ptx::tmem_st8(tx, phi);
-    ptx::tmem_st8(tx + 8, plo);
+  ptx::tmem_st8(ty, shi);
+  ptx::tmem_st8(ty + 8, slo);
+}
+
+// One-phase variant for the dq kernel, where only dS is an MMA operand: reads
+// 16 scores X and 16 values Y, writes the hi/lo planes of 2^shift dS over the
+// group of Y.
+template <typename Off, typename Keep>
+__device__ __forceinline__ void softmax_ds_only(uint32_t tx, uint32_t ty, float sl2, Off off, float dd, Keep keep,
+                                                float& dmax) {
+  uint32_t xr[16], yr[16];
+  ptx::tmem_ld16(tx, xr);
+  ptx::tmem_ld16(ty, yr);
+  ptx::tmem_wait_ld();
+  uint32_t shi[8], slo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int j = 2 * e;
+    float p0 = ptx::ex2(fmaf(__uint_as_float(xr[j]), sl2, off(j)));
+    float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
+    if (!keep(j)) p0 = 0.f;
+    if (!keep(j + 1)) p1 = 0.f;
+    const float2 ds = make_float2(p0 * (__uint_as_float(yr[j]) - dd) * kDsShift,
+                                  p1 * (__uint_as_float(yr[j + 1]) - dd) * kDsShift);
+    dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
+    tc::split2<__half>(ds, shi[e], slo[e]);
   }
   ptx::tmem_st8(ty, shi);
   ptx::tmem_st8(ty + 8, slo);
@@ -154,12 +196,13 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
   uint64_t* k_full = bar + 0;
   uint64_t* q_full = bar + 1;    // q, lse, D of a query block
   uint64_t* q_free = bar + 2;
-  uint64_t* s_full = bar + 3;
-  uint64_t* p_full = bar + 4;
+  uint64_t* s_full = bar + 3;    // X = S^T complete
+  uint64_t* p_full = bar + 4;    // the softmax wrote P^T and dS^T
   uint64_t* o_done = bar + 5;
   uint64_t* y_full = bar + 6;    // dy planes of a query block
   uint64_t* y_free = bar + 7;
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
+  uint64_t* d_full = bar + 8;    // Y = dP^T complete
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 9);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a2 = blockIdx.y, bh = blockIdx.z;
@@ -179,6 +222,7 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
     ptx::mbar_init(o_done, 1);
     ptx::mbar_init(y_full, 1);
     ptx::mbar_init(y_free, 1);
+    ptx::mbar_init(d_full, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -256,13 +300,14 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
         if (!ok) break;
         scores(tX, aK, aQ, true);              // S^T = k~_hi q^T + k~_lo q^T
         scores(tX, aK + kPl, aQ, false);
+        ptx::mma_commit(s_full);
         ok = ptx::mbar_wait(y_full, j & 1);
         ptx::tc_fence_after();
         if (!ok) break;
         scores(tY, aZ, aY, true);              // dP^T = z dy^T (hi hi, lo hi, hi lo)
         scores(tY, aZ + kPl, aY, false);
         scores(tY, aZ, aY + kPl, false);
-        ptx::mma_commit(s_full);
+        ptx::mma_commit(d_full);
         ok = ptx::mbar_wait(p_full, j & 1);
         ptx::tc_fence_after();
         if (!ok) break;
@@ -293,13 +338,20 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
       const int lim = min(kBlk, g.b1q - q0);   // valid queries of the block
       const int lo = qstart - q0;              // queries below this one do not see the key tile
 #pragma unroll
-      for (int g16 = 0; g16 < 2; ++g16) {
+      for (int g16 = 0; g16 < 2; ++g16) {      // P^T while dP^T is computed
         const int cb = 32 * cq + 16 * g16;
         const float* l = sL + cb;
+        softmax_p(tX + lane_off + cb, g.sl2, [&](int jj) { return hb - l[jj]; },
+                  [&](int jj) { return cb + jj < lim && cb + jj >= lo; });
+      }
+      ptx::tmem_wait_st();   // P is read back below
+      ok = ok && ptx::mbar_wait(d_full, j & 1);
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int g16 = 0; g16 < 2; ++g16) {
+        const int cb = 32 * cq + 16 * g16;
         const float* dv = sD + cb;
-        softmax_group<true>(
-            tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hb - l[jj]; },
-            [&](int jj) { return dv[jj]; }, [&](int jj) { return cb + jj < lim && cb + jj >= lo; }, dsum, dmax);
+        softmax_ds(tX + lane_off + cb, tY + lane_off + cb, [&](int jj) { return dv[jj]; }, dsum, dmax);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
@@ -352,12 +404,13 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
   uint64_t* c_full = bar + 0;
   uint64_t* k_full = bar + 1;    // k~ planes and h of a key block
   uint64_t* k_free = bar + 2;
-  uint64_t* s_full = bar + 3;
-  uint64_t* p_full = bar + 4;
+  uint64_t* s_full = bar + 3;    // X = S complete
+  uint64_t* p_full = bar + 4;    // the softmax wrote dS
   uint64_t* o_done = bar + 5;
   uint64_t* z_full = bar + 6;    // z planes of a key block
   uint64_t* z_free = bar + 7;
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
+  uint64_t* d_full = bar + 8;    // Y = dP complete
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 9);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int a2 = blockIdx.y, bh = blockIdx.z;
@@ -376,6 +429,7 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
     ptx::mbar_init(o_done, 1);
     ptx::mbar_init(z_full, 1);
     ptx::mbar_init(z_free, 1);
+    ptx::mbar_init(d_full, 1);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -449,13 +503,14 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
         if (!ok) break;
         scores(tX, aQ, aK, true);              // S = q k~_hi^T + q k~_lo^T
         scores(tX, aQ, aK + kPl, false);
+        ptx::mma_commit(s_full);
         ok = ptx::mbar_wait(z_full, j & 1);
         ptx::tc_fence_after();
         if (!ok) break;
         scores(tY, aY, aZ, true);              // dP = dy z^T (hi hi, lo hi, hi lo)
         scores(tY, aY + kPl, aZ, false);
         scores(tY, aY, aZ + kPl, false);
-        ptx::mma_commit(s_full);
+        ptx::mma_commit(d_full);
         ptx::mma_commit(z_free);
         ok = ptx::mbar_wait(p_full, j & 1);
         ptx::tc_fence_after();
@@ -476,20 +531,21 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
     const long long lr = (long long)zrow * g.b1q_pad + (row_ok ? a1 : 0);
     const float l = lse[lr], dd = ddv[lr];
     const int climit = key_limit(g, row_ok ? a1 : g.b1q - 1);   // visible key tiles [0, climit)
-    float dsum = 0.f, dmax = 0.f;
+    float dmax = 0.f;
     bool ok = true;
     for (int j = 0; j < nblk; ++j) {
       const int k0 = j * kBlk;
       ok = ok && ptx::mbar_wait(s_full, j & 1) && ptx::mbar_wait(k_full, j & 1);
       ptx::tc_fence_after();
       const int lim = climit - k0;
+      ok = ok && ptx::mbar_wait(d_full, j & 1);
+      ptx::tc_fence_after();
 #pragma unroll
       for (int g16 = 0; g16 < 2; ++g16) {
         const int cb = 32 * cq + 16 * g16;
         const float* hv = sH + cb;
-        softmax_group<false>(
-            tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; },
-            [&](int jj) { return dd; }, [&](int jj) { return cb + jj < lim; }, dsum, dmax);
+        softmax_ds_only(tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; }, dd,
+                        [&](int jj) { return cb + jj < lim; }, dmax);
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
