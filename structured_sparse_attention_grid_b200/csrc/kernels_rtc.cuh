@@ -1,7 +1,9 @@
 // R step on the tensor cores for bf16 / f16 inputs.
 //
-// A CTA takes a group of G = floor(128 / r8) consecutive key tiles of one head
-// (r8 = b2 rounded up to 8) and stacks their rows: row r = g r8 + a2 holds
+// A CTA takes a group of G <= floor(128 / r8) consecutive key tiles of one head
+// (r8 = b2 rounded up to 8) and stacks their rows at a stride rs (32 when at
+// most four tiles of at most 32 positions are stacked, else r8): row
+// r = g rs + a2 holds
 // position a2 of key tile c1_0 + g.  With A = the stacked q~ rows (hi and lo
 // planes, or the exact query rows) and B = the stacked key rows, one
 // 128 x 128 score block
@@ -90,6 +92,10 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
   const int r8 = (g.b2 + 7) & ~7;   // G * r8 <= 128 (the host's choice of G)
+  // rows per stacked tile: 32 when four tiles of at most 32 positions fit, so
+  // that each row warp holds one tile and reads one 32-column chunk of S;
+  // else b2 rounded up to 8
+  const int rs = (g.b2 <= 32 && G * 32 <= kRtcRows) ? 32 : r8;
   const int c1_0 = blockIdx.x * G;
   const int Gn = min(G, g.b1k - c1_0);
 
@@ -112,7 +118,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   // K and V rows there meet zero R entries, and 0 * NaN would not be zero.
   for (int i = tid; i < kRtcRows * NH * 8; i += kRtcThreads) {
     const int row = i / (NH * 8), rem = i - row * (NH * 8), hf = rem >> 3, ch = rem & 7;
-    const int gg = row / r8, a = row - gg * r8;
+    const int gg = row / rs, a = row - gg * rs;
     if (gg >= Gn || a >= g.b2) {
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
       const uint32_t o = hf * kRBox + row * 128 + ch * 16;
@@ -155,7 +161,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         const int c1 = c1_0 + gg;
         int t, y0, x0;
         tile_coords(c1, t, y0, x0);
-        const uint32_t row0 = (uint32_t)(gg * r8) * 128;
+        const uint32_t row0 = (uint32_t)(gg * rs) * 128;
         for (int hf = 0; hf < NH; ++hf)
           ptx::tma_load_4d(sK + hf * kRBox + row0, &maps.k, bar_ld, hf * 64, x0, y0, bh * g.Tk + t);
         if (mode == QT_BUFFER) {
@@ -177,7 +183,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
           const int c1 = c1_0 + gg;
           if (!exact_q(c1)) continue;
           for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(&maps.qb, sA + hf * kRBox + (uint32_t)(gg * r8) * 128, hf * 64, c1 - g.off,
+            ptx::tma_store_3d(&maps.qb, sA + hf * kRBox + (uint32_t)(gg * rs) * 128, hf * 64, c1 - g.off,
                               bh * g.b2);
         }
         ptx::bulk_commit();
@@ -212,7 +218,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
             int t, y0, x0;
             tile_coords(c1_0 + gg, t, y0, x0);
             for (int hf = 0; hf < NH; ++hf)
-              ptx::tma_load_4d(sA + hf * kRBox + (uint32_t)(gg * r8) * 128, &maps.v, bar_v, hf * 64, x0, y0,
+              ptx::tma_load_4d(sA + hf * kRBox + (uint32_t)(gg * rs) * 128, &maps.v, bar_v, hf * 64, x0, y0,
                                bh * g.Tk + t);
           }
         }
@@ -243,7 +249,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   } else {
     // ------------------------------------------------------------- row warps
     const int r = tid;                          // stacked row = TMEM lane
-    const int gg = r / r8, a2 = r - gg * r8;
+    const int gg = r / rs, a2 = r - gg * rs;
     const int c1 = c1_0 + gg;
     const bool valid = gg < Gn && a2 < g.b2;
     const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
@@ -312,7 +318,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         for (int t = 0; t < Gn; ++t) {
           if (!exact_q(c1_0 + t)) continue;
           for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * r8) * 128, hf * 64,
+            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * rs) * 128, hf * 64,
                               c1_0 + t - g.off, bh * g.b2);
         }
         ptx::bulk_commit();
@@ -330,9 +336,9 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     // are read from TMEM once and kept in registers.
     ok = ptx::mbar_wait(bar_s, 0) && ok;
     ptx::tc_fence_after();
-    const int cb = gg * r8;
-    const int wg0 = (32 * warp) / r8, wg1 = min((32 * warp + 31) / r8, G - 1);
-    const int ch_lo = (wg0 * r8) >> 5, ch_hi = min((wg1 * r8 + g.b2 - 1) >> 5, 3);
+    const int cb = gg * rs;
+    const int wg0 = (32 * warp) / rs, wg1 = min((32 * warp + 31) / rs, G - 1);
+    const int ch_lo = (wg0 * rs) >> 5, ch_hi = min((wg1 * rs + g.b2 - 1) >> 5, 3);
     auto in_tile = [&](int c) { return (unsigned)(c - cb) < (unsigned)g.b2; };
     uint32_t sv[3][32];
 #pragma unroll
@@ -342,21 +348,25 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     // Branch-free: columns outside this row's tile become -inf (p = 0).  The
     // entropy uses sum p s (raw scores, finite everywhere) so that masked
     // terms are exactly zero; four partial sums shorten the dependency chains.
+    // (chunks past ch_hi are skipped: ch_hi - ch_lo is the same for the whole warp)
     float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-    for (int j = 0; j < 3; ++j)
+    for (int j = 0; j < 3; ++j) {
+      if (ch_lo + j > ch_hi) break;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const bool in = ch_lo + j <= ch_hi && in_tile(32 * (ch_lo + j) + i);
+        const bool in = in_tile(32 * (ch_lo + j) + i);
         const float x = in ? __uint_as_float(sv[j][i]) : -INFINITY;
         sv[j][i] = __float_as_uint(x);
         mq[i & 3] = fmaxf(mq[i & 3], x);
       }
+    }
     const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
     const float ms = (m == -INFINITY) ? 0.f : m * g.sl2;   // base-2 units; a row with no column stays 0
     float lq[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int j = 0; j < 3; ++j)
+    for (int j = 0; j < 3; ++j) {
+      if (ch_lo + j > ch_hi) break;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
         const float x = __uint_as_float(sv[j][i]);
@@ -365,6 +375,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         pq[i & 3] = (p > 0.f) ? fmaf(p, x, pq[i & 3]) : pq[i & 3];
         sv[j][i] = __float_as_uint(p);
       }
+    }
     const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
     // sum p (x s2 - ms) with x the raw score
     const float xe = g.sl2 * ((pq[0] + pq[1]) + (pq[2] + pq[3])) - ms * l;
@@ -427,7 +438,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
       for (int t = 0; t < Gn; ++t)
         for (int p = 0; p < 2; ++p)
           for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(map, (p ? slo : shi) + hf * kRBox + (uint32_t)(t * r8) * 128, hf * 64, c1_0 + t,
+            ptx::tma_store_3d(map, (p ? slo : shi) + hf * kRBox + (uint32_t)(t * rs) * 128, hf * 64, c1_0 + t,
                               (p * g.BH + bh) * g.b2);
       ptx::bulk_commit();
     };
