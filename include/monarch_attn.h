@@ -78,7 +78,7 @@ int monarch_attn_fwd(const void* q, const void* k, const void* v, void* out,
                      int dtype, int out_dtype, cudaStream_t stream);
 
 /* monarch_attn_fwd with the frame-chunk causal mask used when training over
- * the whole sequence (DEFINITION.md D9; MonarchRT explainers, gist.science §1
+ * the whole sequence (MonarchRT explainers, gist.science §1
  * "auto-regressive generation"): frames form chunks of chunk_frames from
  * frame 0, and a query of chunk i attends only to keys of chunks <= i.  In
  * the Monarch form this restricts the support of the factor L: the R step
