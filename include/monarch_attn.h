@@ -154,6 +154,13 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
                           int tile_h, int tile_w, int iters, long kv_len,
                           int dtype, int out_dtype, cudaStream_t stream);
 
+/* monarch_attn_fwd_host with the frame-chunk causal mask of
+ * monarch_attn_fwd_ex (chunk_frames as there). */
+int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, int B, int heads, int T, int H, int W, int d,
+                             int tile_h, int tile_w, int iters, long kv_len, int chunk_frames,
+                             int dtype, int out_dtype, cudaStream_t stream);
+
 /* Allocation-free forward (no counterpart in the paper: an interface for
  * callers that cannot allocate device memory while they run, such as a
  * real-time generation loop that must never stall or fail on an allocation,

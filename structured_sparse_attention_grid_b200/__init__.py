@@ -32,6 +32,8 @@ _SIGS = {
                                  + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_fwd_host": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                               + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
+    "monarch_attn_fwd_host_ex": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
+                                 + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_workspace_layout": (ctypes.c_size_t, [ctypes.c_int] * 9
                                       + [ctypes.c_long, ctypes.c_int, ctypes.POINTER(ctypes.c_size_t)]),
     "monarch_attn_launch_count": (ctypes.c_ulonglong, []),
@@ -180,14 +182,20 @@ def monarch_attn_fwd_noalloc(q, k, v, out, T, H, W, tile_h, tile_w, iters, strea
     return out
 
 
-def monarch_attn_fwd_host(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None):
+def monarch_attn_fwd_host(q, k, v, out, T, H, W, tile_h, tile_w, iters, stream=None, chunk_frames=0):
     """End-to-end call on HOST tensors (pinned for asynchronous copies): the
-    library copies in, computes, copies out and synchronises the stream."""
+    library copies in, computes, copies out and synchronises the stream.
+    ``chunk_frames`` > 0 applies the frame-chunk causal mask."""
     lib = load_library()
     _check_tensors(q, k, v, out)
     args = _shape_args(q, k, T, H, W, tile_h, tile_w, iters)
-    _check(lib.monarch_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                     *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
+    if chunk_frames:
+        _check(lib.monarch_attn_fwd_host_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                            *args, int(chunk_frames), _dtype_code(q), _dtype_code(out),
+                                            _stream_ptr(stream)))
+    else:
+        _check(lib.monarch_attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                         *args, _dtype_code(q), _dtype_code(out), _stream_ptr(stream)))
     return out
 
 

@@ -968,13 +968,13 @@ int monarch_attn_bwd(const void* q, const void* k, const void* v, const void* dy
   return rc;
 }
 
-int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
-                          void* out_host, int B, int heads, int T, int H, int W, int d,
-                          int tile_h, int tile_w, int iters, long kv_len, int dtype,
-                          int out_dtype, cudaStream_t stream) {
+int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void* v_host,
+                             void* out_host, int B, int heads, int T, int H, int W, int d,
+                             int tile_h, int tile_w, int iters, long kv_len, int chunk_frames, int dtype,
+                             int out_dtype, cudaStream_t stream) {
   g_err.clear();
   Plan p;
-  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p);
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &p, chunk_frames);
   if (rc) return rc;
   if (!q_host || !k_host || !v_host || !out_host) return fail(MONARCH_EINVAL, "null host pointer");
   HostStreams hs;
@@ -992,7 +992,8 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
   const long long gs = (U + ng - 1) / ng;
   ng = (int)((U + gs - 1) / gs);
   Plan pg;   // one group of gs units (B = 1, heads = gs); the last group may be smaller
-  if ((rc = make_plan(1, (int)gs, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pg))) return rc;
+  if ((rc = make_plan(1, (int)gs, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pg, chunk_frames)))
+    return rc;
   const size_t oq = 0, ok = align256(U * qu), ov = ok + align256(U * ku), oo = ov + align256(U * ku);
   const size_t ow = oo + align256(U * ou);
   char* buf = nullptr;
@@ -1022,7 +1023,8 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
     for (int gi = 0; gi < ng && rc == MONARCH_OK; ++gi) {
       const long long u0 = gi * gs, n = std::min<long long>(gs, U - u0);
       Plan pn = pg;
-      if (n != gs && (rc = make_plan(1, (int)n, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pn)))
+      if (n != gs &&
+          (rc = make_plan(1, (int)n, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pn, chunk_frames)))
         break;
       cudaStreamWaitEvent(stream, ev[gi], 0);
       rc = dispatch(pn, buf + oq + u0 * qu, buf + ok + u0 * ku, buf + ov + u0 * ku, buf + oo + u0 * ou, buf + ow,
@@ -1044,6 +1046,14 @@ int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_
   e = cudaStreamSynchronize(stream);
   if (rc == MONARCH_OK && e != cudaSuccess) rc = cuda_fail(e, "cudaStreamSynchronize");
   return rc;
+}
+
+int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                          void* out_host, int B, int heads, int T, int H, int W, int d,
+                          int tile_h, int tile_w, int iters, long kv_len, int dtype,
+                          int out_dtype, cudaStream_t stream) {
+  return monarch_attn_fwd_host_ex(q_host, k_host, v_host, out_host, B, heads, T, H, W, d, tile_h, tile_w, iters,
+                                  kv_len, 0, dtype, out_dtype, stream);
 }
 
 }  // extern "C"

@@ -202,6 +202,18 @@ def test_host_buffer_groups_match_the_device_call(name, cuda_lib):
     assert torch.equal(out, dev)
 
 
+def test_host_buffer_groups_with_the_chunk_mask(cuda_lib):
+    """The masked host entry point (6 groups of 2 heads) equals the masked
+    device call."""
+    w = _custom("bf16", 6, 30, 52, 128, 6, 4, 2, B=1, heads=12, C=2)
+    q, k, v = make_inputs(w)
+    out = torch.empty(q.shape, dtype=torch.float32).pin_memory()
+    m.monarch_attn_fwd_host(q.pin_memory(), k.pin_memory(), v.pin_memory(), out, w.T, w.H, w.W, w.th,
+                            w.tw, w.iters, chunk_frames=w.chunk_frames)
+    dev = _run_gpu(w, q, k, v).cpu()
+    assert torch.equal(out, dev)
+
+
 def test_workspace_entry_point_matches_allocating_call(cuda_lib):
     w = WORKLOADS["chunk_4680_bf16"]
     q, k, v = (t.cuda() for t in make_inputs(w))
