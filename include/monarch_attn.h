@@ -134,6 +134,29 @@ int monarch_attn_bwd(const void* q, const void* k, const void* v, const void* dy
                      int tile_h, int tile_w, int chunk_frames,
                      int dtype, int grad_dtype, cudaStream_t stream);
 
+/* Saved-state training pair (bf16 / f16 inputs).  monarch_attn_fwd_train is
+ * the one-step forward of monarch_attn_bwd's setting (iters = 1,
+ * self-attention, chunk_frames as in monarch_attn_fwd_ex) with an f32 output
+ * `out` [B, heads, T*H*W, d] and, in `lse`, the base-2 log-sum-exp of every
+ * row of the factor L: f32, [B*heads][tile_h*tile_w][b1q_pad] with b1q =
+ * T*(H/tile_h)*(W/tile_w) query tiles and b1q_pad = b1q rounded up to a
+ * multiple of 4, monarch_attn_lse_bytes(...) bytes, caller-owned.
+ * monarch_attn_bwd_saved takes that out and lse and returns the gradients of
+ * monarch_attn_bwd without recomputing the output pass (the same values).
+ * Both are asynchronous on `stream`; f32 inputs return MONARCH_EUNSUPPORTED
+ * (use monarch_attn_bwd); other errors as monarch_attn_bwd. */
+size_t monarch_attn_lse_bytes(int B, int heads, int T, int H, int W, int d, int tile_h, int tile_w);
+
+int monarch_attn_fwd_train(const void* q, const void* k, const void* v, float* out, float* lse,
+                           int B, int heads, int T, int H, int W, int d,
+                           int tile_h, int tile_w, int chunk_frames, int dtype, cudaStream_t stream);
+
+int monarch_attn_bwd_saved(const void* q, const void* k, const void* v, const float* out,
+                           const float* lse, const void* dy, void* dq, void* dk, void* dv,
+                           int B, int heads, int T, int H, int W, int d,
+                           int tile_h, int tile_w, int chunk_frames,
+                           int dtype, int grad_dtype, cudaStream_t stream);
+
 /* Bytes of workspace monarch_attn_bwd takes for these arguments (0 on
  * invalid arguments). */
 size_t monarch_attn_bwd_workspace_bytes(int B, int heads, int T, int H, int W, int d,

@@ -24,6 +24,9 @@ _SIGS = {
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p]),
     "monarch_attn_bwd": (ctypes.c_int, [ctypes.c_void_p] * 7 + [ctypes.c_int] * 11 + [ctypes.c_void_p]),
     "monarch_attn_bwd_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 11),
+    "monarch_attn_lse_bytes": (ctypes.c_size_t, [ctypes.c_int] * 8),
+    "monarch_attn_fwd_train": (ctypes.c_int, [ctypes.c_void_p] * 5 + [ctypes.c_int] * 10 + [ctypes.c_void_p]),
+    "monarch_attn_bwd_saved": (ctypes.c_int, [ctypes.c_void_p] * 9 + [ctypes.c_int] * 11 + [ctypes.c_void_p]),
     "monarch_attn_workspace_bytes": (ctypes.c_size_t, [ctypes.c_int] * 9 + [ctypes.c_long, ctypes.c_int]),
     "monarch_attn_fwd_ws": (ctypes.c_int, [ctypes.c_void_p] * 4 + [ctypes.c_int] * 9
                             + [ctypes.c_long, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
@@ -144,6 +147,46 @@ def monarch_attn_bwd(q, k, v, dy, dq, dk, dv, T, H, W, tile_h, tile_w, stream=No
     _check(lib.monarch_attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), dy.data_ptr(), dq.data_ptr(),
                                 dk.data_ptr(), dv.data_ptr(), B, heads, T, H, W, d, tile_h, tile_w,
                                 int(chunk_frames), _dtype_code(q), g, _stream_ptr(stream)))
+    return dq, dk, dv
+
+
+def lse_numel(B, heads, T, H, W, d, tile_h, tile_w) -> int:
+    """float32 elements of the row-LSE buffer of monarch_attn_fwd_train."""
+    n = load_library().monarch_attn_lse_bytes(B, heads, T, H, W, d, tile_h, tile_w)
+    if n == 0:
+        raise MonarchError(-1, _lib.monarch_attn_last_error().decode())
+    return int(n) // 4
+
+
+def monarch_attn_fwd_train(q, k, v, out, lse, T, H, W, tile_h, tile_w, stream=None, chunk_frames=0):
+    """One-step forward (bf16/f16 inputs) that also keeps the row LSE for
+    monarch_attn_bwd_saved: out float32 [B, heads, T*H*W, d], lse float32 with
+    lse_numel(...) elements (contiguous CUDA tensors).  Asynchronous."""
+    lib = load_library()
+    _check_tensors(q, k, v, out, lse)
+    B, heads, nq, d = q.shape
+    import torch
+    if out.dtype != torch.float32 or lse.dtype != torch.float32:
+        raise TypeError("out and lse must be float32")
+    _check(lib.monarch_attn_fwd_train(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      B, heads, T, H, W, d, tile_h, tile_w, int(chunk_frames), _dtype_code(q),
+                                      _stream_ptr(stream)))
+    return out, lse
+
+
+def monarch_attn_bwd_saved(q, k, v, out, lse, dy, dq, dk, dv, T, H, W, tile_h, tile_w, stream=None,
+                           chunk_frames=0):
+    """monarch_attn_bwd with the out and lse of monarch_attn_fwd_train (no
+    recompute of the output pass)."""
+    lib = load_library()
+    _check_tensors(q, k, v, out, lse, dy, dq, dk, dv)
+    B, heads, nq, d = q.shape
+    g = _dtype_code(dy)
+    if any(_dtype_code(t) != g for t in (dq, dk, dv)):
+        raise TypeError("dy, dq, dk, dv must share a dtype")
+    _check(lib.monarch_attn_bwd_saved(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                                      dy.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, heads, T, H, W,
+                                      d, tile_h, tile_w, int(chunk_frames), _dtype_code(q), g, _stream_ptr(stream)))
     return dq, dk, dv
 
 

@@ -611,20 +611,23 @@ int run_bwd(const BwdPlan& bp, const T* q, const T* k, const T* v, const TG* dy,
 // pass recompute k~, z, h, y and the row LSE; dy becomes scaled f16
 // hi/lo planes with D = sigma dy . y; the two tensor-core L-step kernels give
 // dk~, dz, dh and the L-step dq; the per-tile R-step backward finishes.
+// saved_out / saved_lse: the output (f32) and row LSE written by the one-step
+// training forward; when given, the output pass is not recomputed.
 template <typename TQ, typename TG, int D>
 int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const TG* dy, TG* dq, TG* dk, TG* dv,
-               char* ws, cudaStream_t st) {
+               char* ws, cudaStream_t st, const float* saved_out = nullptr, const float* saved_lse = nullptr) {
   const Plan& p = bp.fwd;
   const Geo& g = p.g;
+  const bool saved = saved_out != nullptr;
   Work w;
   w.kt = reinterpret_cast<float*>(ws + p.off[0]);
   w.z = reinterpret_cast<float*>(ws + p.off[1]);
   w.qt = reinterpret_cast<float*>(ws + p.off[2]);
   w.h = reinterpret_cast<float*>(ws + p.off[3]);
-  w.lse = reinterpret_cast<float*>(ws + p.off[4]);
+  w.lse = saved ? const_cast<float*>(saved_lse) : reinterpret_cast<float*>(ws + p.off[4]);   // read only when saved
   w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
   w.qb = ws + p.off[6];
-  float* y = reinterpret_cast<float*>(ws + bp.toff[0]);
+  const float* y = saved ? saved_out : reinterpret_cast<const float*>(ws + bp.toff[0]);
   __half* dyp = reinterpret_cast<__half*>(ws + bp.toff[1]);
   float* ddv = reinterpret_cast<float*>(ws + bp.toff[2]);
   unsigned* amax = reinterpret_cast<unsigned*>(ws + bp.toff[3]);
@@ -680,9 +683,11 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
                r_group);
   });
   // the output pass gives y and the row LSE of the same (hi + lo) scores
-  launch(MONARCH_PHASE_L_OUT, st, [&] {
-    launch_pdl(tc::l_row<__half, float, D, true, true>, grid_q, dim3(tc::kThreads), smem_out, st, y, maps, w.lse, g);
-  });
+  if (!saved)
+    launch(MONARCH_PHASE_L_OUT, st, [&] {
+      launch_pdl(tc::l_row<__half, float, D, true, true>, grid_q, dim3(tc::kThreads), smem_out, st,
+                 const_cast<float*>(y), maps, w.lse, g);
+    });
   cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)g.BH * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   launch(MONARCH_PHASE_BWD_PREP, st, [&] {
@@ -706,6 +711,68 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
   return MONARCH_OK;
+}
+
+// One-step training forward (bf16 / f16): the R step, then the output pass
+// writing the f32 output and the row LSE that monarch_attn_bwd_saved reads.
+template <typename TQ, int D>
+int run_fwd_train_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, float* out, float* lse, char* ws,
+                     cudaStream_t st) {
+  const Geo& g = p.g;
+  Work w;
+  w.kt = reinterpret_cast<float*>(ws + p.off[0]);
+  w.z = reinterpret_cast<float*>(ws + p.off[1]);
+  w.qt = reinterpret_cast<float*>(ws + p.off[2]);
+  w.h = reinterpret_cast<float*>(ws + p.off[3]);
+  w.lse = lse;
+  w.qbar = reinterpret_cast<float*>(ws + p.off[5]);
+  w.qb = ws + p.off[6];
+  TcPlanes<TQ> planes;
+  tc::Maps maps;
+  RtcMaps rmaps;
+  int rc;
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
+  constexpr size_t smem_out = tc::row_smem<D, true>();
+  constexpr size_t smem_r = rtc_smem<D>();
+  static bool attrs_set = false;
+  if (!attrs_set) {
+    cudaError_t e;
+    if ((e = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
+        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
+      return cuda_fail(e, "cudaFuncSetAttribute");
+    attrs_set = true;
+  }
+  const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
+  const int r_group = r_step_group(g, sm_count_of_device());
+  const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
+  launch(MONARCH_PHASE_R_STEP, st, [&] {
+    launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1,
+               r_group);
+  });
+  launch(MONARCH_PHASE_L_OUT, st, [&] {
+    launch_pdl(tc::l_row<__half, float, D, true, true>, grid_q, dim3(tc::kThreads), smem_out, st, out, maps, lse, g);
+  });
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+  return MONARCH_OK;
+}
+
+// Saved-state backward: the bf16 / f16 tensor-core path with y and the LSE
+// from monarch_attn_fwd_train.
+template <typename T>
+int dispatch_bwd_saved(const BwdPlan& bp, const void* q, const void* k, const void* v, const float* out,
+                       const float* lse, const void* dy, void* dq, void* dk, void* dv, char* ws, cudaStream_t st) {
+  const T *qq = (const T*)q, *kk = (const T*)k, *vv = (const T*)v;
+  if (bp.fwd.g.d == 128) {
+    if (bp.grad_dtype == MONARCH_F32)
+      return run_bwd_tc<T, float, 128>(bp, qq, kk, vv, (const float*)dy, (float*)dq, (float*)dk, (float*)dv, ws, st,
+                                       out, lse);
+    return run_bwd_tc<T, T, 128>(bp, qq, kk, vv, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws, st, out, lse);
+  }
+  if (bp.grad_dtype == MONARCH_F32)
+    return run_bwd_tc<T, float, 64>(bp, qq, kk, vv, (const float*)dy, (float*)dq, (float*)dk, (float*)dv, ws, st,
+                                    out, lse);
+  return run_bwd_tc<T, T, 64>(bp, qq, kk, vv, (const T*)dy, (T*)dq, (T*)dk, (T*)dv, ws, st, out, lse);
 }
 
 template <typename T>
@@ -963,6 +1030,77 @@ int monarch_attn_bwd(const void* q, const void* k, const void* v, const void* dy
     return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", bp.total, cudaGetErrorString(e));
   }
   rc = dispatch_bwd(bp, q, k, v, dy, dq, dk, dv, ws, stream);
+  e = cudaFreeAsync(ws, stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+size_t monarch_attn_lse_bytes(int B, int heads, int T, int H, int W, int d, int tile_h, int tile_w) {
+  Plan p;
+  if (make_plan(B, heads, T, H, W, d, tile_h, tile_w, 1, (long)T * H * W, MONARCH_BF16, MONARCH_BF16, &p) != MONARCH_OK)
+    return 0;
+  return (size_t)p.g.BH * p.g.b2 * p.g.b1q_pad * 4;
+}
+
+int monarch_attn_fwd_train(const void* q, const void* k, const void* v, float* out, float* lse, int B, int heads,
+                           int T, int H, int W, int d, int tile_h, int tile_w, int chunk_frames, int dtype,
+                           cudaStream_t stream) {
+  g_err.clear();
+  Plan p;
+  int rc = make_plan(B, heads, T, H, W, d, tile_h, tile_w, 1, (long)T * H * W, dtype, MONARCH_F32, &p, chunk_frames);
+  if (rc) return rc;
+  if (dtype == MONARCH_F32)
+    return fail(MONARCH_EUNSUPPORTED, "the saved-state training pair is for bf16 / f16 inputs (f32: monarch_attn_bwd)");
+  if ((rc = check_io(q, k, v, out)) || (rc = check_ptr(lse, "lse"))) return rc;
+  void* ws = nullptr;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, p.total, pool, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", p.total, cudaGetErrorString(e));
+  }
+  char* w = static_cast<char*>(ws);
+  if (dtype == MONARCH_BF16)
+    rc = d == 128 ? run_fwd_train_tc<__nv_bfloat16, 128>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                          (const __nv_bfloat16*)v, out, lse, w, stream)
+                  : run_fwd_train_tc<__nv_bfloat16, 64>(p, (const __nv_bfloat16*)q, (const __nv_bfloat16*)k,
+                                                         (const __nv_bfloat16*)v, out, lse, w, stream);
+  else
+    rc = d == 128 ? run_fwd_train_tc<__half, 128>(p, (const __half*)q, (const __half*)k, (const __half*)v, out, lse, w,
+                                                   stream)
+                  : run_fwd_train_tc<__half, 64>(p, (const __half*)q, (const __half*)k, (const __half*)v, out, lse, w,
+                                                  stream);
+  e = cudaFreeAsync(ws, stream);
+  if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
+  return rc;
+}
+
+int monarch_attn_bwd_saved(const void* q, const void* k, const void* v, const float* out, const float* lse,
+                           const void* dy, void* dq, void* dk, void* dv, int B, int heads, int T, int H, int W, int d,
+                           int tile_h, int tile_w, int chunk_frames, int dtype, int grad_dtype, cudaStream_t stream) {
+  g_err.clear();
+  BwdPlan bp;
+  int rc = make_bwd_plan(B, heads, T, H, W, d, tile_h, tile_w, chunk_frames, dtype, grad_dtype, &bp);
+  if (rc) return rc;
+  if (dtype == MONARCH_F32)
+    return fail(MONARCH_EUNSUPPORTED, "the saved-state training pair is for bf16 / f16 inputs (f32: monarch_attn_bwd)");
+  if ((rc = check_ptr(q, "q")) || (rc = check_ptr(k, "k")) || (rc = check_ptr(v, "v")) ||
+      (rc = check_ptr(out, "out")) || (rc = check_ptr(lse, "lse")) || (rc = check_ptr(dy, "dy")) ||
+      (rc = check_ptr(dq, "dq")) || (rc = check_ptr(dk, "dk")) || (rc = check_ptr(dv, "dv")))
+    return rc;
+  void* ws = nullptr;
+  cudaMemPool_t pool;
+  if ((rc = workspace_pool(&pool))) return rc;
+  cudaError_t e = cudaMallocFromPoolAsync(&ws, bp.total, pool, stream);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MONARCH_ENOMEM, "cudaMallocFromPoolAsync(%zu): %s", bp.total, cudaGetErrorString(e));
+  }
+  char* w = static_cast<char*>(ws);
+  rc = dtype == MONARCH_BF16
+           ? dispatch_bwd_saved<__nv_bfloat16>(bp, q, k, v, out, lse, dy, dq, dk, dv, w, stream)
+           : dispatch_bwd_saved<__half>(bp, q, k, v, out, lse, dy, dq, dk, dv, w, stream);
   e = cudaFreeAsync(ws, stream);
   if (rc == MONARCH_OK && e != cudaSuccess) return cuda_fail(e, "cudaFreeAsync");
   return rc;

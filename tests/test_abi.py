@@ -149,3 +149,16 @@ def test_backward_workspace_holds_the_gradient_intermediates(lib):
     big = 12 * 24 * 195 * 128 * 4   # fp32 k~, z, dqL, dk~, dz
     assert n >= 5 * big + 4 * 12 * 24 * 195 * 4
     assert lib.monarch_attn_bwd_workspace_bytes(1, 12, 3, 30, 52, 128, 6, 4, 0, 1, 2) == 0
+
+
+def test_lse_bytes_and_training_pair_validation(lib):
+    # 12 heads x 24 positions x b1q = 195 rounded up to 196, float32
+    assert lib.monarch_attn_lse_bytes(1, 12, 3, 30, 52, 128, 6, 4) == 12 * 24 * 196 * 4
+    ptrs = (0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    assert lib.monarch_attn_fwd_train(*ptrs, 1, 2, 3, 8, 12, 64, 2, 4, 0, 0, None) == -4   # f32 inputs
+    assert "bf16" in lib.monarch_attn_last_error().decode()
+    assert lib.monarch_attn_fwd_train(*ptrs[:4], None, 1, 2, 3, 8, 12, 64, 2, 4, 0, 1, None) == -1
+    assert "lse is null" in lib.monarch_attn_last_error().decode()
+    bptrs = (0x1000, 0x2000, 0x3000, 0x4000, None, 0x6000, 0x7000, 0x8000, 0x9000)
+    assert lib.monarch_attn_bwd_saved(*bptrs, 1, 2, 3, 8, 12, 64, 2, 4, 0, 1, 0, None) == -1
+    assert "lse is null" in lib.monarch_attn_last_error().decode()

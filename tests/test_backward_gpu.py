@@ -146,3 +146,29 @@ def test_backward_rejects_a_kv_cache_shape(cuda_lib):
     with pytest.raises(ValueError):
         m.monarch_attn_bwd(q.cuda(), k, k, q.cuda().float(), *(torch.empty_like(q.cuda().float()) for _ in range(3)),
                            w.T, w.H, w.W, w.th, w.tw)
+
+
+@pytest.mark.parametrize("w,gdt", [(_wl("bf16", 5, 12, 20, 128, 4, 4), "f32"),
+                                   (_wl("f16", 6, 8, 8, 64, 4, 2, C=2), "f16")],
+                         ids=["bf16_gf32", "f16_masked_gf16"])
+def test_saved_state_pair_matches_the_recomputing_backward(w, gdt, cuda_lib):
+    """monarch_attn_fwd_train writes the one-step forward's output and row LSE;
+    monarch_attn_bwd_saved with them returns the gradients of monarch_attn_bwd
+    bit for bit (both run the same kernels on the same values)."""
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    dy = make_cotangent(w, gdt).cuda()
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    lse = torch.empty(m.lse_numel(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw), dtype=torch.float32,
+                      device="cuda")
+    m.monarch_attn_fwd_train(q, k, v, out, lse, w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
+    ref_out = torch.empty_like(out)
+    m.monarch_attn_fwd(q, k, v, ref_out, w.T, w.H, w.W, w.th, w.tw, 1, chunk_frames=w.chunk_frames)
+    got = [torch.empty_like(dy) for _ in range(3)]
+    ref = [torch.empty_like(dy) for _ in range(3)]
+    m.monarch_attn_bwd_saved(q, k, v, out, lse, dy, *got, w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
+    m.monarch_attn_bwd(q, k, v, dy, *ref, w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
+    torch.cuda.synchronize()
+    assert m.device_error() == 0
+    assert torch.equal(out, ref_out)
+    for a, b in zip(got, ref):
+        assert torch.equal(a, b)
