@@ -20,7 +20,7 @@
 // the R step), dy (scaled by a power of two sigma per head so that
 // max |sigma dy| lies in [1/2, 1)), P and dS; q is exact in f16.  A product
 // of two split operands takes three MMAs (hi hi, lo hi, hi lo).  dS is scaled
-// by 2^kDsShift before its split; fp32 accumulation throughout.
+// by kDsShift = 16 before its split; fp32 accumulation throughout.
 //
 // TMEM (512 columns): X [0, 128), Y [128, 256), accumulators from 256.  A
 // 16-column group of X or Y that held 16 scores holds, after the softmax, the
@@ -34,6 +34,12 @@
 // Each block's products that read P or dS are issued before the next block's
 // score products, and one thread's MMAs run in issue order, so the next
 // scores never overwrite an operand still in use.
+//
+// Overlap: the streamed operands have their own refill barriers, released in
+// the order their last readers finish (l_bwd_kv: q after dk~, dy after dz;
+// l_bwd_q: z right after dP, k~ after dq), so the next block's loads run under
+// the current block's products.  In l_bwd_kv the score and dP products commit
+// separately and the softmax computes P while dP is still being formed.
 #pragma once
 
 #include "tc_common.cuh"
@@ -89,7 +95,7 @@ constexpr size_t q_smem() {
 //   softmax_ds: reads P back (hi + lo, about 22 bits) and 16 values Y, forms
 //               dS = P (y - dd(j)) and writes the hi/lo planes of 2^shift dS
 //               over the group of Y.  Accumulates dS into dsum; tracks
-//               max |2^shift dS|.
+//               max |kDsShift dS|.
 template <typename Off, typename Keep>
 __device__ __forceinline__ void softmax_p(uint32_t tx, float sl2, Off off, Keep keep) {
   uint32_t xr[16];
@@ -133,7 +139,7 @@ __device__ __forceinline__ void softmax_ds(uint32_t tx, uint32_t ty, Dv dd, floa
 }
 
 // One-phase variant for the dq kernel, where only dS is an MMA operand: reads
-// 16 scores X and 16 values Y, writes the hi/lo planes of 2^shift dS over the
+// 16 scores X and 16 values Y, writes the hi/lo planes of kDsShift dS over the
 // group of Y.
 template <typename Off, typename Keep>
 __device__ __forceinline__ void softmax_ds_only(uint32_t tx, uint32_t ty, float sl2, Off off, float dd, Keep keep,
