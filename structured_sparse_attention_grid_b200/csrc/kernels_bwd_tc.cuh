@@ -93,7 +93,7 @@ constexpr size_t q_smem() {
 //               planes over the group (hi in the first 8 columns, lo in the
 //               last 8);
 //   softmax_ds: reads P back (hi + lo, about 22 bits) and 16 values Y, forms
-//               dS = P (y - dd(j)) and writes the hi/lo planes of 2^shift dS
+//               dS = P (y - dd(j)) and writes the hi/lo planes of kDsShift dS
 //               over the group of Y.  Accumulates dS into dsum; tracks
 //               max |kDsShift dS|.
 template <typename Off, typename Keep>
