@@ -265,3 +265,60 @@ def profile_read(reset: bool = True) -> dict:
 def device_error(reset: bool = False) -> int:
     """0 unless a library kernel gave up a bounded wait (see the header)."""
     return int(load_library().monarch_attn_device_error(1 if reset else 0))
+
+
+def _autograd_function():
+    import torch
+
+    class MonarchAttentionFn(torch.autograd.Function):
+        """One-step Monarch attention with its backward (the finetuned
+        regime): forward through monarch_attn_fwd_train (bf16/f16, keeps the
+        row LSE) or monarch_attn_fwd (f32); backward through
+        monarch_attn_bwd_saved or monarch_attn_bwd, with f32 gradients."""
+
+        @staticmethod
+        def forward(ctx, q, k, v, T, H, W, tile_h, tile_w, chunk_frames):
+            q, k, v = (t.contiguous() for t in (q, k, v))
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+            if q.dtype == torch.float32:
+                monarch_attn_fwd(q, k, v, out, T, H, W, tile_h, tile_w, 1, chunk_frames=chunk_frames)
+                lse = torch.empty(0, dtype=torch.float32, device=q.device)
+            else:
+                B, heads, _, d = q.shape
+                lse = torch.empty(lse_numel(B, heads, T, H, W, d, tile_h, tile_w), dtype=torch.float32,
+                                  device=q.device)
+                monarch_attn_fwd_train(q, k, v, out, lse, T, H, W, tile_h, tile_w, chunk_frames=chunk_frames)
+            ctx.save_for_backward(q, k, v, out, lse)
+            ctx.geom = (T, H, W, tile_h, tile_w, chunk_frames)
+            return out
+
+        @staticmethod
+        def backward(ctx, dy):
+            q, k, v, out, lse = ctx.saved_tensors
+            T, H, W, tile_h, tile_w, chunk_frames = ctx.geom
+            dy = dy.contiguous()
+            if dy.dtype != torch.float32:
+                dy = dy.float()
+            dq, dk, dv = (torch.empty_like(dy) for _ in range(3))
+            if q.dtype == torch.float32:
+                monarch_attn_bwd(q, k, v, dy, dq, dk, dv, T, H, W, tile_h, tile_w, chunk_frames=chunk_frames)
+            else:
+                monarch_attn_bwd_saved(q, k, v, out, lse, dy, dq, dk, dv, T, H, W, tile_h, tile_w,
+                                       chunk_frames=chunk_frames)
+            return dq, dk, dv, None, None, None, None, None, None
+
+    return MonarchAttentionFn
+
+
+_FN = None
+
+
+def monarch_attention(q, k, v, T, H, W, tile_h, tile_w, chunk_frames=0):
+    """Differentiable one-step Monarch attention (self-attention, optional
+    frame-chunk causal mask): CUDA tensors [B, heads, T*H*W, d]; returns the
+    float32 output.  Gradients flow to q, k, v (float32, converted by
+    autograd to the inputs' dtype)."""
+    global _FN
+    if _FN is None:
+        _FN = _autograd_function()
+    return _FN.apply(q, k, v, T, H, W, tile_h, tile_w, chunk_frames)

@@ -172,3 +172,25 @@ def test_saved_state_pair_matches_the_recomputing_backward(w, gdt, cuda_lib):
     assert torch.equal(out, ref_out)
     for a, b in zip(got, ref):
         assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("dtype,C", [("bf16", 0), ("f32", 2)])
+def test_autograd_function_gives_the_library_gradients(dtype, C, cuda_lib):
+    """loss = sum(dy * monarch_attention(q, k, v)); loss.backward() yields the
+    gradients of the backward entry point (f32 gradients, converted to the
+    inputs' dtype by autograd)."""
+    w = _wl(dtype, 4, 8, 12, 64, 2, 4, C=C)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    dy = make_cotangent(w, "f32").cuda()
+    qg, kg, vg = (t.clone().requires_grad_() for t in (q, k, v))
+    y = m.monarch_attention(qg, kg, vg, w.T, w.H, w.W, w.th, w.tw, chunk_frames=C)
+    (y * dy).sum().backward()
+    ref = [torch.empty_like(dy) for _ in range(3)]
+    m.monarch_attn_bwd(q, k, v, dy, *ref, w.T, w.H, w.W, w.th, w.tw, chunk_frames=C)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, 1, chunk_frames=C)
+    torch.cuda.synchronize()
+    assert torch.equal(y.detach(), out)
+    for g, r, t in zip((qg.grad, kg.grad, vg.grad), ref, (q, k, v)):
+        assert g.dtype == t.dtype
+        assert torch.equal(g, r.to(t.dtype))
