@@ -38,8 +38,8 @@
 // Overlap: the streamed operands have their own refill barriers, released in
 // the order their last readers finish (l_bwd_kv: q after dk~, dy after dz;
 // l_bwd_q: z right after dP, k~ after dq), so the next block's loads run under
-// the current block's products.  In l_bwd_kv the score and dP products commit
-// separately and the softmax computes P while dP is still being formed.
+// the current block's products.  The score and dP products commit separately
+// and the softmax computes P while dP is still being formed.
 #pragma once
 
 #include "tc_common.cuh"
@@ -138,17 +138,17 @@ __device__ __forceinline__ void softmax_ds(uint32_t tx, uint32_t ty, Dv dd, floa
   ptx::tmem_st8(ty + 8, slo);
 }
 
-// One-phase variant for the dq kernel, where only dS is an MMA operand: reads
-// 16 scores X and 16 values Y, writes the hi/lo planes of kDsShift dS over the
-// group of Y.
+// Two-phase variant for the dq kernel, where only dS is an MMA operand:
+//   softmax_p_regs: P of 16 columns from X, kept in registers as 8 packed f16
+//                   pairs (P only scales dP - D, so one f16 rounding of P is a
+//                   2^-11 relative error of dS, with no cancellation);
+//   softmax_ds_regs: dS = P (y - dd) from those registers and 16 values Y,
+//                   written over the group of Y as hi/lo planes of kDsShift dS.
 template <typename Off, typename Keep>
-__device__ __forceinline__ void softmax_ds_only(uint32_t tx, uint32_t ty, float sl2, Off off, float dd, Keep keep,
-                                                float& dmax) {
-  uint32_t xr[16], yr[16];
+__device__ __forceinline__ void softmax_p_regs(uint32_t tx, float sl2, Off off, Keep keep, uint32_t (&ph)[8]) {
+  uint32_t xr[16];
   ptx::tmem_ld16(tx, xr);
-  ptx::tmem_ld16(ty, yr);
   ptx::tmem_wait_ld();
-  uint32_t shi[8], slo[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     const int j = 2 * e;
@@ -156,8 +156,21 @@ __device__ __forceinline__ void softmax_ds_only(uint32_t tx, uint32_t ty, float 
     float p1 = ptx::ex2(fmaf(__uint_as_float(xr[j + 1]), sl2, off(j + 1)));
     if (!keep(j)) p0 = 0.f;
     if (!keep(j + 1)) p1 = 0.f;
-    const float2 ds = make_float2(p0 * (__uint_as_float(yr[j]) - dd) * kDsShift,
-                                  p1 * (__uint_as_float(yr[j + 1]) - dd) * kDsShift);
+    const __half2 h = __floats2half2_rn(p0, p1);
+    ph[e] = *reinterpret_cast<const uint32_t*>(&h);
+  }
+}
+
+__device__ __forceinline__ void softmax_ds_regs(uint32_t ty, const uint32_t (&ph)[8], float dd, float& dmax) {
+  uint32_t yr[16];
+  ptx::tmem_ld16(ty, yr);
+  ptx::tmem_wait_ld();
+  uint32_t shi[8], slo[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const float2 p = __half22float2(*reinterpret_cast<const __half2*>(&ph[e]));
+    const float2 ds = make_float2(p.x * (__uint_as_float(yr[2 * e]) - dd) * kDsShift,
+                                  p.y * (__uint_as_float(yr[2 * e + 1]) - dd) * kDsShift);
     dmax = fmaxf(dmax, fmaxf(fabsf(ds.x), fabsf(ds.y)));
     tc::split2<__half>(ds, shi[e], slo[e]);
   }
@@ -544,15 +557,19 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
       ok = ok && ptx::mbar_wait(s_full, j & 1) && ptx::mbar_wait(k_full, j & 1);
       ptx::tc_fence_after();
       const int lim = climit - k0;
-      ok = ok && ptx::mbar_wait(d_full, j & 1);
-      ptx::tc_fence_after();
+      uint32_t ph[2][8];   // P of the two 16-column groups (f16 pairs), formed while dP is computed
 #pragma unroll
       for (int g16 = 0; g16 < 2; ++g16) {
         const int cb = 32 * cq + 16 * g16;
         const float* hv = sH + cb;
-        softmax_ds_only(tX + lane_off + cb, tY + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; }, dd,
-                        [&](int jj) { return cb + jj < lim; }, dmax);
+        softmax_p_regs(tX + lane_off + cb, g.sl2, [&](int jj) { return hv[jj] - l; },
+                       [&](int jj) { return cb + jj < lim; }, ph[g16]);
       }
+      ok = ok && ptx::mbar_wait(d_full, j & 1);
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int g16 = 0; g16 < 2; ++g16)
+        softmax_ds_regs(tY + lane_off + 32 * cq + 16 * g16, ph[g16], dd, dmax);
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();
