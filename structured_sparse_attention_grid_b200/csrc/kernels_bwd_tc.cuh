@@ -591,15 +591,16 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
 
 // ===========================================================================
 // Largest |dy| per head (as the bits of a non-negative float, which order like
-// unsigned integers).  Each thread reads 16 consecutive elements (four 16-byte
-// or 8-byte loads in flight).  grid (ceil(Nq*d / 4096), BH), block 256.
+// unsigned integers).  Grid-stride over the head: each thread takes 16
+// consecutive elements per step (four 16-byte or 8-byte loads in flight).
+// grid (blocks per head, BH), block 256.
 template <typename TG>
 __global__ void __launch_bounds__(256) dy_amax(const TG* __restrict__ dy, unsigned* __restrict__ amax, Geo g) {
   const long long n = g.Nq * g.d;   // a multiple of 64
   const TG* p = dy + (long long)blockIdx.y * n;
-  const long long base = ((long long)blockIdx.x * 256 + threadIdx.x) * 16;
   float m = 0.f;
-  if (base < n) {
+  for (long long base = ((long long)blockIdx.x * 256 + threadIdx.x) * 16; base < n;
+       base += (long long)gridDim.x * 256 * 16) {
     float4 v[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) v[i] = load4(p + base + 4 * i);

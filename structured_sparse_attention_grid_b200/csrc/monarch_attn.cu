@@ -691,8 +691,11 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)g.BH * 4, st);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync");
   launch(MONARCH_PHASE_BWD_PREP, st, [&] {
+    // about 8 blocks of 256 threads per SM over all heads, each striding through its head
     const long long n = g.Nq * D;
-    tcb::dy_amax<TG><<<dim3((unsigned)((n + 4095) / 4096), g.BH), 256, 0, st>>>(dy, amax, g);
+    const long long per_head = std::max<long long>(1, std::min<long long>((n + 4095) / 4096,
+                                                                         (8LL * sm_count_of_device() + g.BH - 1) / g.BH));
+    tcb::dy_amax<TG><<<dim3((unsigned)per_head, g.BH), 256, 0, st>>>(dy, amax, g);
   });
   launch(MONARCH_PHASE_BWD_PREP, st, [&] {
     tcb::dy_planes<TG, D><<<dim3((unsigned)((g.Nq + 7) / 8), g.BH), 256, 0, st>>>(dy, y, amax, dyp, ddv, g);
