@@ -166,7 +166,7 @@ size_t monarch_attn_bwd_workspace_bytes(int B, int heads, int T, int H, int W, i
 /* End-to-end variant on HOST buffers: copies q, k, v host->device, runs the
  * forward and copies out device->host, then synchronises `stream` before
  * returning (so `out` is ready).  The (batch, head) units are split into up
- * to 8 groups whose copies overlap: copies in run on a library-owned stream,
+ * to 8 groups (about 10 MB of input each) whose copies overlap: copies in run on a library-owned stream,
  * each group's forward on `stream` after its inputs have landed, its copy
  * out on a second library-owned stream (one pair of non-blocking streams per
  * device, kept for the process).  Device buffers are allocated stream-ordered

@@ -1129,7 +1129,9 @@ int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void*
   const size_t es = elem_size(dtype), eo = elem_size(out_dtype);
   const size_t qu = (size_t)p.g.Nq * d * es, ku = (size_t)p.g.Nk * d * es, ou = (size_t)p.g.Nq * d * eo;
   const long long in_bytes = (long long)(U * (qu + 2 * ku));
-  int ng = (int)std::max<long long>(1, std::min<long long>({in_bytes / (4LL << 20), U, (long long)kHostGroups}));
+  // about 10 MB of input per group: smaller groups make the forward of a group
+  // latency-bound (measured best: 4 groups for 43 MB, 8 for 216 MB and 604 MB)
+  int ng = (int)std::max<long long>(1, std::min<long long>({in_bytes / (10LL << 20), U, (long long)kHostGroups}));
   const long long gs = (U + ng - 1) / ng;
   ng = (int)((U + gs - 1) / gs);
   Plan pg;   // one group of gs units (B = 1, heads = gs); the last group may be smaller
