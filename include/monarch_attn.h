@@ -261,7 +261,8 @@ int monarch_attn_device_error(int reset);
 /* Thread-local message of the last failing call ("" if none). */
 const char* monarch_attn_last_error(void);
 
-/* ABI version (major*100 + minor). */
+/* ABI version (major*100 + minor): 1.02 adds the backward (monarch_attn_bwd),
+ * the training pair and monarch_attn_fwd_host_ex to the forward of 1.00. */
 int monarch_attn_version(void);
 
 #ifdef __cplusplus

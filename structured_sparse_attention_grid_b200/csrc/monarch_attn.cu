@@ -893,7 +893,7 @@ int check_io(const void* q, const void* k, const void* v, const void* out) {
 
 extern "C" {
 
-int monarch_attn_version(void) { return 100; }
+int monarch_attn_version(void) { return 102; }
 
 unsigned long long monarch_attn_launch_count(void) { return g_launches.load(); }
 
