@@ -74,8 +74,8 @@ def test_toy_separable_matches_dense_attention(cuda_lib):
     assert np.abs(out - ref).max() <= TOL_F32
 
 
-@pytest.mark.parametrize("name", ["chunk_4680_bf16", "kvcache_4680x32760_bf16", "sweep_2048_f16",
-                                  "sweep_8192_f16"])
+@pytest.mark.parametrize("name", ["chunk_4680_bf16", "chunk_4680_bf16_1step", "kvcache_4680x32760_bf16",
+                                  "sweep_2048_f16", "sweep_8192_f16"])
 def test_workload_all_heads(name, cuda_lib):
     w = WORKLOADS[name]
     q, k, v = make_inputs(w)
@@ -86,6 +86,7 @@ def test_workload_all_heads(name, cuda_lib):
 
 @pytest.mark.parametrize("name,heads", [
     ("full_32760_bf16", [(0, 0), (1, 11)]),
+    ("full_32760_bf16_1step", [(1, 5)]),
     ("sweep_32768_f16", [(0, 0), (0, 13), (0, 23)]),
 ])
 def test_workload_sampled_heads(name, heads, cuda_lib):
