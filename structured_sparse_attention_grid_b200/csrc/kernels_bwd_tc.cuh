@@ -178,6 +178,34 @@ __device__ __forceinline__ void softmax_ds_regs(uint32_t ty, const uint32_t (&ph
   ptx::tmem_st8(ty + 8, slo);
 }
 
+// The two MMA shapes of both kernels, issued by one thread (f16 operands,
+// f32 accumulation in TMEM):
+//   mma_scores: D[128 x 128] (+)= A[128 x d] B[128 x d]^T, both K-major
+//               (d along the 128-byte swizzled rows): scores and dP;
+//   mma_accum:  D[128 x d] += A[128 x 128] B[128 x d], A in TMEM (plane pa of
+//               the [hi 8 | lo 8] groups), B MN-major: the accumulations.
+template <int D>
+__device__ __forceinline__ void mma_scores(uint32_t td, uint32_t a, uint32_t b, bool first) {
+  constexpr int NH = D / 64;
+  constexpr uint32_t idS = ptx::idesc_f16(128, kBlk, 0, 0, 0);
+  const uint64_t da = ptx::sw128_desc(a, 16, 1024), db = ptx::sw128_desc(b, 16, 1024);
+#pragma unroll
+  for (int hf = 0; hf < NH; ++hf)
+#pragma unroll
+    for (int k4 = 0; k4 < 4; ++k4)
+      ptx::mma_f16_ss(td, da + ((hf * 2 * kBox + k4 * 32) >> 4), db + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
+                      !(first && hf == 0 && k4 == 0));
+}
+
+template <int D>
+__device__ __forceinline__ void mma_accum(uint32_t tacc, uint32_t ta, int pa, uint32_t b, bool first) {
+  constexpr uint32_t idA = ptx::idesc_f16(128, D, 0, 0, 1);
+  const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
+#pragma unroll
+  for (int kk = 0; kk < kBlk / 16; ++kk)
+    ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
+}
+
 // Writes 16 accumulator columns of this thread's row, times `scale`, as f32.
 __device__ __forceinline__ void store_acc16(uint32_t taddr, float scale, float* dst, bool ok) {
   uint32_t o[16];
@@ -292,25 +320,11 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idS = ptx::idesc_f16(128, kBlk, 0, 0, 0);
-      constexpr uint32_t idA = ptx::idesc_f16(128, D, 0, 0, 1);
       const uint32_t aK = ptx::smem_u32(sK), aZ = ptx::smem_u32(sZ), aQ = ptx::smem_u32(sQ), aY = ptx::smem_u32(sY);
       // score-like product: rows x 128 columns over K = d
-      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) {
-        const uint64_t da = ptx::sw128_desc(a, 16, 1024), db = ptx::sw128_desc(b, 16, 1024);
-#pragma unroll
-        for (int hf = 0; hf < NH; ++hf)
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            ptx::mma_f16_ss(td, da + ((hf * 2 * kBox + k4 * 32) >> 4), db + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
-                            !(first && hf == 0 && k4 == 0));
-      };
-      // accumulation: acc += A (TMEM, planes pa over 128 K columns) * B (MN-major, K = 128 rows, N = d)
+      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) { mma_scores<D>(td, a, b, first); };
       auto accum = [&](uint32_t tacc, uint32_t ta, int pa, uint32_t b, bool first) {
-        const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
+        mma_accum<D>(tacc, ta, pa, b, first);
       };
       bool ok = ptx::mbar_wait(k_full, 0);
       for (int j = 0; j < nblk && ok; ++j) {
@@ -497,23 +511,10 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
     }
   } else if (warp == kMmaWarp) {
     if (lane == 0) {
-      constexpr uint32_t idS = ptx::idesc_f16(128, kBlk, 0, 0, 0);
-      constexpr uint32_t idA = ptx::idesc_f16(128, D, 0, 0, 1);
       const uint32_t aK = ptx::smem_u32(sK), aZ = ptx::smem_u32(sZ), aQ = ptx::smem_u32(sQ), aY = ptx::smem_u32(sY);
-      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) {
-        const uint64_t da = ptx::sw128_desc(a, 16, 1024), db = ptx::sw128_desc(b, 16, 1024);
-#pragma unroll
-        for (int hf = 0; hf < NH; ++hf)
-#pragma unroll
-          for (int k4 = 0; k4 < 4; ++k4)
-            ptx::mma_f16_ss(td, da + ((hf * 2 * kBox + k4 * 32) >> 4), db + ((hf * 2 * kBox + k4 * 32) >> 4), idS,
-                            !(first && hf == 0 && k4 == 0));
-      };
+      auto scores = [&](uint32_t td, uint32_t a, uint32_t b, bool first) { mma_scores<D>(td, a, b, first); };
       auto accum = [&](uint32_t tacc, uint32_t ta, int pa, uint32_t b, bool first) {
-        const uint64_t db = ptx::sw128_desc(b, 2 * kBox, 1024);
-#pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk)
-          ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
+        mma_accum<D>(tacc, ta, pa, b, first);
       };
       bool ok = ptx::mbar_wait(c_full, 0);
       for (int j = 0; j < nblk && ok; ++j) {
