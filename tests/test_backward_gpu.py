@@ -100,6 +100,8 @@ CASES = [
     ("f32", _wl("bf16", 2, 6, 8, 128, 1, 1)),               # tensor cores: b2 = 1
     ("f32", _wl("bf16", 1, 6, 8, 128, 6, 8)),               # tensor cores: b1 = 1
     ("f32", _wl("bf16", 9, 16, 16, 128, 4, 4, C=4, B=1)),   # tensor cores: several 128-tile blocks, masked
+    ("f32", _wl("bf16", 2, 8, 8, 128, 4, 4, B=8, heads=12)),   # 96 head units of 8 tiles: padded blocks
+    ("bf16", _wl("bf16", 6, 12, 16, 64, 4, 4, C=3, B=1)),      # tensor cores: d = 64, masked, bf16 gradients
 ]
 
 
