@@ -123,8 +123,13 @@ int monarch_attn_fwd_ws(const void* q, const void* k, const void* v, void* out,
  * q, k, v: [B, heads, T*H*W, d] in `dtype`; dy, dq, dk, dv: [B, heads,
  * T*H*W, d] in `grad_dtype` (MONARCH_F32 or dtype), all caller-owned device
  * memory, 16-byte aligned; dq, dk, dv are overwritten.  The forward factors
- * are recomputed (nothing is kept from the forward call).  Arithmetic: fp32
- * throughout.  Workspace: allocated stream-ordered from the library's pool,
+ * are recomputed (nothing is kept from the forward call).  Arithmetic: f32
+ * inputs run fp32 CUDA-core kernels (gradients within 1e-3 of the RMS of the
+ * exact ones); bf16/f16 inputs run tensor-core kernels that carry every
+ * computed operand as f16 hi + lo planes with fp32 accumulation (within
+ * 2e-2 of the RMS, plus one rounding of the stored gradient).  The second
+ * uses about 3.2 GB of workspace at 24 heads of 32760 tokens.
+ * Workspace: allocated stream-ordered from the library's pool,
  * monarch_attn_bwd_workspace_bytes(...) bytes.  Asynchronous on `stream`;
  * returns MONARCH_OK or a negative status (MONARCH_EINVAL for the checks of
  * monarch_attn_fwd and a bad grad_dtype, MONARCH_EUNSUPPORTED as there). */
