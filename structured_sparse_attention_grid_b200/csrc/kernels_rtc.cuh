@@ -28,6 +28,12 @@
 // 128-byte swizzle; V reuses the A hi plane once the score MMAs are complete.
 // That is 96 KB for d = 128 and 256 TMEM columns, so two CTAs share an SM and
 // one CTA's loads overlap the other's arithmetic.
+//
+// Threads: eight row warps and a control warp.  Row warps w and w + 4 share
+// TMEM lane quadrant w (rows 32 w .. 32 w + 31) and split the columns: in the
+// softmax each takes one 16-column half of every 32-column chunk of S (the
+// two halves combine their row max and sums through shared memory), in the
+// epilogues and the query conversion each takes one half of d.
 #pragma once
 
 #include "common.cuh"
@@ -55,18 +61,21 @@ struct TcPlanes {
   long long plane;  // elements per plane
 };
 
-constexpr int kRtcThreads = 160;      // 4 row warps (TMEM lanes 0-127) + a control warp
+constexpr int kRtcRowThreads = 256;   // 8 row warps: two per TMEM lane quadrant
+constexpr int kRtcThreads = kRtcRowThreads + 32;   // + the control warp (warp 8)
 constexpr int kRtcRows = 128;
 constexpr uint32_t kRBox = 128 * 128; // one [128 rows][128 B] swizzled box
+constexpr size_t kRtcAux = 16 * 8 + 6 * 128 * 4;   // barriers, TMEM slot, softmax exchange
 
 // At least 80 KB so that at most two CTAs (2 x 256 TMEM columns) share an SM.
 template <int D>
 constexpr size_t rtc_smem() {
-  constexpr size_t need = (size_t)3 * (D / 64) * kRBox + 16 * 8;
+  constexpr size_t need = (size_t)3 * (D / 64) * kRBox + kRtcAux;
   return need > 80 * 1024 ? need : 80 * 1024;
 }
 
 // grid (ceil(b1k / G), BH), block kRtcThreads; 1 <= G <= floor(128 / r8).
+// Two CTAs (18 warps, five on some SM sub-partition) leave 96 registers a thread.
 template <typename TQ, int D>
 __global__ void __launch_bounds__(kRtcThreads, 2)
 r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work w, TcPlanes<TQ> out, Geo g,
@@ -88,6 +97,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   uint64_t* bar_v = bar + 6;     // TMA: values
   uint64_t* bar_q = bar + 7;     // row warps: query rows read (first step, bf16, before V lands)
   uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
+  float* sRed = reinterpret_cast<float*>(bar + 16);   // [max | sum p | sum p s][half][row]
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int bh = blockIdx.y;
@@ -99,15 +109,15 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   const int c1_0 = blockIdx.x * G;
   const int Gn = min(G, g.b1k - c1_0);
 
-  if (tid == 128) {
+  if (tid == kRtcRowThreads) {
     ptx::mbar_init(bar_ld, 1);
-    ptx::mbar_init(bar_a, 4);
+    ptx::mbar_init(bar_a, 8);
     ptx::mbar_init(bar_s, 1);
-    ptx::mbar_init(bar_r, 4);
+    ptx::mbar_init(bar_r, 8);
     ptx::mbar_init(bar_acc, 1);
-    ptx::mbar_init(bar_free, 4);
+    ptx::mbar_init(bar_free, 8);
     ptx::mbar_init(bar_v, 1);
-    ptx::mbar_init(bar_q, 4);
+    ptx::mbar_init(bar_q, 8);
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
@@ -145,7 +155,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   };
   auto exact_q = [&](int c1) { return mode == QT_IDENTITY || (mode == QT_KVINIT && c1 >= g.off); };
 
-  if (warp == 4) {
+  if (warp == kRtcRowThreads / 32) {
     if (lane == 0) {
       // ------------------------------------------------ loads and MMA issue
       ptx::prefetch_tmap(&maps.k);
@@ -248,11 +258,13 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     }
   } else {
     // ------------------------------------------------------------- row warps
-    const int r = tid;                          // stacked row = TMEM lane
+    const int qw = warp & 3, half = warp >> 2;  // lane quadrant, column half
+    const int r = 32 * qw + lane;               // stacked row = TMEM lane
     const int gg = r / rs, a2 = r - gg * rs;
     const int c1 = c1_0 + gg;
     const bool valid = gg < Gn && a2 < g.b2;
-    const uint32_t lane_off = (uint32_t)(32 * warp) << 16;
+    const uint32_t lane_off = (uint32_t)(32 * qw) << 16;
+    constexpr int kSeg = NH * 4;                // 16-byte chunks of a row per half
     bool ok = true;
 
     if (mode == QT_KVINIT) {
@@ -261,23 +273,22 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
       if (valid) {
         const bool ex = exact_q(c1);
         const float* qm = w.qbar + ((long long)bh * g.b2 + a2) * D;
-#pragma unroll 1
-        for (int hf = 0; hf < NH; ++hf)
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            uint4 hi4 = make_uint4(0u, 0u, 0u, 0u), lo4 = make_uint4(0u, 0u, 0u, 0u);
-            if (!ex) {
-              const float4 u = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8);
-              const float4 v4 = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8 + 4);
-              tc::split2<TQ>(make_float2(u.x, u.y), hi4.x, lo4.x);
-              tc::split2<TQ>(make_float2(u.z, u.w), hi4.y, lo4.y);
-              tc::split2<TQ>(make_float2(v4.x, v4.y), hi4.z, lo4.z);
-              tc::split2<TQ>(make_float2(v4.z, v4.w), hi4.w, lo4.w);
-            }
-            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
-            if (!ex) *reinterpret_cast<uint4*>(sA + o) = hi4;
-            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = lo4;
+        for (int k = 0; k < kSeg; ++k) {
+          const int i = half * kSeg + k, hf = i >> 3, ch = i & 7;
+          uint4 hi4 = make_uint4(0u, 0u, 0u, 0u), lo4 = make_uint4(0u, 0u, 0u, 0u);
+          if (!ex) {
+            const float4 u = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8);
+            const float4 v4 = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8 + 4);
+            tc::split2<TQ>(make_float2(u.x, u.y), hi4.x, lo4.x);
+            tc::split2<TQ>(make_float2(u.z, u.w), hi4.y, lo4.y);
+            tc::split2<TQ>(make_float2(v4.x, v4.y), hi4.z, lo4.z);
+            tc::split2<TQ>(make_float2(v4.z, v4.w), hi4.w, lo4.w);
           }
+          const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+          if (!ex) *reinterpret_cast<uint4*>(sA + o) = hi4;
+          *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = lo4;
+        }
       }
       ptx::fence_proxy_async();
       __syncwarp();
@@ -291,29 +302,28 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     auto convert_and_store_q = [&]() {
       if (valid && exact_q(c1)) {
         bool over = false;
-#pragma unroll 1
-        for (int hf = 0; hf < NH; ++hf)
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
-            const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
-            uint4 u = *reinterpret_cast<const uint4*>(sA + o);
-            uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
+        for (int k = 0; k < kSeg; ++k) {
+          const int i = half * kSeg + k, hf = i >> 3, ch = i & 7;
+          const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+          uint4 u = *reinterpret_cast<const uint4*>(sA + o);
+          uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              // a finite bf16 of magnitude >= 2^16 (exponent field >= 143) has no f16 value
-              const uint32_t a0 = wv[e] & 0x7FFFu, a1 = (wv[e] >> 16) & 0x7FFFu;
-              over |= (a0 >= 0x4780u && a0 < 0x7F80u) || (a1 >= 0x4780u && a1 < 0x7F80u);
-              const __half2 hv = __floats2half2_rn(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
-              wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
-            }
-            *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
+          for (int e = 0; e < 4; ++e) {
+            // a finite bf16 of magnitude >= 2^16 (exponent field >= 143) has no f16 value
+            const uint32_t a0 = wv[e] & 0x7FFFu, a1 = (wv[e] >> 16) & 0x7FFFu;
+            over |= (a0 >= 0x4780u && a0 < 0x7F80u) || (a1 >= 0x4780u && a1 < 0x7F80u);
+            const __half2 hv = __floats2half2_rn(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
+            wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
+          *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
+        }
         if (over) atomicExch(&ptx::g_device_error, ptx::kErrRange);
       }
       ptx::fence_proxy_async();
       __syncwarp();
       if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
-      ptx::named_bar(1, 128);
+      ptx::named_bar(1, kRtcRowThreads);
       if (tid == 0 && ok) {
         for (int t = 0; t < Gn; ++t) {
           if (!exact_q(c1_0 + t)) continue;
@@ -332,18 +342,19 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     }
 
     // ---- R = softmax over this row's tile columns [cb, cb + b2) of S.  The
-    // rows of a warp need at most three 32-column chunks, from ch_lo on: they
-    // are read from TMEM once and kept in registers.
+    // rows of a quadrant need at most three 32-column chunks, from ch_lo on;
+    // this warp reads the 16-column half c0 of each into registers.
     ok = ptx::mbar_wait(bar_s, 0) && ok;
     ptx::tc_fence_after();
     const int cb = gg * rs;
-    const int wg0 = (32 * warp) / rs, wg1 = min((32 * warp + 31) / rs, G - 1);
+    const int wg0 = (32 * qw) / rs, wg1 = min((32 * qw + 31) / rs, G - 1);
     const int ch_lo = (wg0 * rs) >> 5, ch_hi = min((wg1 * rs + g.b2 - 1) >> 5, 3);
+    const int c0 = 16 * half;
     auto in_tile = [&](int c) { return (unsigned)(c - cb) < (unsigned)g.b2; };
-    uint32_t sv[3][32];
+    uint32_t sv[3][16];
 #pragma unroll
     for (int j = 0; j < 3; ++j)
-      if (ch_lo + j <= ch_hi) ptx::tmem_ld32(tS + lane_off + 32 * (ch_lo + j), sv[j]);
+      if (ch_lo + j <= ch_hi) ptx::tmem_ld16(tS + lane_off + 32 * (ch_lo + j) + c0, sv[j]);
     ptx::tmem_wait_ld();
     // Branch-free: columns outside this row's tile become -inf (p = 0).  The
     // entropy uses sum p s (raw scores, finite everywhere) so that masked
@@ -354,21 +365,27 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     for (int j = 0; j < 3; ++j) {
       if (ch_lo + j > ch_hi) break;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const bool in = in_tile(32 * (ch_lo + j) + i);
+      for (int i = 0; i < 16; ++i) {
+        const bool in = in_tile(32 * (ch_lo + j) + c0 + i);
         const float x = in ? __uint_as_float(sv[j][i]) : -INFINITY;
         sv[j][i] = __float_as_uint(x);
         mq[i & 3] = fmaxf(mq[i & 3], x);
       }
     }
-    const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+    // the two halves' maxima; every S read of the quadrant completes before
+    // either warp writes R over S
+    sRed[half * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+    ptx::tc_fence_before();
+    ptx::named_bar(1, kRtcRowThreads);
+    ptx::tc_fence_after();
+    const float m = fmaxf(sRed[r], sRed[128 + r]);
     const float ms = (m == -INFINITY) ? 0.f : m * g.sl2;   // base-2 units; a row with no column stays 0
     float lq[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       if (ch_lo + j > ch_hi) break;
 #pragma unroll
-      for (int i = 0; i < 32; ++i) {
+      for (int i = 0; i < 16; ++i) {
         const float x = __uint_as_float(sv[j][i]);
         const float p = ptx::ex2(fmaf(x, g.sl2, -ms));
         lq[i & 3] += p;
@@ -376,57 +393,61 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         sv[j][i] = __float_as_uint(p);
       }
     }
-    const float l = (lq[0] + lq[1]) + (lq[2] + lq[3]);
+    sRed[256 + half * 128 + r] = (lq[0] + lq[1]) + (lq[2] + lq[3]);
+    sRed[512 + half * 128 + r] = (pq[0] + pq[1]) + (pq[2] + pq[3]);
+    ptx::named_bar(1, kRtcRowThreads);
+    const float l = sRed[256 + r] + sRed[384 + r];
     // sum p (x s2 - ms) with x the raw score
-    const float xe = g.sl2 * ((pq[0] + pq[1]) + (pq[2] + pq[3])) - ms * l;
+    const float xe = g.sl2 * (sRed[512 + r] + sRed[640 + r]) - ms * l;
     const float inv = 1.f / l;
     const float2 inv2 = make_float2(inv, inv);
-    // R over S: chunk ch -> columns [32 ch, 32 ch + 16) hi, [32 ch + 16, 32 ch + 32) lo
+    // R over S: chunk ch -> columns [32 ch, 32 ch + 16) hi, [32 ch + 16, 32 ch + 32) lo;
+    // this warp's 16 keys are the 8 hi and 8 lo columns at offset c0 / 2
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       if (ch_lo + j > ch_hi) continue;
-      uint32_t hi[16], lo[16];
+      uint32_t hi[8], lo[8];
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
+      for (int i = 0; i < 8; ++i)
         tc::split2<TQ>(tc::mul2(make_float2(__uint_as_float(sv[j][2 * i]), __uint_as_float(sv[j][2 * i + 1])), inv2),
                        hi[i], lo[i]);
-      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j), hi);
-      ptx::tmem_st16(tS + lane_off + 32 * (ch_lo + j) + 16, lo);
+      ptx::tmem_st8(tS + lane_off + 32 * (ch_lo + j) + c0 / 2, hi);
+      ptx::tmem_st8(tS + lane_off + 32 * (ch_lo + j) + 16 + c0 / 2, lo);
     }
     {
+      // chunks no row of the quadrant uses: this warp zeroes 16 of their 32 columns
       uint32_t zero[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) zero[i] = 0u;
       for (int ch = 0; ch < 4; ++ch)
-        if (ch < ch_lo || ch > ch_hi) {
-          ptx::tmem_st16(tS + lane_off + 32 * ch, zero);
-          ptx::tmem_st16(tS + lane_off + 32 * ch + 16, zero);
-        }
+        if (ch < ch_lo || ch > ch_hi) ptx::tmem_st16(tS + lane_off + 32 * ch + c0, zero);
     }
     ptx::tmem_wait_st();
     ptx::tc_fence_before();
     __syncwarp();
     if (lane == 0) ptx::mbar_arrive(bar_r);
     // h in bits: -sum R log2 R = log2 l - sum R (x - m)
-    if (valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
+    if (half == 0 && valid && ok) w.h[((long long)bh * g.b2 + a2) * g.b1k_pad + c1] = log2f(l) - xe * inv;
     if (bf16 && mode == QT_KVINIT) convert_and_store_q();
-    // ---- epilogue: a row of k~ (or z) from TMEM, split into hi / lo planes,
-    // staged in two swizzled [d half][128 rows][128 B] regions
+    // ---- epilogue: this warp's half of a row of k~ (or z) from TMEM, split
+    // into hi / lo planes, staged in two swizzled [d half][128 rows][128 B]
+    // regions
     auto stage_row = [&](uint8_t* shi, uint8_t* slo, auto tag) {
       using TP = decltype(tag);
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t a[32];
-        ptx::tmem_ld32(tAcc + lane_off + 32 * cc, a);
+      for (int k = 0; k < D / 32; ++k) {
+        const int cc = half * (D / 32) + k;   // 16-column group of the accumulator
+        uint32_t a[16];
+        ptx::tmem_ld16(tAcc + lane_off + 16 * cc, a);
         ptx::tmem_wait_ld();
-        uint32_t hi[16], lo[16];
+        uint32_t hi[8], lo[8];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 8; ++i)
           tc::split2<TP>(make_float2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), hi[i], lo[i]);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const int ch8 = (cc & 1) * 4 + v;
-          const uint32_t o = (cc >> 1) * kRBox + r * 128 + ((ch8 ^ (r & 7)) << 4);
+        for (int v = 0; v < 2; ++v) {
+          const int ch8 = (cc & 3) * 2 + v;
+          const uint32_t o = (cc >> 2) * kRBox + r * 128 + ((ch8 ^ (r & 7)) << 4);
           *reinterpret_cast<uint4*>(shi + o) = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
           *reinterpret_cast<uint4*>(slo + o) = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
         }
@@ -446,24 +467,24 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     ptx::tc_fence_after();
     if (bf16 && mode != QT_BUFFER) {
       if (tid == 0) ptx::bulk_wait_read();   // the q copy has read the A lo plane
-      ptx::named_bar(1, 128);
+      ptx::named_bar(1, kRtcRowThreads);
     }
     // k~ (f16 planes): hi plane staged over the A lo plane, lo plane over K
     // (both read by now: S and k~ are complete)
     stage_row(sA + NH * kRBox, sK, __half{});
     ptx::tc_fence_before();
-    ptx::named_bar(1, 128);
+    ptx::named_bar(1, kRtcRowThreads);
     if (final_step && lane == 0) ptx::mbar_arrive(bar_free);   // TMEM accumulator read out
     if (tid == 0 && ok) store_tiles(&maps.kt, sA + NH * kRBox, sK);
     if (final_step) {
       ok = ok && ptx::mbar_wait(bar_acc, 1);
       ptx::tc_fence_after();
       if (tid == 0) ptx::bulk_wait_read();   // the k~ stores have read their staging
-      ptx::named_bar(1, 128);
+      ptx::named_bar(1, kRtcRowThreads);
       // z: hi plane over the A hi plane (V is consumed), lo over the A lo plane
       stage_row(sA, sA + NH * kRBox, __half{});
       ptx::tc_fence_before();
-      ptx::named_bar(1, 128);
+      ptx::named_bar(1, kRtcRowThreads);
       if (tid == 0 && ok) store_tiles(&maps.z, sA, sA + NH * kRBox);
     }
     if (tid == 0) ptx::bulk_wait_read();
