@@ -431,19 +431,29 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     if (bf16 && mode == QT_KVINIT) convert_and_store_q();
     // ---- epilogue: this warp's half of a row of k~ (or z) from TMEM, split
     // into hi / lo planes, staged in two swizzled [d half][128 rows][128 B]
-    // regions
-    auto stage_row = [&](uint8_t* shi, uint8_t* slo, auto tag) {
-      using TP = decltype(tag);
+    // regions.  The next 16-column group is read while the current one is
+    // converted; with release set, the warp hands the accumulator back to the
+    // MMA warp (bar_free) once its last read has landed.
+    auto stage_row = [&](uint8_t* shi, uint8_t* slo, bool release) {
+      constexpr int NG = D / 32;   // 16-column groups per half
+      uint32_t a[2][16];
+      ptx::tmem_ld16(tAcc + lane_off + 16 * (half * NG), a[0]);
 #pragma unroll
-      for (int k = 0; k < D / 32; ++k) {
-        const int cc = half * (D / 32) + k;   // 16-column group of the accumulator
-        uint32_t a[16];
-        ptx::tmem_ld16(tAcc + lane_off + 16 * cc, a);
+      for (int k = 0; k < NG; ++k) {
+        const int cc = half * NG + k;   // 16-column group of the accumulator
         ptx::tmem_wait_ld();
+        if (k + 1 < NG) {
+          ptx::tmem_ld16(tAcc + lane_off + 16 * (cc + 1), a[(k + 1) & 1]);
+        } else if (release) {
+          ptx::tc_fence_before();
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(bar_free);
+        }
         uint32_t hi[8], lo[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i)
-          tc::split2<TP>(make_float2(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), hi[i], lo[i]);
+          tc::split2<__half>(make_float2(__uint_as_float(a[k & 1][2 * i]), __uint_as_float(a[k & 1][2 * i + 1])),
+                             hi[i], lo[i]);
 #pragma unroll
         for (int v = 0; v < 2; ++v) {
           const int ch8 = (cc & 3) * 2 + v;
@@ -471,10 +481,8 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     }
     // k~ (f16 planes): hi plane staged over the A lo plane, lo plane over K
     // (both read by now: S and k~ are complete)
-    stage_row(sA + NH * kRBox, sK, __half{});
-    ptx::tc_fence_before();
+    stage_row(sA + NH * kRBox, sK, final_step != 0);
     ptx::named_bar(1, kRtcRowThreads);
-    if (final_step && lane == 0) ptx::mbar_arrive(bar_free);   // TMEM accumulator read out
     if (tid == 0 && ok) store_tiles(&maps.kt, sA + NH * kRBox, sK);
     if (final_step) {
       ok = ok && ptx::mbar_wait(bar_acc, 1);
@@ -482,8 +490,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
       if (tid == 0) ptx::bulk_wait_read();   // the k~ stores have read their staging
       ptx::named_bar(1, kRtcRowThreads);
       // z: hi plane over the A hi plane (V is consumed), lo over the A lo plane
-      stage_row(sA, sA + NH * kRBox, __half{});
-      ptx::tc_fence_before();
+      stage_row(sA, sA + NH * kRBox, false);
       ptx::named_bar(1, kRtcRowThreads);
       if (tid == 0 && ok) store_tiles(&maps.z, sA, sA + NH * kRBox);
     }
