@@ -43,7 +43,7 @@ L2_BYTES = 126 * 2**20
 # a kernel without a capture of its current code reports null.
 NCU_TRAFFIC = {
     ("full_32760_bf16", "l_col"): 877.8e6,   # 292.6 MB at 8 heads x 3
-    ("chunk_4680_bf16", "r_step"): 48.5e6,   # mean of the call's two launches (30.4 and 66.6 MB)
+    ("chunk_4680_bf16", "r_step"): 48.2e6,   # mean of the call's two launches (30.2 and 66.2 MB)
 }
 # FP32 FMA ceiling of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
