@@ -244,8 +244,8 @@ l_bwd_dkv_simt(const T* __restrict__ q, const TG* __restrict__ dy, Work w, BwdWo
 // of the tile's tokens in grid order.  Positions are padded with zero rows to
 // P4 = b2 rounded up to 4; shared rows of k, v, q, dk~, dz hold D + 4 floats
 // and rows of R and dSr P4 floats, so that every shared access is a float4.
-// The contractions run in register blocks: 2 x 2 (a2, c2) for the scores and
-// G, 4 positions x 4 channels for dk/dv and for dq.
+// The contractions run in register blocks: 4 x 4 (a2, c2) over a slice of the
+// channels for the scores and G, 4 positions x 4 channels for dk/dv and for dq.
 // grid (b1k, BH), block 256, dynamic smem r_bwd_smem_bytes(b2, D).
 __host__ __device__ constexpr int r_bwd_p4(int b2) { return (b2 + 3) & ~3; }
 __host__ __device__ constexpr size_t r_bwd_smem_bytes(int b2, int d) {
@@ -332,40 +332,76 @@ r_bwd_simt(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict
   }
   __syncthreads();
 
-  // scores (base 2) and G = dk~ k^T + dz v^T in 2 x 2 blocks of (a2, c2):
-  // rows {a, a + nb} and columns {c, c + nb}, so that neighbouring threads read
-  // neighbouring rows (D + 4 floats apart: distinct banks for float4 loads)
-  const int nb = P4 / 2;
-  for (int blk = threadIdx.x; blk < nb * nb; blk += blockDim.x) {
-    const int a = blk / nb, c = blk % nb;
-    float sc[2][2] = {}, gg[2][2] = {};
-#pragma unroll 4
-    for (int cc = 0; cc < D; cc += 4) {
-      float4 qa[2], ka[2], za[2], kc[2], vc[2];
+  // scores (base 2) and G = dk~ k^T + dz v^T in 4 x 4 blocks of (a2, c2): rows
+  // {a + i nb} and columns {c + j nb}.  The channels are split into ds slices
+  // (ds lanes per block, ds a power of two chosen to fill the CTA) whose
+  // partial sums are added by shuffles.  Slice sl reads float4 columns
+  // sl w + (u mod w) + 8 (u / w), w = 8 / ds, at step u: the 8 lanes of one
+  // shared-memory phase (8 / ds blocks of neighbouring c, rows D + 4 floats
+  // apart) then touch 8 distinct bank groups.
+  {
+    const int nb = P4 / 4, nblk = nb * nb;
+    int ds = 1;
+    while (ds < 8 && nblk * ds * 2 <= (int)blockDim.x) ds *= 2;
+    const int w = 8 / ds, cs = C4 / ds, items = nblk * ds;
+    const int lane = threadIdx.x & 31;
+    // whole warps iterate together (the shuffles need every lane); a block's
+    // ds lanes are all valid or all idle, since ds divides 32
+    for (int base = threadIdx.x & ~31; base < items; base += blockDim.x) {
+      const int item = base + lane;
+      const bool live = item < items;
+      const int blk = live ? item / ds : 0, sl = item & (ds - 1);
+      const int a = blk / nb, c = blk - a * nb;
+      float sc[4][4], gg[4][4];
 #pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        qa[i] = *reinterpret_cast<const float4*>(sQ + (a + i * nb) * DP + cc);
-        ka[i] = *reinterpret_cast<const float4*>(sDK + (a + i * nb) * DP + cc);
-        za[i] = *reinterpret_cast<const float4*>(sDZ + (a + i * nb) * DP + cc);
-        kc[i] = *reinterpret_cast<const float4*>(sK + (c + i * nb) * DP + cc);
-        vc[i] = *reinterpret_cast<const float4*>(sV + (c + i * nb) * DP + cc);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[i][j] = gg[i][j] = 0.f;
+#pragma unroll 1
+      for (int u = 0; u < cs; ++u) {
+        const int cc = 4 * (sl * w + (u % w) + 8 * (u / w));
+        float4 kc[4], x[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kc[j] = *reinterpret_cast<const float4*>(sK + (c + j * nb) * DP + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const float4*>(sQ + (a + i * nb) * DP + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sc[i][j] = dot4(x[i], kc[j], sc[i][j]);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const float4*>(sDK + (a + i * nb) * DP + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) gg[i][j] = dot4(x[i], kc[j], gg[i][j]);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) kc[j] = *reinterpret_cast<const float4*>(sV + (c + j * nb) * DP + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) x[i] = *reinterpret_cast<const float4*>(sDZ + (a + i * nb) * DP + cc);
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) gg[i][j] = dot4(x[i], kc[j], gg[i][j]);
       }
+      for (int o = 1; o < ds; o <<= 1)
 #pragma unroll
-      for (int i = 0; i < 2; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          sc[i][j] = dot4(qa[i], kc[j], sc[i][j]);
-          gg[i][j] = dot4(za[i], vc[j], dot4(ka[i], kc[j], gg[i][j]));
-        }
+          for (int j = 0; j < 4; ++j) {
+            sc[i][j] += __shfl_xor_sync(0xffffffffu, sc[i][j], o);
+            gg[i][j] += __shfl_xor_sync(0xffffffffu, gg[i][j], o);
+          }
+      // lane sl of the block writes the entries e = 4 i + j with e mod ds = sl
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (live && ((4 * i + j) & (ds - 1)) == sl && a + i * nb < b2 && c + j * nb < b2) {
+            sR[(a + i * nb) * P4 + c + j * nb] = sc[i][j] * g.sl2;
+            sG[(a + i * nb) * P4 + c + j * nb] = gg[i][j];
+          }
     }
-#pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-        if (a + i * nb < b2 && c + j * nb < b2) {
-          sR[(a + i * nb) * P4 + c + j * nb] = sc[i][j] * g.sl2;
-          sG[(a + i * nb) * P4 + c + j * nb] = gg[i][j];
-        }
   }
   __syncthreads();
 
