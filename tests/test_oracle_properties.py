@@ -12,6 +12,10 @@ steps, head dimension) and the same facts must hold on every draw:
   * with scores separable across the two Monarch axes the output is the
     (masked) dense softmax attention, the case the aligned blocks represent
     exactly.
+The backward of the one-step forward (self-attention, optional mask) must
+match central finite differences of the forward in random directions, and
+keep the two exact invariants of a row-stochastic operator: sum_keys dv =
+sum_queries dy, and sum_keys dk = 0.
 Draws are derandomised, so the CPU suite sees the same cases on every run.
 Planted mistakes (positions reversed inside every tile, a missing beta
 normalisation) fail one of the two properties on a fixed masked KV grid.
@@ -115,3 +119,32 @@ def test_missing_beta_normalisation_fails_the_separable_case(monkeypatch):
 def test_unmutated_oracle_passes_the_planted_cases():
     _check_factored(_MASKED_KV, 2, 3, seed=5)
     _check_separable(_MASKED_KV, 2, seed=5)
+
+
+@st.composite
+def self_grids(draw):
+    g = draw(grids())
+    return om.Grid(g.T, g.H, g.W, g.th, g.tw, chunk_frames=g.chunk_frames)
+
+
+@settings(max_examples=30, deadline=None, derandomize=True)
+@given(g=self_grids(), d=st.sampled_from([2, 3, 5]), seed=st.integers(0, 2**16))
+def test_backward_matches_finite_differences_on_random_grids(g, d, seed):
+    rng = np.random.default_rng(seed)
+    q, k, v, dy = (rng.standard_normal((1, 1, g.Nq, d)) for _ in range(4))
+    grads = dict(zip("qkv", om.monarch_attention_backward(q, k, v, dy, g)))
+    eps = 1e-6
+    for which in "qkv":
+        delta = rng.standard_normal(q.shape)
+
+        def f(x):
+            args = {"q": q, "k": k, "v": v, which: x}
+            return float((om.monarch_attention(args["q"], args["k"], args["v"], g, 1) * dy).sum())
+        x = {"q": q, "k": k, "v": v}[which]
+        fd = (f(x + eps * delta) - f(x - eps * delta)) / (2 * eps)
+        an = float((grads[which] * delta).sum())
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(fd)), (which, fd, an)
+    # a row-stochastic operator: dv = M^T dy keeps the column sums of dy; the
+    # scores enter through softmaxes, whose gradients sum to zero over keys
+    np.testing.assert_allclose(grads["v"].sum(axis=2), dy.sum(axis=2), atol=1e-10, rtol=0)
+    assert np.abs(grads["k"].sum(axis=2)).max() <= 1e-10 * max(1.0, np.abs(grads["k"]).sum(axis=2).max())
