@@ -43,6 +43,53 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(_declared_functions()) == set(m._SIGS)
 
 
+def _c_kind(decl: str):
+    """(kind, bytes) of a C type: pointers (and the opaque stream handle) are
+    ("ptr", 8); integers carry their sign and width."""
+    t = " ".join(re.sub(r"\bconst\b", "", decl).split())
+    if "*" in t or t == "cudaStream_t":
+        return ("ptr", 8)
+    return {"int": ("int", 4), "long": ("int", 8), "size_t": ("uint", 8), "unsigned long long": ("uint", 8),
+            "unsigned": ("uint", 4), "void": ("void", 0)}[t]
+
+
+def _param_type(p: str) -> str:
+    """The type of one named parameter; an array parameter decays to a pointer."""
+    m_ = re.match(r"^(.*?[\s\*])(\w+)\s*(\[[^\]]*\])?$", p.strip())
+    assert m_, p
+    return m_.group(1).strip() + ("*" if m_.group(3) else "")
+
+
+def _ctypes_kind(t):
+    if t is None:
+        return ("void", 0)
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or (isinstance(t, type) and issubclass(t, ctypes._Pointer)):
+        return ("ptr", 8)
+    return ("int" if t(-1).value < 0 else "uint", ctypes.sizeof(t))
+
+
+def _prototypes():
+    src = open(os.path.join(ROOT, "include", "monarch_attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    out = {}
+    for ret, name, params in re.findall(r"^([A-Za-z_][\w \t\*]*?)\b(monarch_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.M):
+        plist = [p.strip() for p in params.split(",") if p.strip() and p.strip() != "void"]
+        out[name] = (ret.strip(), plist)
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    protos = _prototypes()
+    assert set(protos) == set(m._SIGS)
+    for name, (ret, params) in protos.items():
+        res, args = m._SIGS[name]
+        assert _ctypes_kind(res) == _c_kind(ret), (name, ret, res)
+        assert len(args) == len(params), (name, len(args), len(params))
+        for i, (a, p) in enumerate(zip(args, params)):
+            assert _ctypes_kind(a) == _c_kind(_param_type(p)), (name, i, p, a)
+
+
 def test_version(lib):
     assert lib.monarch_attn_version() >= 102
 
