@@ -28,6 +28,8 @@ using namespace monarch;
 
 namespace {
 
+constexpr int kMaxDevices = 64;   // device ordinals with per-device state
+
 thread_local std::string g_err;
 
 int fail(int code, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
@@ -262,6 +264,20 @@ cudaError_t allow_smem(K kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
+// Runs `set` (a call site's shared-memory limits) once per device: a function
+// attribute belongs to the current device's context.  Ordinals outside the
+// table are set on every call.
+template <typename F>
+cudaError_t once_per_device(std::atomic<bool> (&done)[kMaxDevices], F&& set) {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool cached = dev >= 0 && dev < kMaxDevices;
+  if (cached && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  const cudaError_t e = set();
+  if (e == cudaSuccess && cached) done[dev].store(true, std::memory_order_release);
+  return e;
+}
+
 // Key tiles per R-step CTA.  At most floor(128 / r8) fit the 128 MMA rows;
 // fewer give more, shorter CTAs.  Two CTAs run per SM, so the launch takes
 // ceil(CTAs / (2 * SMs)) rounds of CTAs whose time grows with G plus a fixed
@@ -286,16 +302,17 @@ int r_step_group(const Geo& g, int sm_count) {
 }
 
 int sm_count_of_device() {
-  static int n[64] = {};
+  static std::atomic<int> n[kMaxDevices];
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) return 148;
-  if (!n[dev]) {
-    int v = 0;
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  int v = n[dev].load(std::memory_order_relaxed);
+  if (!v) {
     cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
-    n[dev] = v > 0 ? v : 1;
+    if (v <= 0) v = 1;
+    n[dev].store(v, std::memory_order_relaxed);
   }
-  return n[dev];
+  return v;
 }
 
 // Workspace views and tensor maps of the tensor-core forward (shared by the
@@ -383,25 +400,22 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   constexpr size_t smem_col = tc::col_smem<D>();
   constexpr size_t smem_r = rtc_smem<D>();
 
-  static bool attrs_set = false;
-  if (!attrs_set) {
-    cudaError_t e;
-    if ((e = allow_smem(tc::l_lse<D>, smem_lse)) != cudaSuccess ||
-        (e = allow_smem(tc::l_row<__half, TO, D, true>, smem_out)) != cudaSuccess ||
-        (e = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
-      return cuda_fail(e, "cudaFuncSetAttribute");
-    attrs_set = true;
+  static std::atomic<bool> attrs_set[kMaxDevices];
+  {
+    const cudaError_t e = once_per_device(attrs_set, [&] {
+      cudaError_t r;
+      if ((r = allow_smem(tc::l_lse<D>, smem_lse)) != cudaSuccess ||
+          (r = allow_smem(tc::l_row<__half, TO, D, true>, smem_out)) != cudaSuccess ||
+          (r = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
+          (r = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
+        return r;
+      return cudaSuccess;
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);  // two 128-row tiles per CTA
   // persistent column pass: one CTA per SM over (head, position, 256 key tiles) items
-  static int sm_count = 0;
-  if (!sm_count) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&sm_count, cudaDevAttrMultiProcessorCount, dev);
-    if (sm_count <= 0) sm_count = 1;
-  }
+  const int sm_count = sm_count_of_device();
   const long long col_items = (long long)g.BH * g.b2 * ((g.b1k + 2 * kTile - 1) / (2 * kTile));
   const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
   const int r_group = r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
@@ -664,16 +678,19 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   constexpr size_t smem_q = tcb::q_smem<D>();
   static_assert(smem_kv <= (size_t)tc::kMaxSmem && smem_q <= (size_t)tc::kMaxSmem, "backward shared memory");
   const size_t rb_smem = r_bwd_smem_bytes(g.b2, D);
-  static bool attrs_set = false;
-  if (!attrs_set) {
-    cudaError_t e;
-    if ((e = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess ||
-        (e = allow_smem(tcb::l_bwd_kv<D>, smem_kv)) != cudaSuccess ||
-        (e = allow_smem(tcb::l_bwd_q<D>, smem_q)) != cudaSuccess ||
-        (e = allow_smem(r_bwd_simt<TQ, TG, D>, r_bwd_smem_bytes(kMaxB2, D))) != cudaSuccess)
-      return cuda_fail(e, "cudaFuncSetAttribute");
-    attrs_set = true;
+  static std::atomic<bool> attrs_set[kMaxDevices];
+  {
+    const cudaError_t e = once_per_device(attrs_set, [&] {
+      cudaError_t r;
+      if ((r = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
+          (r = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess ||
+          (r = allow_smem(tcb::l_bwd_kv<D>, smem_kv)) != cudaSuccess ||
+          (r = allow_smem(tcb::l_bwd_q<D>, smem_q)) != cudaSuccess ||
+          (r = allow_smem(r_bwd_simt<TQ, TG, D>, r_bwd_smem_bytes(kMaxB2, D))) != cudaSuccess)
+        return r;
+      return cudaSuccess;
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
   const int r_group = r_step_group(g, sm_count_of_device());
@@ -737,13 +754,16 @@ int run_fwd_train_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, float
   if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_r = rtc_smem<D>();
-  static bool attrs_set = false;
-  if (!attrs_set) {
-    cudaError_t e;
-    if ((e = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
-        (e = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
-      return cuda_fail(e, "cudaFuncSetAttribute");
-    attrs_set = true;
+  static std::atomic<bool> attrs_set[kMaxDevices];
+  {
+    const cudaError_t e = once_per_device(attrs_set, [&] {
+      cudaError_t r;
+      if ((r = allow_smem(tc::l_row<__half, float, D, true, true>, smem_out)) != cudaSuccess ||
+          (r = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
+        return r;
+      return cudaSuccess;
+    });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
   const int r_group = r_step_group(g, sm_count_of_device());
@@ -817,11 +837,11 @@ int dispatch_bwd(const BwdPlan& bp, const void* q, const void* k, const void* v,
 // it without returning memory to the driver between calls.
 int workspace_pool(cudaMemPool_t* out) {
   static std::mutex mu;
-  static cudaMemPool_t pools[64] = {};
+  static cudaMemPool_t pools[kMaxDevices] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  if (dev < 0 || dev >= kMaxDevices) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
   std::lock_guard<std::mutex> lk(mu);
   if (!pools[dev]) {
     cudaMemPoolProps props = {};
@@ -850,15 +870,15 @@ struct HostStreams {
 
 // One host-buffer call at a time per device: the call holds this lock until
 // its copies are done, since the events above are shared.
-std::mutex g_host_call_mu[64];
+std::mutex g_host_call_mu[kMaxDevices];
 
 int host_streams(HostStreams* hs, int* dev_out) {
   static std::mutex mu;
-  static HostStreams per_dev[64];
+  static HostStreams per_dev[kMaxDevices];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= 64) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
+  if (dev < 0 || dev >= kMaxDevices) return fail(MONARCH_EUNSUPPORTED, "device ordinal %d out of range", dev);
   std::lock_guard<std::mutex> lk(mu);
   HostStreams& s = per_dev[dev];
   if (!s.in) {
@@ -1213,7 +1233,6 @@ constexpr size_t kNoAllocScratchBytes = size_t(128) << 20;  // 128 MiB per devic
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-constexpr int kMaxDevices = 64;
 std::mutex g_scratch_mu;
 void* g_scratch_ptr[kMaxDevices] = {};
 
