@@ -48,6 +48,17 @@ maximiser over row-stochastic M is softmax(S)); this is what the tests pin.
 
 Everything here is fp64 numpy; ``np.matmul`` is the only library primitive
 used as a step.  Loops run over (batch, head) so memory stays one head deep.
+
+How it is pinned (tests/test_oracle_pins.py, test_oracle_properties.py,
+test_oracle_mutations.py, test_oracle_backward.py): the grid -> block map
+against a hand-written table; the factored output against M materialised
+entry by entry from token coordinates (non-negative, row-stochastic, zero
+outside the mask), on fixed and on randomly drawn tiny grids; separable
+scores and the one-position or one-tile grids against dense softmax
+attention; each block update against random feasible perturbations of F; the
+backward against central finite differences of the forward and two exact
+invariants.  For generic inputs no printed value exists, so the output values
+are pinned through these properties only, not against a worked example.
 """
 
 from __future__ import annotations
