@@ -94,11 +94,30 @@ def work_model(w):
         "l_out": dict(flops=BH * 2 * FL, bytes=nq + 2 * nk + hb + no),   # q, k~, z, h -> out
         "l_lse": dict(flops=BH * FL, bytes=nq + nk + hb + lse),          # q, k~, h -> lse
         "l_col": dict(flops=BH * FL, bytes=nq + nk + hb + lse + nk),     # q, k~, h, lse -> q~
-        "r_step": dict(flops=BH * 2 * FR, bytes=3 * nk),                 # q~, k -> k~ (final: +v, z)
+        # q~ (or q), k in and k~ out, plus v in and z out in the final
+        # launch; h out every launch.  Mean over the call's `iters` launches.
+        "r_step": dict(flops=BH * (2 * w.iters + 1) * FR / w.iters,
+                       bytes=(3 * (w.iters - 1) * nk + 5 * nk) / w.iters + hb),
         "qbar": dict(flops=0.0, bytes=nq),
     }
-    return dict(flops=flops_total, io_bytes=nq + 2 * nk + no, dense_flops=4.0 * BH * w.Nq * w.Nk * w.d * fv,
+    # compulsory call bytes: Q, K, V in and O out, all in the input dtype
+    # (the output is written as f32 by default, which adds nq bytes; the
+    # roofline keeps the smaller count)
+    return dict(flops=flops_total, io_bytes=2 * nq + 2 * nk, io_bytes_f32_out=nq + 2 * nk + no,
+                dense_flops=4.0 * BH * w.Nq * w.Nk * w.d * fv,
                 phases=phases, FL=FL, FR=FR, visible_fraction=fv)
+
+
+def call_roofline(w, model, peaks, ms):
+    """Whole-call roofline: the slower of the Monarch FLOPs at the measured
+    bf16 tensor peak and the compulsory Q/K/V/O bytes at the measured HBM
+    bandwidth; frac = that time / the measured time."""
+    t_flop = model["flops"] / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = model["io_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    roof_ms = 1e3 * max(t_flop, t_hbm)
+    return {"roofline_ms": roof_ms, "frac": roof_ms / ms, "bound": "tensor" if t_flop >= t_hbm else "hbm",
+            "flop_ms": 1e3 * t_flop, "hbm_ms": 1e3 * t_hbm, "io_bytes": model["io_bytes"],
+            "peak_source": peaks["source"]}
 
 
 def backward_work_model(w):
@@ -200,52 +219,117 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
 
 
 # ---------------------------------------------------------------------------
+_INPUT_CACHE = {}
+
+
+def inputs_of(w):
+    """Seeded inputs of a workload; workloads that differ only in name,
+    iterations or mask share one draw."""
+    key = (w.B, w.heads, w.T, w.H, w.W, w.d, w.dtype, w.seed, w.kind, w.Tk, w.planted)
+    if key not in _INPUT_CACHE:
+        _INPUT_CACHE.clear()
+        _INPUT_CACHE[key] = make_inputs(w)
+    return _INPUT_CACHE[key]
+
+
+def time_forward(m, w, qd, kd, vd, out, steps, warmup, stream, flush, world=1, clocks=None):
+    """Per-step device times (ms) of `steps` forward calls after `warmup`
+    untimed ones, each bracketed by CUDA events on the launching stream, with
+    an L2 flush before every call when `flush` is given.  Returns the list and
+    the number of library kernels launched in the timed region."""
+    def step():
+        m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters, stream=stream,
+                           chunk_frames=w.chunk_frames)
+
+    for _ in range(warmup):
+        if flush is not None:
+            flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = m.launch_count()
+    if clocks:
+        clocks.begin()
+    for i in range(steps):
+        if flush is not None:
+            flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if clocks:
+        clocks.end()
+    launches = m.launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    return [a.elapsed_time(b) for a, b in zip(starts, ends)], launches, step
+
+
+# Every configuration the headline metric covers (N = 4680 to 32760), timed in
+# the same run as the headline: the toy, the KV-cache step, the shape sweep, the
+# full sequence, and the one-step and chunk-causal training forms (the three
+# full-sequence workloads share one input draw, so they run back to back).
+EXTRA_WORKLOADS = ["toy_256_f32", "kvcache_4680x32760_bf16", "sweep_2048_f16", "sweep_8192_f16",
+                   "sweep_32768_f16", "chunk_4680_bf16_1step", "full_32760_bf16", "full_32760_bf16_1step",
+                   "train_32760_bf16_causal"]
+
+
+def extra_configs(m, args, device, stream, flush_buf, peaks, world):
+    """ms per call (median of CUDA-event-timed steps), effective TFLOP/s and
+    the whole-call roofline fraction of every other configuration, with dense
+    SDPA on the same tensors as context."""
+    res = {}
+    for name in EXTRA_WORKLOADS:
+        if name == args.workload:
+            continue
+        w = WORKLOADS[name]
+        model = work_model(w)
+        q, k, v = inputs_of(w)
+        qd, kd, vd = (t.to(device) for t in (q, k, v))
+        out = torch.empty(qd.shape, dtype=torch.float32, device=device)
+        flush = flush_buf if model["io_bytes"] < 4 * L2_BYTES else None
+        steps = max(5, min(args.steps, 20 if model["flops"] > 5e11 else 50))
+        times, _, _ = time_forward(m, w, qd, kd, vd, out, steps, args.warmup, stream, flush, world)
+        ms = max_over_ranks(statistics.median(times), world, device)
+        rec = {"ms_per_call": ms, "mean_ms": statistics.fmean(times), "steps": steps,
+               "value": world * model["flops"] / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "monarch_gflop_per_call": model["flops"] / 1e9, "dtype": w.dtype,
+               "config": {"B": w.B, "heads": w.heads, "grid": [w.T, w.H, w.W], "kv_frames": w.Tkey,
+                          "head_dim": w.d, "tile": [w.th, w.tw], "iters": w.iters,
+                          "chunk_frames": w.chunk_frames},
+               "call_roofline": call_roofline(w, model, peaks, ms),
+               "l2": "flushed between steps" if flush is not None else "inputs larger than L2"}
+        rec["dense_context"] = dense_context(qd, kd, vd, model, flush, stream, ms)
+        res[name] = rec
+        del qd, kd, vd, out
+        torch.cuda.empty_cache()
+    return res
+
+
 def run_ours(args, rank, world, device):
     import structured_sparse_attention_grid_b200 as m
     w = WORKLOADS[args.workload]
     model = work_model(w)
     peaks = load_peaks()
-    q, k, v = make_inputs(w)
+    q, k, v = inputs_of(w)
     qd, kd, vd = (t.to(device) for t in (q, k, v))
-    out = torch.empty(qd.shape, dtype=torch.float32, device=device)  # f32 output: see DESIGN
+    out = torch.empty(qd.shape, dtype=torch.float32, device=device)  # the library's default f32 output
     stream = torch.cuda.current_stream(device)
     io_bytes = model["io_bytes"]
-    flush = torch.empty(int(2 * L2_BYTES), dtype=torch.uint8, device=device)
+    flush_buf = torch.empty(int(2 * L2_BYTES), dtype=torch.uint8, device=device)
     flush_l2 = io_bytes < 4 * L2_BYTES  # inputs smaller than ~4x L2: flush between steps
-
-    def step():
-        m.monarch_attn_fwd(qd, kd, vd, out, w.T, w.H, w.W, w.th, w.tw, w.iters, stream=stream,
-                           chunk_frames=w.chunk_frames)
-
-    for _ in range(args.warmup):
-        if flush_l2:
-            flush.zero_()
-        step()
-    torch.cuda.synchronize(device)
+    flush = flush_buf if flush_l2 else None
 
     clocks = ClockSampler(torch.cuda.current_device() if device.index is None else device.index)
     clocks.start()
     time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize(device)
-    launches0 = m.launch_count()
-    clocks.begin()
-    for i in range(args.steps):
-        if flush_l2:
-            flush.zero_()
-        starts[i].record(stream)
-        step()
-        ends[i].record(stream)
-    torch.cuda.synchronize(device)
-    clocks.end()
-    launches = m.launch_count() - launches0
-    if world > 1:
-        torch.distributed.barrier()
-    per_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    ms = sum(per_step) / len(per_step)
+    per_step, launches, step = time_forward(m, w, qd, kd, vd, out, args.steps, args.warmup, stream, flush,
+                                            world, clocks)
+    ms = statistics.median(per_step)
     # If the timed steps were short, keep sampling clocks for a moment under load.
     if sum(per_step) < 1000.0:
         t_end = time.time() + 1.0
@@ -256,6 +340,7 @@ def run_ours(args, rank, world, device):
     clocks.stop()
 
     ms = max_over_ranks(ms, world, device)
+    mean_ms = max_over_ranks(statistics.fmean(per_step), world, device)
 
     # Per-kernel times: the same step, with CUDA events around every launch.
     m.profile_enable(True)
@@ -263,7 +348,7 @@ def run_ours(args, rank, world, device):
     nprof = max(3, min(args.steps, 20))
     for _ in range(nprof):
         if flush_l2:
-            flush.zero_()
+            flush_buf.zero_()
         step()
     torch.cuda.synchronize(device)
     prof = m.profile_read(reset=True)
@@ -284,11 +369,11 @@ def run_ours(args, rank, world, device):
     roof["traffic_unit"] = "bytes per launch (ncu DRAM read + write)"
     roof["kernel"] = dom
     roof["launch_ms"] = dom_ms
+    roof["algorithmic_per_launch"] = ph["bytes"] if roof["bound"] == "hbm" else ph["flops"]
     roof["peak_source"] = peaks["source"]
 
-    call_roof_ms = 1e3 * max(model["flops"] / (peaks["bf16_tflops"] * 1e12), io_bytes / (peaks["hbm_gbs"] * 1e9))
-    dense = dense_context(qd, kd, vd, model, flush if flush_l2 else None, stream, ms)
-    backward = backward_line(m, w, qd, kd, vd, flush if flush_l2 else None, stream)
+    dense = dense_context(qd, kd, vd, model, flush, stream, ms)
+    backward = backward_line(m, w, qd, kd, vd, flush, stream)
 
     # End to end (copies inside the timed region): the host-buffer entry point
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -304,15 +389,19 @@ def run_ours(args, rank, world, device):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(device)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
+    e2e_times = []
     for _ in range(e2e_n):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         e2e_call()
-    e1.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = e0.elapsed_time(e1) / e2e_n
-    e2e_ms = max_over_ranks(e2e_ms, world, device)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        e2e_times.append(e0.elapsed_time(e1))
+    e2e_ms = max_over_ranks(statistics.median(e2e_times), world, device)
+    del qh, kh, vh, oh
+
+    configs = extra_configs(m, args, device, stream, flush_buf, peaks, world) if not args.no_configs else {}
 
     es = q.element_size()
     rec = {
@@ -323,6 +412,8 @@ def run_ours(args, rank, world, device):
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": ms,
+        "ms_per_step_mean": mean_ms,
+        "timing": "median of per-step CUDA-event times on the launching stream; max over ranks",
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -334,9 +425,7 @@ def run_ours(args, rank, world, device):
                    "l2": "flushed between steps" if flush_l2 else "inputs larger than L2"},
         "monarch_gflop_per_call": model["flops"] / 1e9,
         "dense_gflop_per_call": model["dense_flops"] / 1e9,
-        "call_roofline": {"roofline_ms": call_roof_ms, "frac": call_roof_ms / ms,
-                          "bound": "tensor" if model["flops"] / (peaks["bf16_tflops"] * 1e12)
-                          >= io_bytes / (peaks["hbm_gbs"] * 1e9) else "hbm"},
+        "call_roofline": call_roofline(w, model, peaks, ms),
         "roofline": roof,
         "kernels": {p: {"ms_per_launch": prof[p][0] / prof[p][1], "launches_per_step": prof[p][1] / nprof}
                     for p in prof if prof[p][1] > 0},
@@ -348,6 +437,7 @@ def run_ours(args, rank, world, device):
         "clocks": clocks.summary(),
         "dense_context": dense,
         "backward": backward,
+        "configs": configs,
     }
     return rec, (q, k, v, w)
 
@@ -582,6 +672,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="time only --workload (skip the per-configuration timings of the other workloads)")
     ap.add_argument("--batch", type=int, default=0, help="override the workload's batch (profiler cases)")
     ap.add_argument("--heads", type=int, default=0, help="override the workload's head count (profiler cases)")
     ap.add_argument("--profile-calls", type=int, default=0,

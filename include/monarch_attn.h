@@ -200,7 +200,9 @@ int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void*
  * (monarch_attn_workspace_bytes) exceeds 128 MiB are rejected with
  * MONARCH_ENOMEM and a message.  The first call on a device looks up the
  * array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture.  All calls on a device
+ * make that first call before any stream capture.  The address is kept for
+ * the life of the process: after cudaDeviceReset on a device this entry point
+ * must not be called there again in the same process.  All calls on a device
  * share the one array and it keeps the last call's contents (every value is
  * written before it is read, so nothing needs clearing): calls whose GPU work
  * overlaps (different streams, or different host threads) race on it and
@@ -211,15 +213,17 @@ int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* 
                              int dtype, int out_dtype, cudaStream_t stream);
 
 /* Byte offsets, inside a workspace, of the intermediates left by the last
- * iteration (for inspection in tests): [0] k~ [B*heads][b2][b1k][d] (f32 for
- * f32 inputs; otherwise a high plane of the input type followed by a low
- * plane), [1] z (f32 for f32 inputs; otherwise f16 high and low planes),
- * [2] q~ of the last R step with iters >= 2 (f32, same shape), [3] h
- * [B*heads][b2][b1k_pad] (f32; in nats for f32 inputs, in bits, i.e. base-2
- * entropy, for bf16/f16 inputs), [4] row log2-sum-exp of the last non-final
- * L step [B*heads][b2][b1q_pad] (f32, base-2 logits s*log2(e)*q.k~ +
- * log2(e)*h), [5] KV-init mean query [B*heads][b2][d] (f32), [6] queries in
- * block-major order [B*heads][b2][b1q][d] (input type; bf16/f16 only).
+ * iteration (for inspection in tests), each [B*heads][b2][b1k][d] per plane
+ * with b2 = tile_h*tile_w positions and b1k = kv_len/(H*W) * (H/tile_h) *
+ * (W/tile_w) key tiles: [0] k~ (f32 for f32 inputs; otherwise an f16 high
+ * plane followed by an f16 low plane, k~ = high + low), [1] z (same types),
+ * [2] q~ of the last R step with iters >= 2 (f32 for f32 inputs; otherwise a
+ * high and a low plane of the input type), [3] h [B*heads][b2][b1k_pad]
+ * (f32; in nats for f32 inputs, in bits, i.e. base-2 entropy, for bf16/f16
+ * inputs), [4] row log2-sum-exp of the last non-final L step
+ * [B*heads][b2][b1q_pad] (f32, base-2 logits s*log2(e)*q.k~ + log2(e)*h),
+ * [5] KV-init mean query [B*heads][b2][d] (f32), [6] queries in block-major
+ * order [B*heads][b2][b1q][d] (f16 for bf16/f16 inputs; absent for f32).
  * b1k_pad and b1q_pad are b1k and b1q rounded up to a multiple of 4.
  * Returns the total bytes, 0 on invalid arguments. */
 size_t monarch_attn_workspace_layout(int B, int heads, int T, int H, int W, int d,
@@ -238,7 +242,9 @@ enum {
   MONARCH_PHASE_BWD_DQ = 6,   /* L-step part of dq, per query row               */
   MONARCH_PHASE_BWD_DKV = 7,  /* dk~, dz, dh per key column                      */
   MONARCH_PHASE_BWD_R = 8,    /* R-step backward per tile: dk, dv, dq finished */
-  MONARCH_NUM_PHASES = 9
+  /* one refinement step (iters = 1, bf16/f16) as one kernel: R step and output pass */
+  MONARCH_PHASE_ONESTEP = 9,
+  MONARCH_NUM_PHASES = 10
 };
 
 /* Number of kernels this process has launched through the library (host
@@ -267,7 +273,8 @@ int monarch_attn_device_error(int reset);
 const char* monarch_attn_last_error(void);
 
 /* ABI version (major*100 + minor): 1.02 adds the backward (monarch_attn_bwd),
- * the training pair and monarch_attn_fwd_host_ex to the forward of 1.00. */
+ * the training pair and monarch_attn_fwd_host_ex to the forward of 1.00; 1.03
+ * adds MONARCH_PHASE_ONESTEP (one refinement step runs as one kernel). */
 int monarch_attn_version(void);
 
 #ifdef __cplusplus

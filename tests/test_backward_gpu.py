@@ -7,10 +7,11 @@ RMS(ref) + (u/2) |ref|.  f32 inputs run the fp32 CUDA-core backward, tol =
 1e-3: dS = L (dy.z - D) subtracts two rounded dot products of length d whose
 difference is small where L is peaked, so the relative error of dS, not of
 the output, sets it.  bf16/f16 inputs run the tensor-core backward, tol =
-2e-2, the bar of every bf16/f16 result of this library: its own products
-carry every operand as f16 hi/lo planes, and the rest is the precision of the
-forward it recomputes (R rounded to the input type in k~ = R k and z = R v, P
-a single f16 in y = P z).
+1e-2, half the forward's 2e-2 bar: its own products carry every operand as
+f16 hi/lo planes, and the rest is the precision of the forward it recomputes
+(R rounded to the input type in k~ = R k and z = R v, P a single f16 in
+y = P z), measured at most 0.8e-2 of the RMS (a ragged 75-tile grid), so a
+doubling of that error fails.
 The second is the one rounding of the stored gradient (u/2 = 2^-8 for bf16,
 2^-11 for f16, 0 for f32), which on peaked rows' entries of many times the RMS
 is larger than any fixed fraction of the RMS.  Full-size workloads compare
@@ -28,7 +29,7 @@ from structured_sparse_attention_grid_b200.workloads import (DTYPES, WORKLOADS, 
 
 pytestmark = pytest.mark.gpu
 
-TOL_GRAD = {"f32": 1e-3, "bf16": 2e-2, "f16": 2e-2}   # by input dtype
+TOL_GRAD = {"f32": 1e-3, "bf16": 1e-2, "f16": 1e-2}   # by input dtype
 # largest relative error of one round-to-nearest store in the gradient type,
 # 2^-p for p significand bits (8 for bf16, 11 for f16)
 HALF_ULP = {torch.float32: 0.0, torch.bfloat16: 2.0 ** -8, torch.float16: 2.0 ** -11}

@@ -41,3 +41,19 @@ def test_visible_fraction_counts_the_oracle_mask():
         g = om.Grid(w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
         vis = g.visible() if w.chunk_frames else np.ones((1, 1), dtype=bool)
         assert abs(bench.visible_fraction(w) - float(vis.mean())) < 1e-12
+
+
+def test_roofline_bytes_of_the_chunk_workload():
+    """Compulsory call bytes = Q, K, V, O in the input dtype (57.5 MB for 12
+    heads of 4680 tokens at d = 128, bf16); the R-step launch moves q~ (or q),
+    k in and k~ out, and in the final launch also v in and z out, plus h."""
+    w = WORKLOADS["chunk_4680_bf16"]
+    m = bench.work_model(w)
+    n = 12 * 4680 * 128 * 2                      # bytes of one [heads, N, d] bf16 tensor
+    assert m["io_bytes"] == 4 * n
+    hb = 12 * 24 * 195 * 4
+    assert m["phases"]["r_step"]["bytes"] == (3 * n + 5 * n) / 2 + hb
+    peaks = {"bf16_tflops": 1646.3, "hbm_gbs": 6550.4, "source": "measured"}
+    r = bench.call_roofline(w, m, peaks, 1.0)
+    assert abs(r["roofline_ms"] - 4 * n / 6550.4e9 * 1e3) < 1e-12 and r["bound"] == "hbm"
+    assert abs(r["roofline_ms"] * 1e3 - 8.78) < 0.01   # microseconds

@@ -18,7 +18,7 @@ import pytest
 import torch
 
 import structured_sparse_attention_grid_b200 as m
-from structured_sparse_attention_grid_b200.workloads import WORKLOADS, make_inputs
+from structured_sparse_attention_grid_b200.workloads import WORKLOADS, Workload, make_inputs
 
 TOL_F32 = 1e-4
 TOL_LOWP = 2e-2
@@ -31,20 +31,26 @@ def _abi_call(fn, q, k, v, out, w, stream):
               ctypes.c_long(w.Nk), code[q.dtype], code[out.dtype], ctypes.c_void_p(stream))
 
 
+# a small KV-cache step: one query frame against three key frames
+KV_SMALL = Workload("noalloc_kv_1x3", 1, 2, 1, 12, 20, 128, 4, 4, 2, "bf16", 9, "pos_planted", Tk=3, planted=4)
+CASES = [(WORKLOADS["chunk_4680_bf16"], torch.float32), (WORKLOADS["toy_256_f32"], torch.float32),
+         (WORKLOADS["sweep_2048_f16"], torch.float32), (KV_SMALL, torch.float32),
+         (WORKLOADS["chunk_4680_bf16"], torch.bfloat16)]
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", ["chunk_4680_bf16", "toy_256_f32", "sweep_2048_f16"])
-def test_noalloc_matches_the_allocating_entry_point(name, cuda_lib):
+@pytest.mark.parametrize("w,out_dtype", CASES, ids=[f"{w.name}-{str(dt)[6:]}" for w, dt in CASES])
+def test_noalloc_matches_the_allocating_entry_point(w, out_dtype, cuda_lib):
     lib = m.load_library()
-    w = WORKLOADS[name]
     q, k, v = (t.cuda() for t in make_inputs(w))
     stream = torch.cuda.current_stream().cuda_stream
-    ref = torch.empty(q.shape, dtype=torch.float32, device="cuda")
-    assert _abi_call(lib.monarch_attn_fwd, q, k, v, ref, w, stream) == 0, lib.monarch_attn_last_error()
+    ref = torch.empty(q.shape, dtype=out_dtype, device="cuda")
+    assert _abi_call(lib.monarch_attn_fwd, q, k, v, ref, w, stream) == 0, lib.monarch_attn_last_error().decode()
     torch.cuda.synchronize()
     rms = float(ref.double().pow(2).mean().sqrt())
     tol = TOL_F32 if w.dtype == "f32" else TOL_LOWP * rms
     for call in range(2):
-        got = torch.full(q.shape, float("nan"), dtype=torch.float32, device="cuda")
+        got = torch.full(q.shape, float("nan"), dtype=out_dtype, device="cuda")
         rc = _abi_call(lib.monarch_attn_fwd_noalloc, q, k, v, got, w, stream)
         assert rc == 0, lib.monarch_attn_last_error().decode()
         torch.cuda.synchronize()
@@ -56,7 +62,7 @@ def test_noalloc_matches_the_allocating_entry_point(name, cuda_lib):
 @pytest.mark.gpu
 def test_noalloc_rejects_a_problem_larger_than_its_scratch(cuda_lib):
     lib = m.load_library()
-    w = WORKLOADS["full_32760_bf16"]  # about 1.6 GB of workspace
+    w = WORKLOADS["full_32760_bf16"]  # about 1.35 GiB of workspace
     assert lib.monarch_attn_workspace_bytes(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw, w.iters, w.Nk, 1) > (128 << 20)
     q = torch.empty(16, dtype=torch.bfloat16, device="cuda")  # never touched: the size check comes first
     rc = lib.monarch_attn_fwd_noalloc(q.data_ptr(), q.data_ptr(), q.data_ptr(), q.data_ptr(), w.B, w.heads, w.T,
