@@ -242,7 +242,10 @@ enum {
   MONARCH_PHASE_BWD_DQ = 6,   /* L-step part of dq, per query row               */
   MONARCH_PHASE_BWD_DKV = 7,  /* dk~, dz, dh per key column                      */
   MONARCH_PHASE_BWD_R = 8,    /* R-step backward per tile: dk, dv, dq finished */
-  /* one refinement step (iters = 1, bf16/f16) as one kernel: R step and output pass */
+  /* one refinement step (iters = 1, bf16/f16) as one kernel, R step and output
+   * pass together; used when the environment variable MONARCH_ONESTEP_KERNEL
+   * is "1" at the call (the default runs the two kernels, which is faster on
+   * B200; both give the same values bit for bit) */
   MONARCH_PHASE_ONESTEP = 9,
   MONARCH_NUM_PHASES = 10
 };
@@ -274,7 +277,7 @@ const char* monarch_attn_last_error(void);
 
 /* ABI version (major*100 + minor): 1.02 adds the backward (monarch_attn_bwd),
  * the training pair and monarch_attn_fwd_host_ex to the forward of 1.00; 1.03
- * adds MONARCH_PHASE_ONESTEP (one refinement step runs as one kernel). */
+ * adds MONARCH_PHASE_ONESTEP (one refinement step as one kernel, on request). */
 int monarch_attn_version(void);
 
 #ifdef __cplusplus

@@ -230,7 +230,6 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
   constexpr int NH = D / 64;
   constexpr uint32_t kPl = NH * 2 * kBox;   // one 128-row operand plane: [d half][row half][64 rows][128 B]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
   if (tc::smem_misaligned(smem_raw)) return;
   uint8_t* sK = smem_raw;               // k~ [plane]
   uint8_t* sZ = sK + 2 * kPl;           // z  [plane]
@@ -279,6 +278,9 @@ l_bwd_kv(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps 
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
   ptx::griddep_wait();
   const uint32_t tmem = *sTmem;
   const uint32_t tX = tmem, tY = tmem + 128, tZ = tmem + 256, tK = tmem + 256 + D;
@@ -426,7 +428,6 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
   constexpr int NH = D / 64;
   constexpr uint32_t kPl = NH * 2 * kBox;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
   if (tc::smem_misaligned(smem_raw)) return;
   uint8_t* sQ = smem_raw;               // q
   uint8_t* sY = sQ + kPl;               // sigma dy [plane]
@@ -472,6 +473,9 @@ l_bwd_q(const __grid_constant__ tc::Maps maps, const __grid_constant__ BwdMaps b
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
   ptx::griddep_wait();
   const uint32_t tmem = *sTmem;
   const uint32_t tX = tmem, tY = tmem + 128, tA = tmem + 256;

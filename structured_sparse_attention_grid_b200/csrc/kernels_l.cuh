@@ -77,16 +77,21 @@ constexpr size_t row_smem() {
 // TMEM, tile t at column 256 t.  OUT: S [0, 128) (q.k~_hi in [0, 64), q.k~_lo
 // in [64, 128); P over [0, 32)), O [128, 128 + D).  !OUT: S buffers [0, 128),
 // [128, 256).
-template <typename TQ, typename TO, int D, bool OUT, bool LSE_OUT = false>
-__global__ void __launch_bounds__(kThreads, 1)
-l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
+// One row-pass item (query tiles a1_base, a1_base + 128 of head bh,
+// position a2) run by all kThreads threads of the CTA on `smem_raw`
+// (row_smem<D, OUT>() bytes, 1024-byte aligned) and 512 TMEM columns at
+// `tmem`.  ready != nullptr: the load warp waits (bounded, acquire) for
+// *ready >= ready_need before its first load, instead of the item waiting for
+// the previous grid, so it may overlap the R-step items that produce its
+// inputs (in the same grid or in the kernel before).
+template <typename TQ, typename TO, int D, bool OUT, bool LSE_OUT>
+__device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& maps, float* __restrict__ lse,
+                                           const Geo& g, int a1_base, int a2, int bh, uint8_t* smem_raw,
+                                           uint32_t tmem, const int* ready, int ready_need) {
   constexpr int NH = D / 64;
   constexpr uint32_t kQt = NH * 2 * kBox;    // q of one tile (128 rows)
   constexpr uint32_t kKst = 2 * NH * kBox;   // k~ hi+lo, 64 rows: [d half][plane][64 rows]
   constexpr uint32_t kZst = 2 * NH * kBox;   // z hi+lo, 64 rows:  [plane][d half][64 rows]
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
-  if (smem_misaligned(smem_raw)) return;
   uint8_t* sQ = smem_raw;                                             // [2 tiles]
   uint8_t* sK = sQ + 2 * kQt;                                         // [kKS]
   uint8_t* sZ = sK + kKS * kKst;                                      // [2] (OUT)
@@ -103,11 +108,9 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
   uint64_t* s_free = bar + 15;   // [tile][buf]   (!OUT)
   uint64_t* p_full = bar + 19;   // [tile]        (OUT)
   uint64_t* o_done = bar + 21;   // [tile]        (OUT)
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 23);
+  // bar + 23: the TMEM slot of a one-item kernel (row_tmem_slot)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int a2 = blockIdx.y, bh = blockIdx.z;
-  const int a1_base = blockIdx.x * 2 * kTile;
   const int zrow = bh * g.b2 + a2;
   const int plane_rows = g.BH * g.b2;
   // key blocks any row of this CTA sees (all of them without a causal mask)
@@ -135,15 +138,12 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     }
     ptx::fence_mbar_init();
   }
-  if (warp == 0) {
-    ptx::tmem_alloc(sTmem, 512);
-    ptx::tmem_relinquish();
-  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
-  const uint32_t tmem = *sTmem;
+  // set-up done: global data of the previous kernel from here on (or of the
+  // items counted in *ready, which the load warp waits for)
+  if (!ready) ptx::griddep_wait();
   auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
   auto tO = [&](int t) { return tmem + 256 * t + 128; };
 
@@ -151,6 +151,12 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
     if (lane == 0) {
       // --------------------------------------------------------- TMA producer
       ptx::prefetch_tmap(&maps.kt);
+      if (ready) {
+        // the R-step items of this head are done: their TMA and h stores are
+        // visible (acquire), and this thread's loads below come after it
+        ptx::wait_count(ready, ready_need);
+        ptx::fence_proxy_async_global();
+      }
       ptx::mbar_expect_tx(q_full, 2 * kQt);
       for (int t = 0; t < 2; ++t)
         for (int hf = 0; hf < NH; ++hf)
@@ -429,9 +435,38 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
       }
     }
   }
+}
+
+template <int D, bool OUT>
+constexpr uint32_t row_tmem_slot() {
+  constexpr int NH = D / 64;
+  return (uint32_t)(2 * NH * 2 * kBox + kKS * 2 * NH * kBox + (OUT ? 2 * 2 * NH * kBox : 0) + kKS * kBlk * 4 +
+                    2 * xchg_tile_bytes<OUT ? 1 : 0>() + 23 * 8);
+}
+
+// One row-pass item per CTA: grid (ceil(b1q / 256), b2, BH), kThreads threads.
+template <typename TQ, typename TO, int D, bool OUT, bool LSE_OUT = false>
+__global__ void __launch_bounds__(kThreads, 1)
+l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (smem_misaligned(smem_raw)) return;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem_raw + row_tmem_slot<D, OUT>());
+  if (threadIdx.x < 32) {
+    ptx::tmem_alloc(sTmem, 512);
+    ptx::tmem_relinquish();
+  }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(tmem, 512);
+  ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
+  const uint32_t tmem = *sTmem;
+  l_row_item<TQ, TO, D, OUT, LSE_OUT>(out, maps, lse, g, blockIdx.x * 2 * kTile, blockIdx.y, blockIdx.z, smem_raw,
+                                      tmem, nullptr, 0);
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) ptx::tmem_dealloc(tmem, 512);
 }
 
 // ===========================================================================
@@ -466,7 +501,6 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   constexpr uint32_t kKst = NH * 2 * kBox;   // k~ hi of one block: [d half][128 keys]
   constexpr int kXt = xchg_tile_bytes<0>();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
   if (smem_misaligned(smem_raw)) return;
   uint8_t* sQ = smem_raw;                                      // [2 tiles]
   uint8_t* sK = sQ + 2 * kQt;                                  // [kLS]
@@ -508,6 +542,9 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
   ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
   const uint32_t tmem = *sTmem;
   auto tS = [&](int t, int b) { return tmem + 256 * t + 128 * b; };
@@ -687,7 +724,6 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   constexpr uint32_t kKt = 2 * NH * 2 * kBox;   // k~ hi+lo of one tile: [plane][d half][128 rows]
   constexpr uint32_t kQst = NH * 2 * kBox;      // 128 query rows: [d half][128 rows]
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
   if (smem_misaligned(smem_raw)) return;
   uint8_t* sK = smem_raw;                                    // [2 tiles]
   uint8_t* sQ = sK + 2 * kKt;                                // [kQS]
@@ -740,6 +776,9 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
   ptx::griddep_wait();   // set-up done: global data of the previous kernel from here on
   const uint32_t tmem = *sTmem;
   auto tS = [&](int t) { return tmem + 256 * t; };
@@ -922,7 +961,10 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
         const float beta = beta2.x + beta2.y + xs[(hf ^ 1) * kTile + r];
         ok = ok && ptx::mbar_wait(o_done + t, icnt & 1);
         ptx::tc_fence_after();
-        const float inv = 1.f / beta;
+        // beta = 0: every query gives this key tile a weight below 2^-141, so
+        // every 2^(x - lse + 15) flushed to zero; the accumulator is zero too,
+        // and q~ = 0 replaces the 0/0 that would spread NaN to every row
+        const float inv = beta > 0.f ? 1.f / beta : 0.f;
         const float2 inv2 = make_float2(inv, inv);
         // q~ as hi / lo planes of the input type: the A operand of the next R step
         TQ* dst = qt + ((long long)zrow * g.b1k + (c1 < g.b1k ? c1 : 0)) * D + hf * (D / 2);

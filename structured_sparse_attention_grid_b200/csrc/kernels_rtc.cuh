@@ -74,17 +74,37 @@ constexpr size_t rtc_smem() {
   return need > 80 * 1024 ? need : 80 * 1024;
 }
 
-// grid (ceil(b1k / G), BH), block kRtcThreads; 1 <= G <= floor(128 / r8).
-// Two CTAs (18 warps, five on some SM sub-partition) leave 96 registers a thread.
+// Bytes of shared memory one R-step item uses (operand boxes, barriers,
+// softmax exchange), and where a kernel running one item per CTA keeps the
+// TMEM address (inside the item's barrier area, in a slot the item leaves
+// alone).
+template <int D>
+constexpr uint32_t rtc_item_bytes() { return (uint32_t)(3 * (D / 64) * kRBox + kRtcAux); }
+template <int D>
+constexpr uint32_t rtc_tmem_slot() { return (uint32_t)(3 * (D / 64) * kRBox + 8 * 8); }
+
+// One R-step item: key tiles [c1_0, c1_0 + G) of head bh (fewer at the end of
+// the head), run by 288 threads with item-local thread index tid (eight row
+// warps, then the control warp) on `smem` (1024-byte aligned,
+// rtc_item_bytes<D>()) and 256 TMEM columns at `tmem`.  bar_row and bar_all
+// are the named barriers of the item's row warps and of all its threads;
+// warp0 is the CTA warp index of the item's first warp (its row warps reach
+// the TMEM lane quadrants (warp0 + w) mod 4, two warps each).
+// ready != nullptr: the control thread waits (bounded, acquire) for
+// *ready >= ready_need before its loads, and the item does not wait for the
+// previous grid (the count stands for it).
+// done != nullptr: once every output of the item (k~, z and the block-major q
+// copy through TMA, h by the row threads) is written and visible at GPU
+// scope, one thread adds 1 to *done (release), for consumers in other CTAs
+// that read these outputs with TMA after an acquire of the count.
 template <typename TQ, int D>
-__global__ void __launch_bounds__(kRtcThreads, 2)
-r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work w, TcPlanes<TQ> out, Geo g,
-           int mode, int final_step, int G) {
+__device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __restrict__ q, const Work& w,
+                                            const TcPlanes<TQ>& out, const Geo& g, int mode, int final_step, int G,
+                                            int c1_0, int bh, uint8_t* smem_raw, uint32_t tmem, int tid,
+                                            int warp0, int bar_row, int bar_all, const int* ready, int ready_need,
+                                            int* done) {
   constexpr int NH = D / 64;
   constexpr int bf16 = TcType<TQ>::kBf16;
-  extern __shared__ __align__(1024) uint8_t smem_raw[];
-  ptx::griddep_launch();
-  if (tc::smem_misaligned(smem_raw)) return;
   uint8_t* sA = smem_raw;                  // [plane][d half] boxes; V in plane 0 later
   uint8_t* sK = sA + 2 * NH * kRBox;       // [d half] boxes
   uint64_t* bar = reinterpret_cast<uint64_t*>(sK + NH * kRBox);
@@ -96,17 +116,15 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   uint64_t* bar_free = bar + 5;  // row warps: k~ read out of TMEM
   uint64_t* bar_v = bar + 6;     // TMA: values
   uint64_t* bar_q = bar + 7;     // row warps: query rows read (first step, bf16, before V lands)
-  uint32_t* sTmem = reinterpret_cast<uint32_t*>(bar + 8);
+  // bar + 8: the TMEM slot of a one-item kernel (rtc_tmem_slot)
   float* sRed = reinterpret_cast<float*>(bar + 16);   // [max | sum p | sum p s][half][row]
 
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.y;
+  const int warp = tid >> 5, lane = tid & 31;
   const int r8 = (g.b2 + 7) & ~7;   // G * r8 <= 128 (the host's choice of G)
   // rows per stacked tile: 32 when four tiles of at most 32 positions fit, so
   // that each row warp holds one tile and reads one 32-column chunk of S;
   // else b2 rounded up to 8
   const int rs = (g.b2 <= 32 && G * 32 <= kRtcRows) ? 32 : r8;
-  const int c1_0 = blockIdx.x * G;
   const int Gn = min(G, g.b1k - c1_0);
 
   if (tid == kRtcRowThreads) {
@@ -119,10 +137,6 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     ptx::mbar_init(bar_v, 1);
     ptx::mbar_init(bar_q, 8);
     ptx::fence_mbar_init();
-  }
-  if (warp == 0) {
-    ptx::tmem_alloc(sTmem, 256);
-    ptx::tmem_relinquish();
   }
   // Zero every row that no load writes (in-tile padding, tiles past the end):
   // K and V rows there meet zero R entries, and 0 * NaN would not be zero.
@@ -139,11 +153,10 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
   }
   ptx::fence_proxy_async();
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::named_bar(bar_all, kRtcThreads);
   ptx::tc_fence_after();
   // set-up done: from here on global memory of the previous kernel is used
-  ptx::griddep_wait();
-  const uint32_t tmem = *sTmem;
+  if (!ready) ptx::griddep_wait();
   const uint32_t tS = tmem, tAcc = tmem + 128;
 
   // tile c1 -> (frame, tile row, tile column) of its grid box
@@ -159,6 +172,11 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     if (lane == 0) {
       // ------------------------------------------------ loads and MMA issue
       ptx::prefetch_tmap(&maps.k);
+      if (ready) {
+        // the items this one reads from are done (acquire), before the loads
+        ptx::wait_count(ready, ready_need);
+        ptx::fence_proxy_async_global();
+      }
       bool ok = true;
       uint32_t bytes = 0;
       for (int gg = 0; gg < Gn; ++gg) {
@@ -254,11 +272,12 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
         ptx::tc_fence_after();
         if (ok) issue_rb(sA);
       }
-      ptx::bulk_wait_read();
+      if (done) ptx::bulk_wait_all(); else ptx::bulk_wait_read();
     }
   } else {
     // ------------------------------------------------------------- row warps
-    const int qw = warp & 3, half = warp >> 2;  // lane quadrant, column half
+    // lane quadrant: a warp reaches the TMEM lanes of its CTA warp index mod 4
+    const int qw = (warp + warp0) & 3, half = warp >> 2;   // lane quadrant, column half
     const int r = 32 * qw + lane;               // stacked row = TMEM lane
     const int gg = r / rs, a2 = r - gg * rs;
     const int c1 = c1_0 + gg;
@@ -323,7 +342,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
       ptx::fence_proxy_async();
       __syncwarp();
       if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
-      ptx::named_bar(1, kRtcRowThreads);
+      ptx::named_bar(bar_row, kRtcRowThreads);
       if (tid == 0 && ok) {
         for (int t = 0; t < Gn; ++t) {
           if (!exact_q(c1_0 + t)) continue;
@@ -376,7 +395,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     // either warp writes R over S
     sRed[half * 128 + r] = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
     ptx::tc_fence_before();
-    ptx::named_bar(1, kRtcRowThreads);
+    ptx::named_bar(bar_row, kRtcRowThreads);
     ptx::tc_fence_after();
     const float m = fmaxf(sRed[r], sRed[128 + r]);
     const float ms = (m == -INFINITY) ? 0.f : m * g.sl2;   // base-2 units; a row with no column stays 0
@@ -395,7 +414,7 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     }
     sRed[256 + half * 128 + r] = (lq[0] + lq[1]) + (lq[2] + lq[3]);
     sRed[512 + half * 128 + r] = (pq[0] + pq[1]) + (pq[2] + pq[3]);
-    ptx::named_bar(1, kRtcRowThreads);
+    ptx::named_bar(bar_row, kRtcRowThreads);
     const float l = sRed[256 + r] + sRed[384 + r];
     // sum p (x s2 - ms) with x the raw score
     const float xe = g.sl2 * (sRed[512 + r] + sRed[640 + r]) - ms * l;
@@ -477,28 +496,64 @@ r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work 
     ptx::tc_fence_after();
     if (bf16 && mode != QT_BUFFER) {
       if (tid == 0) ptx::bulk_wait_read();   // the q copy has read the A lo plane
-      ptx::named_bar(1, kRtcRowThreads);
+      ptx::named_bar(bar_row, kRtcRowThreads);
     }
     // k~ (f16 planes): hi plane staged over the A lo plane, lo plane over K
     // (both read by now: S and k~ are complete)
     stage_row(sA + NH * kRBox, sK, final_step != 0);
-    ptx::named_bar(1, kRtcRowThreads);
+    ptx::named_bar(bar_row, kRtcRowThreads);
     if (tid == 0 && ok) store_tiles(&maps.kt, sA + NH * kRBox, sK);
     if (final_step) {
       ok = ok && ptx::mbar_wait(bar_acc, 1);
       ptx::tc_fence_after();
       if (tid == 0) ptx::bulk_wait_read();   // the k~ stores have read their staging
-      ptx::named_bar(1, kRtcRowThreads);
+      ptx::named_bar(bar_row, kRtcRowThreads);
       // z: hi plane over the A hi plane (V is consumed), lo over the A lo plane
       stage_row(sA, sA + NH * kRBox, false);
-      ptx::named_bar(1, kRtcRowThreads);
+      ptx::named_bar(bar_row, kRtcRowThreads);
       if (tid == 0 && ok) store_tiles(&maps.z, sA, sA + NH * kRBox);
     }
-    if (tid == 0) ptx::bulk_wait_read();
+    if (tid == 0) {
+      if (done) ptx::bulk_wait_all(); else ptx::bulk_wait_read();
+    }
+    if (done) __threadfence();   // this thread's h store, before the count below
+  }
+  ptx::tc_fence_before();
+  ptx::named_bar(bar_all, kRtcThreads);
+  if (done && tid == 0) {
+    // the TMA stores are complete (waited above by the threads that issued
+    // them); order them and the h stores before the release of the count
+    ptx::fence_proxy_async_global();
+    __threadfence();
+    ptx::red_release_add(done, 1);
+  }
+}
+
+// grid (ceil(b1k / G), BH), block kRtcThreads; 1 <= G <= floor(128 / r8).
+// Two CTAs (18 warps, five on some SM sub-partition) leave 96 registers a thread.
+template <typename TQ, int D>
+__global__ void __launch_bounds__(kRtcThreads, 2)
+r_step_tc5(const __grid_constant__ RtcMaps maps, const TQ* __restrict__ q, Work w, TcPlanes<TQ> out, Geo g,
+           int mode, int final_step, int G) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  if (tc::smem_misaligned(smem_raw)) return;
+  uint32_t* sTmem = reinterpret_cast<uint32_t*>(smem_raw + rtc_tmem_slot<D>());
+  if (threadIdx.x < 32) {
+    ptx::tmem_alloc(sTmem, 256);
+    ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 0) ptx::tmem_dealloc(tmem, 256);
+  ptx::tc_fence_after();
+  // dependents may start once every CTA of this grid holds its TMEM, so none
+  // of theirs can take the columns a CTA of this grid still has to allocate
+  ptx::griddep_launch();
+  const uint32_t tmem = *sTmem;
+  r_step_item<TQ, D>(maps, q, w, out, g, mode, final_step, G, blockIdx.x * G, blockIdx.y, smem_raw, tmem,
+                     threadIdx.x, 0, 1, 2, nullptr, 0, nullptr);
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x < 32) ptx::tmem_dealloc(tmem, 256);
 }
 
 }  // namespace monarch

@@ -21,6 +21,7 @@
 #include "kernels_tc.cuh"
 #include "kernels_rtc.cuh"
 #include "kernels_l.cuh"
+#include "kernels_onestep.cuh"
 #include "kernels_bwd.cuh"
 #include "kernels_bwd_tc.cuh"
 
@@ -83,6 +84,15 @@ bool debug_sync() {
 
 int read_device_error(int reset);
 
+// MONARCH_ONESTEP_KERNEL=1 (read at every call): run one refinement step
+// (bf16 / f16) as the single kernel onestep_tc instead of the R-step kernel
+// followed by the output-pass kernel.  Both compute the same values bit for
+// bit; the two kernels are the faster of the two on B200 and the default.
+bool onestep_fused() {
+  const char* e = getenv("MONARCH_ONESTEP_KERNEL");
+  return e && e[0] == '1';
+}
+
 // Launches one kernel through `f`, counting it and, when profiling is on,
 // bracketing it with events on its stream.
 template <typename F>
@@ -90,7 +100,7 @@ void launch(int phase, cudaStream_t st, F&& f) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (debug_sync()) {
     static const char* names[] = {"qbar", "r_step", "l_lse", "l_out", "l_col",
-                                  "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r"};
+                                  "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r", "onestep"};
     fprintf(stderr, "[monarch] launch %s ...\n", names[phase]);
     auto t0 = std::chrono::steady_clock::now();
     f();
@@ -135,6 +145,7 @@ struct Plan {
   int iters;
   bool kv;
   size_t off[kRegions];
+  size_t counters;   // int [1 + BH]: the ticket and per-head R-item counts of onestep_tc
   size_t total;
 };
 
@@ -205,6 +216,8 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
     p->off[i] = o;
     o += align256(sizes[i]);
   }
+  p->counters = o;
+  o += align256((size_t)(1 + BH) * sizeof(int));
   p->total = o;
   return MONARCH_OK;
 }
@@ -420,6 +433,30 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
   const int r_group = r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
+  if (p.iters == 1 && onestep_fused()) {
+    // one refinement step: the R step and the output pass in one kernel
+    constexpr size_t smem_one = onestep_smem<D>();
+    static std::atomic<bool> one_set[kMaxDevices];
+    cudaError_t e = once_per_device(one_set, [&] { return allow_smem(onestep_tc<TQ, TO, D>, smem_one); });
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(onestep)");
+    int* counters = reinterpret_cast<int*>(ws + p.counters);
+    if ((e = cudaMemsetAsync(counters, 0, (size_t)(1 + g.BH) * sizeof(int), st)) != cudaSuccess)
+      return cuda_fail(e, "cudaMemsetAsync(counters)");
+    if (p.kv)
+      launch(MONARCH_PHASE_QBAR, st, [&] {
+        launch_pdl(qbar_kernel<TQ>, dim3(g.b2, g.BH), dim3(kQbarThreads), 0, st, q, w.qbar, g);
+      });
+    const long long n_r = (long long)grid_r.x * g.BH;
+    const long long n_l = (long long)grid_q.x * grid_q.y * grid_q.z;
+    // launched in plain stream order (after the counters are zeroed)
+    launch(MONARCH_PHASE_ONESTEP, st, [&] {
+      onestep_tc<TQ, TO, D><<<(unsigned)((n_r + 1) / 2 + n_l), tc::kThreads, smem_one, st>>>(
+          rmaps, maps, q, w, planes, out, g, p.kv ? (int)QT_KVINIT : (int)QT_IDENTITY, r_group, counters);
+    });
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
+    return MONARCH_OK;
+  }
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
     int mode = QT_BUFFER;
@@ -913,7 +950,7 @@ int check_io(const void* q, const void* k, const void* v, const void* out) {
 
 extern "C" {
 
-int monarch_attn_version(void) { return 102; }
+int monarch_attn_version(void) { return 103; }
 
 unsigned long long monarch_attn_launch_count(void) { return g_launches.load(); }
 

@@ -226,6 +226,41 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until every bulk store of this thread has finished reading shared memory.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Waits until every bulk store of this thread is complete (its writes to
+// global memory performed).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// ---------------------------------------------------------------- hand-off between CTAs
+// Orders this thread's global-memory accesses across the generic and async
+// proxies (TMA stores made visible before a generic release; a generic
+// acquire before later TMA loads).
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// *p += v with release semantics at GPU scope.
+__device__ __forceinline__ void red_release_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// *p with acquire semantics at GPU scope.
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// Waits until *p >= target (acquire).  Gives up after about 2^31 SM clocks,
+// records kErrMbarTimeout and returns false.
+__device__ __forceinline__ bool wait_count(const int* p, int target) {
+  if (ld_acquire(p) >= target) return true;
+  const long long t0 = clock64();
+  while (ld_acquire(p) < target) {
+    if (clock64() - t0 > (1LL << 31)) {
+      atomicExch(&g_device_error, kErrMbarTimeout);
+      return false;
+    }
+    __nanosleep(64);
+  }
+  return true;
+}
 
 // Programmatic dependent launch.  A kernel launched with programmatic
 // stream serialization may start before the previous kernel on its stream has

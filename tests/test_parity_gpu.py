@@ -323,3 +323,58 @@ def test_chunk_mask_with_a_kv_cache_is_unsupported(cuda_lib):
     with pytest.raises(m.MonarchError) as e:
         m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, w.iters, chunk_frames=1)
     assert e.value.code == -4
+
+
+ONESTEP = [
+    WORKLOADS["chunk_4680_bf16_1step"],
+    _custom("f16", 5, 12, 20, 64, 4, 4, 1),
+    _custom("bf16", 3, 12, 21, 64, 3, 7, 1),
+    _custom("bf16", 7, 12, 20, 128, 4, 4, 1, C=3),
+]
+
+
+@pytest.mark.parametrize("w", ONESTEP, ids=[w.name for w in ONESTEP])
+def test_one_step_kernel_equals_the_two_kernel_forward(w, cuda_lib, monkeypatch):
+    """iters = 1 runs the R step and the output pass as two kernels, or, with
+    MONARCH_ONESTEP_KERNEL=1, as one kernel whose output items wait for the
+    R-step items of their head; the training forward runs the same arithmetic
+    as two kernels and also keeps the row LSE.  The three outputs agree bit
+    for bit."""
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    outs = [torch.full(q.shape, float("nan"), dtype=torch.float32, device=q.device) for _ in range(3)]
+    lse = torch.empty(m.lse_numel(w.B, w.heads, w.T, w.H, w.W, w.d, w.th, w.tw), dtype=torch.float32,
+                      device=q.device)
+    m.profile_enable(True)
+    m.profile_read(reset=True)
+    for fused, out in ((True, outs[0]), (False, outs[1])):
+        if fused:
+            monkeypatch.setenv("MONARCH_ONESTEP_KERNEL", "1")
+        else:
+            monkeypatch.delenv("MONARCH_ONESTEP_KERNEL", raising=False)
+        m.monarch_attn_fwd(q, k, v, out, w.T, w.H, w.W, w.th, w.tw, 1, chunk_frames=w.chunk_frames)
+        torch.cuda.synchronize()
+        prof = m.profile_read(reset=True)
+        if fused:
+            assert prof["onestep"][1] == 1 and prof["r_step"][1] == 0 and prof["l_out"][1] == 0
+        else:
+            assert prof["onestep"][1] == 0 and prof["r_step"][1] == 1 and prof["l_out"][1] == 1
+    m.profile_enable(False)
+    m.monarch_attn_fwd_train(q, k, v, outs[2], lse, w.T, w.H, w.W, w.th, w.tw, chunk_frames=w.chunk_frames)
+    torch.cuda.synchronize()
+    assert m.device_error() == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[1], outs[2])
+
+
+def test_one_step_kernel_with_a_kv_cache(cuda_lib, monkeypatch):
+    """The single one-step kernel on a KV-cache step (the mean-query kernel
+    runs first, cached tiles start from it) equals the two-kernel call bit for
+    bit and the oracle within the bar."""
+    w = _custom("bf16", 2, 12, 20, 128, 4, 4, 1, Tk=5)
+    q, k, v = make_inputs(w)
+    monkeypatch.setenv("MONARCH_ONESTEP_KERNEL", "1")
+    a = _run_gpu(w, q, k, v)
+    monkeypatch.delenv("MONARCH_ONESTEP_KERNEL")
+    b = _run_gpu(w, q, k, v)
+    assert m.device_error() == 0
+    assert torch.equal(a, b)
+    _compare(w, a, q, k, v)
