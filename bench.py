@@ -99,6 +99,11 @@ def work_model(w):
         "r_step": dict(flops=BH * (2 * w.iters + 1) * FR / w.iters,
                        bytes=(3 * (w.iters - 1) * nk + 5 * nk) / w.iters + hb),
         "qbar": dict(flops=0.0, bytes=nq),
+        # one refinement step in one kernel: R step (scores, k~, z) and output
+        # pass; its compulsory bytes are the call's q, k, v in and out
+        "onestep": dict(flops=BH * (3 * FR + 2 * FL), bytes=nq + 2 * nk + no),
+        # LSE and column passes in one kernel: q, k~, h in; q~ out
+        "l_lsecol": dict(flops=BH * 2 * FL, bytes=nq + nk + hb + nk),
     }
     # compulsory call bytes: Q, K, V in and O out, all in the input dtype
     # (the output is written as f32 by default, which adds nq bytes; the

@@ -247,7 +247,10 @@ enum {
    * is "1" at the call (the default runs the two kernels, which is faster on
    * B200; both give the same values bit for bit) */
   MONARCH_PHASE_ONESTEP = 9,
-  MONARCH_NUM_PHASES = 10
+  /* a non-final L step with at most 256 query and 256 key tiles: the LSE
+   * pass and the column pass in one kernel, operands kept on chip */
+  MONARCH_PHASE_L_LSECOL = 10,
+  MONARCH_NUM_PHASES = 11
 };
 
 /* Number of kernels this process has launched through the library (host
@@ -277,7 +280,8 @@ const char* monarch_attn_last_error(void);
 
 /* ABI version (major*100 + minor): 1.02 adds the backward (monarch_attn_bwd),
  * the training pair and monarch_attn_fwd_host_ex to the forward of 1.00; 1.03
- * adds MONARCH_PHASE_ONESTEP (one refinement step as one kernel, on request). */
+ * adds MONARCH_PHASE_ONESTEP (one refinement step as one kernel, on request)
+ * and MONARCH_PHASE_L_LSECOL. */
 int monarch_attn_version(void);
 
 #ifdef __cplusplus

@@ -14,7 +14,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libmonarch_attn.so")
 
 MONARCH_F32, MONARCH_BF16, MONARCH_F16 = 0, 1, 2
-PHASES = ("qbar", "r_step", "l_lse", "l_out", "l_col", "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r", "onestep")
+PHASES = ("qbar", "r_step", "l_lse", "l_out", "l_col", "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r", "onestep",
+          "l_lsecol")
 
 # Every symbol the header declares, with its ctypes signature.
 _SIGS = {

@@ -22,6 +22,7 @@
 #include "kernels_rtc.cuh"
 #include "kernels_l.cuh"
 #include "kernels_onestep.cuh"
+#include "kernels_lsecol.cuh"
 #include "kernels_bwd.cuh"
 #include "kernels_bwd_tc.cuh"
 
@@ -100,7 +101,7 @@ void launch(int phase, cudaStream_t st, F&& f) {
   g_launches.fetch_add(1, std::memory_order_relaxed);
   if (debug_sync()) {
     static const char* names[] = {"qbar", "r_step", "l_lse", "l_out", "l_col",
-                                  "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r", "onestep"};
+                                  "bwd_prep", "bwd_dq", "bwd_dkv", "bwd_r", "onestep", "l_lsecol"};
     fprintf(stderr, "[monarch] launch %s ...\n", names[phase]);
     auto t0 = std::chrono::steady_clock::now();
     f();
@@ -412,6 +413,10 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_col = tc::col_smem<D>();
   constexpr size_t smem_r = rtc_smem<D>();
+  constexpr size_t smem_lc = tc::LsecolLayout<D>::smem();
+  // at most 256 query and 256 key tiles: a non-final L step is one kernel
+  // (l_lsecol) that keeps its operands on chip for both of its passes
+  const bool small_l = g.b1q <= 2 * kTile && g.b1k <= 2 * kTile;
 
   static std::atomic<bool> attrs_set[kMaxDevices];
   {
@@ -420,6 +425,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
       if ((r = allow_smem(tc::l_lse<D>, smem_lse)) != cudaSuccess ||
           (r = allow_smem(tc::l_row<__half, TO, D, true>, smem_out)) != cudaSuccess ||
           (r = allow_smem(tc::l_col<TQ, D>, smem_col)) != cudaSuccess ||
+          (r = allow_smem(tc::l_lsecol<TQ, D>, smem_lc)) != cudaSuccess ||
           (r = allow_smem(r_step_tc5<TQ, D>, smem_r)) != cudaSuccess)
         return r;
       return cudaSuccess;
@@ -466,7 +472,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
         launch(MONARCH_PHASE_QBAR, st, [&] {
           launch_pdl(qbar_kernel<TQ>, dim3(g.b2, g.BH), dim3(kQbarThreads), 0, st, q, w.qbar, g);
         });
-    } else {
+    } else if (!small_l) {
       launch(MONARCH_PHASE_L_COL, st, [&] {
         launch_pdl(tc::l_col<TQ, D>, grid_k, dim3(tc::kThreads), smem_col, st, maps, (const float*)w.h,
                    reinterpret_cast<TQ*>(w.qt), g);
@@ -479,6 +485,11 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
         launch_pdl(tc::l_row<__half, TO, D, true>, grid_q, dim3(tc::kThreads), smem_out, st, out, maps, w.lse, g);
+      });
+    } else if (small_l) {
+      launch(MONARCH_PHASE_L_LSECOL, st, [&] {
+        launch_pdl(tc::l_lsecol<TQ, D>, dim3(g.b2, g.BH), dim3(tc::kThreads), smem_lc, st, maps, w.lse,
+                   reinterpret_cast<TQ*>(w.qt), g);
       });
     } else {
       launch(MONARCH_PHASE_L_LSE, st, [&] {
