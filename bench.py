@@ -42,8 +42,11 @@ L2_BYTES = 126 * 2**20
 # scaled to the workload's heads where the capture used fewer (profiles/);
 # a kernel without a capture of its current code reports null.
 NCU_TRAFFIC = {
-    ("full_32760_bf16", "l_col"): 877.8e6,   # 292.6 MB at 8 heads x 3
-    ("chunk_4680_bf16", "r_step"): 48.2e6,   # mean of the call's two launches (30.2 and 66.2 MB)
+    ("chunk_4680_bf16", "r_step"): 47.77e6,     # mean of the call's two launches (30.44 and 65.10 MB)
+    ("chunk_4680_bf16", "l_lsecol"): 43.82e6,
+    ("chunk_4680_bf16", "l_out"): 75.62e6,
+    ("full_32760_bf16", "l_col"): 875.9e6,      # 291.96 MB at 8 heads x 3
+    ("full_32760_bf16", "l_lse"): 418.1e6,      # 139.36 MB at 8 heads x 3
 }
 # FP32 FMA ceiling of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz
 ALU_F32_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
