@@ -281,6 +281,7 @@ CAUSAL = [
     _custom("f16", 6, 16, 16, 64, 8, 8, 2, C=2),            # 64-position tiles
     _custom("bf16", 4, 9, 10, 128, 3, 5, 2, C=2),           # b2 not a multiple of 8
     _custom("f32", 5, 8, 12, 64, 2, 4, 2, C=2),             # CUDA-core path
+    _custom("bf16", 20, 12, 20, 128, 4, 4, 2, C=3, B=1, heads=2),   # 300 tiles: separate LSE and column kernels
 ]
 
 

@@ -164,6 +164,9 @@ INTER = [
     _custom("bf16", 3, 12, 20, 128, 4, 4, 2, B=1, heads=2),
     _custom("f16", 3, 12, 20, 64, 3, 5, 2, B=1, heads=2),
     _custom("bf16", 2, 12, 20, 128, 4, 4, 2, Tk=4, B=1, heads=2),
+    # more than 256 key tiles: the separate LSE and column kernels
+    _custom("bf16", 1, 12, 20, 128, 4, 4, 2, Tk=18, B=1, heads=2),
+    _custom("f16", 18, 12, 20, 64, 4, 4, 2, B=1, heads=1),
 ]
 
 
