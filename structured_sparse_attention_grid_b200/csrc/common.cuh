@@ -29,6 +29,11 @@ struct Geo {
   long long Nq, Nk;
   float sl2;     // s * log2(e), s = 1/sqrt(d)
   int cq;        // key/query tiles per frame-chunk of the causal mask; 0 = no mask
+  // Stacked positions (L step of small grids): pk positions of a head share
+  // one row block, position p's tiles at rows [p pb1, (p + 1) pb1), so b2,
+  // b1q, b1k above count stacked positions and rows; pb1q, pb1k are one
+  // position's tiles.  pk = 1: no stacking.
+  int pk, pb1q, pb1k;
 };
 
 // Frame-chunk causal mask (self-attention, chunks of C frames, cq = C * P
@@ -39,6 +44,30 @@ __device__ __forceinline__ int key_limit(const Geo& g, int a1) {
   return g.cq ? min(g.b1k, (a1 / g.cq + 1) * g.cq) : g.b1k;
 }
 __device__ __forceinline__ int query_start(const Geo& g, int c1) { return g.cq ? (c1 / g.cq) * g.cq : 0; }
+
+// The key rows that query row a1 sees: [lo, hi).  With stacked positions,
+// the keys of the row's own position (and its causal window there).
+__device__ __forceinline__ void row_keys(const Geo& g, int a1, int& lo, int& hi) {
+  if (g.pk == 1) {
+    lo = 0;
+    hi = key_limit(g, a1);
+    return;
+  }
+  const int p = a1 / g.pb1q, a = a1 - p * g.pb1q;
+  lo = p * g.pb1k;
+  hi = lo + (g.cq ? min(g.pb1k, (a / g.cq + 1) * g.cq) : g.pb1k);
+}
+// The query rows that see key row c1: [lo, hi).
+__device__ __forceinline__ void col_queries(const Geo& g, int c1, int& lo, int& hi) {
+  if (g.pk == 1) {
+    lo = query_start(g, c1);
+    hi = g.b1q;
+    return;
+  }
+  const int p = c1 / g.pb1k, c = c1 - p * g.pb1k;
+  lo = p * g.pb1q + (g.cq ? (c / g.cq) * g.cq : 0);
+  hi = (p + 1) * g.pb1q;
+}
 
 // Token index (within one head) of tile c1, position c2.
 __device__ __forceinline__ long long token_of(const Geo& g, int c1, int c2) {

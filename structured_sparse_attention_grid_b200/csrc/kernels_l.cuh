@@ -113,8 +113,10 @@ __device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& map
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int zrow = bh * g.b2 + a2;
   const int plane_rows = g.BH * g.b2;
-  // key blocks any row of this CTA sees (all of them without a causal mask)
-  const int kmax = key_limit(g, min(a1_base + 2 * kTile, g.b1q) - 1);
+  // key blocks any row of this CTA sees (all of them without a causal mask);
+  // the last row's window ends highest
+  int klast_lo, kmax;
+  row_keys(g, min(a1_base + 2 * kTile, g.b1q) - 1, klast_lo, kmax);
   const int nkb = (kmax + kBlk - 1) / kBlk;
   const int ntiles = (g.b1q - a1_base > kTile) ? 2 : 1;
 
@@ -264,7 +266,8 @@ __device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& map
     const int r = 32 * (warp & 3) + lane;
     const uint32_t lane_off = (uint32_t)(32 * (warp & 3)) << 16;
     const int a1 = a1_base + t * kTile + r;
-    const int rowlim = key_limit(g, min(a1, g.b1q - 1));   // visible key tiles [0, rowlim)
+    int klo, khi;   // visible key rows [klo, khi)
+    row_keys(g, min(a1, g.b1q - 1), klo, khi);
     if (t < ntiles) {
       float m = -INFINITY, l = 0.f;
       float lx = 0.f;   // LSE_OUT: the row sum of the unrounded exponentials
@@ -304,12 +307,13 @@ __device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& map
           ptx::mbar_arrive(k_free + ks);
           if (!OUT) ptx::mbar_arrive(s_free + 2 * t + b);
         }
-        const int valid = min(kBlk, rowlim - j * kBlk) - 32 * hf;   // keys of this half (may be <= 0)
-        if (valid < 32) {  // only the last block of a ragged row
+        // this half's visible keys are [vlo, vhi) of its 32
+        const int vlo = klo - (j * kBlk + 32 * hf), vhi = khi - (j * kBlk + 32 * hf);
+        if (vlo > 0 || vhi < 32) {  // a ragged row end, or stacked positions
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            if (2 * i >= valid) x[i].x = -INFINITY;
-            if (2 * i + 1 >= valid) x[i].y = -INFINITY;
+            if (2 * i < vlo || 2 * i >= vhi) x[i].x = -INFINITY;
+            if (2 * i + 1 < vlo || 2 * i + 1 >= vhi) x[i].y = -INFINITY;
           }
         }
         float mb = -INFINITY;
@@ -398,7 +402,10 @@ __device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& map
         ok = ok && ptx::mbar_wait(o_done + t, 0);
         ptx::tc_fence_after();
         const float inv = 1.f / lt;
-        TO* orow = out + ((long long)bh * g.Nq + (a1 < g.b1q ? token_of(g, a1, a2) : 0)) * D + hf * (D / 2);
+        // row a1 of stacked position p: tile a1 mod pb1q of position a2 pk + p
+        const int sp = a1 / g.pb1q;
+        const long long tok = a1 < g.b1q ? token_of(g, a1 - sp * g.pb1q, a2 * g.pk + sp) : 0;
+        TO* orow = out + ((long long)bh * g.Nq + tok) * D + hf * (D / 2);
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[16];

@@ -203,7 +203,8 @@ l_lsecol(const __grid_constant__ Maps maps, float* __restrict__ lse, TQ* __restr
     // ------------------------------------------------- phase A: row LSE
     if (t < nq) {
       const int a1 = t * kTile + r;
-      const int rowlim = key_limit(g, min(a1, g.b1q - 1));   // visible key tiles [0, rowlim)
+      int klo, khi;   // visible key rows [klo, khi)
+      row_keys(g, min(a1, g.b1q - 1), klo, khi);
       float m = -INFINITY, l = 0.f;
       for (int b = 0; b < nk; ++b) {
         ok = ok && ptx::mbar_wait(s_full + 2 * t + b, 0) && ptx::mbar_wait(k_full + b, 0);
@@ -223,12 +224,14 @@ l_lsecol(const __grid_constant__ Maps maps, float* __restrict__ lse, TQ* __restr
             x[2 * i + 1] = fma2(make_float2(__uint_as_float(s[4 * i + 2]), __uint_as_float(s[4 * i + 3])), sl2,
                                 make_float2(h4.z, h4.w));
           }
-          const int valid = min(kTile, rowlim - b * kTile) - 64 * hf - 32 * sb;
-          if (valid < 32) {
+          // these 32 keys' visible part is [vlo, vhi)
+          const int kb0 = b * kTile + 64 * hf + 32 * sb;
+          const int vlo = klo - kb0, vhi = khi - kb0;
+          if (vlo > 0 || vhi < 32) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              if (2 * i >= valid) x[i].x = -INFINITY;
-              if (2 * i + 1 >= valid) x[i].y = -INFINITY;
+              if (2 * i < vlo || 2 * i >= vhi) x[i].x = -INFINITY;
+              if (2 * i + 1 < vlo || 2 * i + 1 >= vhi) x[i].y = -INFINITY;
             }
           }
           float mb = -INFINITY;
@@ -274,15 +277,16 @@ l_lsecol(const __grid_constant__ Maps maps, float* __restrict__ lse, TQ* __restr
       // by other warps before a_done): wait on both barriers itself
       ok = ok && ptx::mbar_wait(k_full + t, 0) && ptx::mbar_wait(a_done, 0);
       const int c1 = t * kTile + r;
-      const int qstart = query_start(g, min(c1, g.b1k - 1));   // queries [qstart, b1q) see this tile
+      int qlo, qhi;   // the query rows that see this key row: [qlo, qhi)
+      col_queries(g, min(c1, g.b1k - 1), qlo, qhi);
       const float hb = (c1 < g.b1k) ? sH[c1] + kColShift : 0.f;
       const float2 hb2 = make_float2(hb, hb);
       float2 beta2 = make_float2(0.f, 0.f);
       for (int i = 0; i < nq; ++i) {
         ok = ok && ptx::mbar_wait(t_full + t, i & 1);
         ptx::tc_fence_after();
-        const int valid = min(kTile, g.b1q - i * kTile);
-        const int vlo = qstart - i * kTile;   // queries of this block below it are masked
+        const int valid = min(kTile, qhi - i * kTile);   // queries of this block at or past it are masked
+        const int vlo = qlo - i * kTile;                   // and those below this
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {      // 32 queries at a time
           const int cb = 64 * hf + 32 * hh;   // first S^T column (query) of this chunk

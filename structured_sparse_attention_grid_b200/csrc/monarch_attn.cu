@@ -200,6 +200,9 @@ int make_plan(int B, int heads, int T, int H, int W, int d, int th, int tw, int 
                 "the frame-chunk causal mask is for self-attention (kv_len == T*H*W); with a KV cache the "
                 "query chunk is the newest and sees every key");
   g.cq = (chunk_frames > 0 && chunk_frames < T) ? chunk_frames * g.P : 0;   // C >= T: one chunk, no mask
+  g.pk = 1;
+  g.pb1q = g.b1q;
+  g.pb1k = g.b1k;
   p->dtype = dtype;
   p->out_dtype = out_dtype;
   p->iters = iters;
@@ -329,16 +332,32 @@ int sm_count_of_device() {
   return v;
 }
 
-// Workspace views and tensor maps of the tensor-core forward (shared by the
-// forward and the backward's recompute).
-template <typename TQ, int D>
-int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& w, TcPlanes<TQ>& planes,
-               tc::Maps& maps, RtcMaps& rmaps) {
-  planes.kt_hi = reinterpret_cast<__half*>(w.kt);
-  planes.z_hi = reinterpret_cast<__half*>(w.z);
-  planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
-  const CUtensorMapDataType dq =
-      TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+// Geometry of the L-step kernels.  On small self-attention grids (one
+// position's problem is b1 x b1 with b1 a multiple of 4 that divides 128) the
+// L step stacks pk = 128 / b1 positions of a head in one 128-row block, each
+// row seeing only its own position's keys (row_keys / col_queries): one CTA
+// then does pk positions' work, where each would otherwise fill a 128-row
+// tensor-core tile with b1 rows.  Positions are contiguous in every
+// position-major buffer ([BH][b2][b1][d] and the padded h and LSE rows, whose
+// padding is zero when b1 is a multiple of 4), so the stacked geometry views
+// the same memory.
+Geo stacked_geometry(const Geo& g) {
+  Geo s = g;
+  const int b1 = g.b1q;
+  if (g.Tk != g.T || g.b1k != b1 || b1 % 4 || b1 >= kTile || kTile % b1) return s;
+  const int pk = kTile / b1;
+  if (g.b2 % pk) return s;
+  s.pk = pk;
+  s.pb1q = s.pb1k = b1;
+  s.b2 = g.b2 / pk;
+  s.b1q = s.b1k = s.b1q_pad = s.b1k_pad = kTile;
+  return s;
+}
+
+// Tensor maps of the L-step kernels (block-major q copy, k~ and z planes, h,
+// row LSE) for geometry g, which may stack positions (stacked_geometry).
+template <int D>
+int tc_l_maps(const Geo& g, const Work& w, const __half* kt_hi, const __half* z_hi, tc::Maps& maps) {
   int rc;
   {
     const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
@@ -355,15 +374,30 @@ int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& 
     // the L step computes in f16: q (block-major copy) and the k~ planes are f16
     if ((rc = make_map(&maps.qb, w.qb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dq3, sq3, box3,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&maps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
+        (rc = make_map(&maps.kt, kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&maps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
+        (rc = make_map(&maps.z, z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dk3, sk3, box3,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&maps.h, w.h, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dh2, sh2, box2, CU_TENSOR_MAP_SWIZZLE_NONE)) ||
         (rc = make_map(&maps.lse, w.lse, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, dl2, sl2, box2,
                        CU_TENSOR_MAP_SWIZZLE_NONE)))
       return rc;
   }
+  return MONARCH_OK;
+}
+
+// Workspace views and tensor maps of the tensor-core forward (shared by the
+// forward and the backward's recompute).
+template <typename TQ, int D>
+int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& w, TcPlanes<TQ>& planes,
+               tc::Maps& maps, RtcMaps& rmaps) {
+  planes.kt_hi = reinterpret_cast<__half*>(w.kt);
+  planes.z_hi = reinterpret_cast<__half*>(w.z);
+  planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
+  const CUtensorMapDataType dq =
+      TcType<TQ>::kBf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  int rc;
+  if ((rc = tc_l_maps<D>(g, w, planes.kt_hi, planes.z_hi, maps))) return rc;
   // R-step maps: the key / value / query grids as (d, W, H, frames) with one
   // tile per box, and the q~ planes as (d, b1k, 2*BH*b2) with one key tile per box
   {
@@ -463,6 +497,10 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     if (e != cudaSuccess) return cuda_fail(e, "kernel launch");
     return MONARCH_OK;
   }
+  // the L-step kernels below run on the stacked geometry when it applies
+  const Geo gl = stacked_geometry(g);
+  if (gl.pk > 1 && (rc = tc_l_maps<D>(gl, w, planes.kt_hi, planes.z_hi, maps))) return rc;
+  const dim3 grid_ql((gl.b1q + 2 * kTile - 1) / (2 * kTile), gl.b2, gl.BH);
   for (int it = 0; it < p.iters; ++it) {
     const int final_step = it == p.iters - 1;
     int mode = QT_BUFFER;
@@ -484,12 +522,12 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
     });
     if (final_step) {
       launch(MONARCH_PHASE_L_OUT, st, [&] {
-        launch_pdl(tc::l_row<__half, TO, D, true>, grid_q, dim3(tc::kThreads), smem_out, st, out, maps, w.lse, g);
+        launch_pdl(tc::l_row<__half, TO, D, true>, grid_ql, dim3(tc::kThreads), smem_out, st, out, maps, w.lse, gl);
       });
     } else if (small_l) {
       launch(MONARCH_PHASE_L_LSECOL, st, [&] {
-        launch_pdl(tc::l_lsecol<TQ, D>, dim3(g.b2, g.BH), dim3(tc::kThreads), smem_lc, st, maps, w.lse,
-                   reinterpret_cast<TQ*>(w.qt), g);
+        launch_pdl(tc::l_lsecol<TQ, D>, dim3(gl.b2, gl.BH), dim3(tc::kThreads), smem_lc, st, maps, w.lse,
+                   reinterpret_cast<TQ*>(w.qt), gl);
       });
     } else {
       launch(MONARCH_PHASE_L_LSE, st, [&] {

@@ -112,6 +112,12 @@ EDGE = [
     _custom("f16", 2, 10, 15, 64, 5, 5, 3),
     _custom("bf16", 2, 9, 10, 128, 3, 5, 2, Tk=5),
     _custom("bf16", 3, 12, 21, 64, 3, 7, 1),
+    # small grids whose L step stacks positions: 32 tiles (four a block), 64
+    # tiles (two), 16 tiles (eight), with one, two and three iterations
+    _custom("f16", 2, 16, 16, 64, 4, 4, 2),
+    _custom("bf16", 4, 8, 8, 128, 2, 2, 1),
+    _custom("bf16", 1, 16, 32, 128, 4, 4, 2),
+    _custom("f16", 1, 16, 16, 64, 4, 4, 3),
 ]
 
 
@@ -282,6 +288,8 @@ CAUSAL = [
     _custom("bf16", 4, 9, 10, 128, 3, 5, 2, C=2),           # b2 not a multiple of 8
     _custom("f32", 5, 8, 12, 64, 2, 4, 2, C=2),             # CUDA-core path
     _custom("bf16", 20, 12, 20, 128, 4, 4, 2, C=3, B=1, heads=2),   # 300 tiles: separate LSE and column kernels
+    _custom("bf16", 4, 8, 16, 128, 2, 4, 2, C=2),          # 64 tiles, two positions stacked, masked
+    _custom("f16", 8, 8, 8, 64, 4, 4, 2, C=3),             # 32 tiles, four stacked, ragged last chunk
 ]
 
 

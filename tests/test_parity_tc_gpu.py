@@ -137,6 +137,10 @@ PROBE = [
     _custom("bf16", 2, 9, 10, 128, 3, 5, 2),
     _custom("f16", 4, 16, 16, 64, 4, 4, 2, Tk=6),
     _custom("f32", 3, 8, 12, 128, 2, 4, 2),
+    # small grids whose L step stacks positions (32 tiles: 4 a block; 64 tiles: 2)
+    _custom("f16", 2, 16, 16, 64, 4, 4, 2),
+    _custom("bf16", 4, 8, 8, 128, 2, 2, 2),
+    _custom("bf16", 4, 8, 8, 128, 2, 2, 1),
 ]
 
 
@@ -164,6 +168,8 @@ INTER = [
     _custom("bf16", 3, 12, 20, 128, 4, 4, 2, B=1, heads=2),
     _custom("f16", 3, 12, 20, 64, 3, 5, 2, B=1, heads=2),
     _custom("bf16", 2, 12, 20, 128, 4, 4, 2, Tk=4, B=1, heads=2),
+    # 32 tiles a head: the L step stacks four positions in one block
+    _custom("f16", 2, 16, 16, 64, 4, 4, 2, B=1, heads=2),
     # more than 256 key tiles: the separate LSE and column kernels
     _custom("bf16", 1, 12, 20, 128, 4, 4, 2, Tk=18, B=1, heads=2),
     _custom("f16", 18, 12, 20, 64, 4, 4, 2, B=1, heads=1),
