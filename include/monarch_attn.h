@@ -222,7 +222,8 @@ int monarch_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* 
  * (f32; in nats for f32 inputs, in bits, i.e. base-2 entropy, for bf16/f16
  * inputs), [4] row log2-sum-exp of the last non-final L step
  * [B*heads][b2][b1q_pad] (f32, base-2 logits s*log2(e)*q.k~ + log2(e)*h),
- * [5] KV-init mean query [B*heads][b2][d] (f32), [6] queries in block-major
+ * [5] KV-init mean query [B*heads][b2][d] (f32 for f32 inputs; otherwise a
+ * high and a low plane of the input type), [6] queries in block-major
  * order [B*heads][b2][b1q][d] (f16 for bf16/f16 inputs; absent for f32).
  * b1k_pad and b1q_pad are b1k and b1q rounded up to a multiple of 4.
  * Returns the total bytes, 0 on invalid arguments. */

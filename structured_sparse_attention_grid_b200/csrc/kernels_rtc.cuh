@@ -48,6 +48,7 @@ struct RtcMaps {
   CUtensorMap k;    // keys       {d, W, H, BH*Tk},       box {64, tw, th, 1}
   CUtensorMap v;    // values     {d, W, H, BH*Tk},       box {64, tw, th, 1}
   CUtensorMap qt;   // q~ planes  {d, b1k, 2*BH*b2},      box {64, 1, b2}
+  CUtensorMap qm;   // mean-query planes (KV init) {d, 1, 2*BH*b2}, box {64, 1, b2}
   CUtensorMap qb;   // block-major q, f16 (store) {d, b1q, BH*b2},   box {64, 1, b2}
   CUtensorMap kt;   // k~ planes, f16 (store)     {d, b1k, 2*BH*b2}, box {64, 1, b2}
   CUtensorMap z;    // z planes, f16 (store) {d, b1k, 2*BH*b2},   box {64, 1, b2}
@@ -109,7 +110,7 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
   uint8_t* sK = sA + 2 * NH * kRBox;       // [d half] boxes
   uint64_t* bar = reinterpret_cast<uint64_t*>(sK + NH * kRBox);
   uint64_t* bar_ld = bar + 0;    // TMA: keys and query rows
-  uint64_t* bar_a = bar + 1;     // row warps: query rows written by threads (KV init)
+  // bar + 1: unused
   uint64_t* bar_s = bar + 2;     // MMA: S complete
   uint64_t* bar_r = bar + 3;     // row warps: R in TMEM
   uint64_t* bar_acc = bar + 4;   // MMA: k~ (phase 0), z (phase 1) complete
@@ -129,7 +130,6 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
 
   if (tid == kRtcRowThreads) {
     ptx::mbar_init(bar_ld, 1);
-    ptx::mbar_init(bar_a, 8);
     ptx::mbar_init(bar_s, 1);
     ptx::mbar_init(bar_r, 8);
     ptx::mbar_init(bar_acc, 1);
@@ -138,16 +138,21 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
     ptx::mbar_init(bar_q, 8);
     ptx::fence_mbar_init();
   }
+  auto exact_q = [&](int c1) { return mode == QT_IDENTITY || (mode == QT_KVINIT && c1 >= g.off); };
   // Zero every row that no load writes (in-tile padding, tiles past the end):
   // K and V rows there meet zero R entries, and 0 * NaN would not be zero.
+  // With a KV cache the score MMA reads the A lo plane, which the exact query
+  // rows leave unwritten: zero it there too.
   for (int i = tid; i < kRtcRows * NH * 8; i += kRtcThreads) {
     const int row = i / (NH * 8), rem = i - row * (NH * 8), hf = rem >> 3, ch = rem & 7;
     const int gg = row / rs, a = row - gg * rs;
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    const uint32_t o = hf * kRBox + row * 128 + ch * 16;
     if (gg >= Gn || a >= g.b2) {
-      const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-      const uint32_t o = hf * kRBox + row * 128 + ch * 16;
       *reinterpret_cast<uint4*>(sK + o) = z4;
       *reinterpret_cast<uint4*>(sA + o) = z4;
+      *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = z4;
+    } else if (mode == QT_KVINIT && exact_q(c1_0 + gg)) {
       *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = z4;
     }
   }
@@ -166,7 +171,6 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
     y0 = ty * g.th;
     x0 = (rem - ty * g.ntx) * g.tw;
   };
-  auto exact_q = [&](int c1) { return mode == QT_IDENTITY || (mode == QT_KVINIT && c1 >= g.off); };
 
   if (warp == kRtcRowThreads / 32) {
     if (lane == 0) {
@@ -181,7 +185,8 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
       uint32_t bytes = 0;
       for (int gg = 0; gg < Gn; ++gg) {
         const int c1 = c1_0 + gg;
-        const int planes = mode == QT_BUFFER ? 2 : (exact_q(c1) ? 1 : 0);
+        // q~ planes, or the exact query rows, or (cached tiles) the mean-query planes
+        const int planes = (mode == QT_BUFFER || !exact_q(c1)) ? 2 : 1;
         bytes += (uint32_t)(NH * g.b2 * 128 * (1 + planes));
       }
       ptx::mbar_expect_tx(bar_ld, bytes);
@@ -201,6 +206,12 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
           const int tq = t - (g.Tk - g.T);   // the aligned query frame (== t without a cache)
           for (int hf = 0; hf < NH; ++hf)
             ptx::tma_load_4d(sA + hf * kRBox + row0, &maps.q, bar_ld, hf * 64, x0, y0, bh * g.T + tq);
+        } else {
+          // a cached tile (KV init): the mean query of each position, hi and lo
+          for (int p = 0; p < 2; ++p)
+            for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_load_3d(sA + (p * NH + hf) * kRBox + row0, &maps.qm, bar_ld, hf * 64, 0,
+                               (p * g.BH + bh) * g.b2);
         }
       }
       ok = ptx::mbar_wait(bar_ld, 0);
@@ -216,7 +227,6 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
         }
         ptx::bulk_commit();
       }
-      if (mode == QT_KVINIT) ok = ok && ptx::mbar_wait(bar_a, 0);
       ptx::tc_fence_after();
       // S = A K^T: both operands K-major (d along the 128-byte rows)
       if (ok) {
@@ -286,33 +296,6 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
     constexpr int kSeg = NH * 4;                // 16-byte chunks of a row per half
     bool ok = true;
 
-    if (mode == QT_KVINIT) {
-      // rows no load brings: cached tiles take the mean query (split into hi /
-      // lo), the lo plane of exact rows is zero
-      if (valid) {
-        const bool ex = exact_q(c1);
-        const float* qm = w.qbar + ((long long)bh * g.b2 + a2) * D;
-#pragma unroll
-        for (int k = 0; k < kSeg; ++k) {
-          const int i = half * kSeg + k, hf = i >> 3, ch = i & 7;
-          uint4 hi4 = make_uint4(0u, 0u, 0u, 0u), lo4 = make_uint4(0u, 0u, 0u, 0u);
-          if (!ex) {
-            const float4 u = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8);
-            const float4 v4 = *reinterpret_cast<const float4*>(qm + hf * 64 + ch * 8 + 4);
-            tc::split2<TQ>(make_float2(u.x, u.y), hi4.x, lo4.x);
-            tc::split2<TQ>(make_float2(u.z, u.w), hi4.y, lo4.y);
-            tc::split2<TQ>(make_float2(v4.x, v4.y), hi4.z, lo4.z);
-            tc::split2<TQ>(make_float2(v4.z, v4.w), hi4.w, lo4.w);
-          }
-          const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
-          if (!ex) *reinterpret_cast<uint4*>(sA + o) = hi4;
-          *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = lo4;
-        }
-      }
-      ptx::fence_proxy_async();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(bar_a);
-    }
 
     // First step, bf16 input: the L step reads q in f16 (exact for |q| <
     // 65504; larger finite magnitudes set kErrRange).  The loaded rows are

@@ -15,12 +15,15 @@ namespace monarch {
 // tiles in the first R step of a KV-cache call.  grid (b2, BH), block
 // kQbarThreads: thread (group, pair) sums column pair `pair` over the query
 // tiles group, group + groups, ... (a warp reads 32 consecutive pairs of one
-// token row), then the groups are added in shared memory.
+// token row), then the groups are added in shared memory.  Output: f32
+// [BH][b2][d] for f32 inputs; for bf16 / f16 inputs the tensor-core R step's
+// A operand, a high plane round(m) and a low plane round(m - high) of the
+// input type, [2][BH][b2][d] (the same bytes).
 constexpr int kQbarThreads = 512;
 
 template <typename T>
 __global__ void __launch_bounds__(kQbarThreads)
-qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, Geo g) {
+qbar_kernel(const T* __restrict__ q, void* __restrict__ qbar, Geo g) {
   __shared__ float2 part[kQbarThreads];
   ptx::griddep_launch();
   ptx::griddep_wait();
@@ -44,9 +47,20 @@ qbar_kernel(const T* __restrict__ q, float* __restrict__ qbar, Geo g) {
       acc.y += o.y;
     }
     const float inv = 1.f / (float)g.b1q;
-    float* dst = qbar + ((long long)bh * g.b2 + a2) * g.d + 2 * pair;
-    dst[0] = acc.x * inv;
-    dst[1] = acc.y * inv;
+    const long long o = ((long long)bh * g.b2 + a2) * g.d + 2 * pair;
+    const float m0 = acc.x * inv, m1 = acc.y * inv;
+    if constexpr (sizeof(T) == 4) {
+      float* dst = static_cast<float*>(qbar) + o;
+      dst[0] = m0;
+      dst[1] = m1;
+    } else {
+      T* hi = static_cast<T*>(qbar) + o;
+      T* lo = hi + (long long)g.BH * g.b2 * g.d;
+      hi[0] = from_f<T>(m0);
+      hi[1] = from_f<T>(m1);
+      lo[0] = from_f<T>(m0 - to_f(hi[0]));
+      lo[1] = from_f<T>(m1 - to_f(hi[1]));
+    }
   }
 }
 

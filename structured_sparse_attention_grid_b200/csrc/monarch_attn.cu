@@ -408,10 +408,14 @@ int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& 
     cuuint32_t boxt[3] = {64, 1, (cuuint32_t)g.b2};
     cuuint64_t dt3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1k, 2 * (cuuint64_t)g.BH * g.b2};
     cuuint64_t st3[2] = {(cuuint64_t)D * 2, (cuuint64_t)g.b1k * D * 2};
+    // the mean-query planes of the KV-init step: [2][BH][b2][d], one "tile"
+    cuuint64_t dm3[3] = {(cuuint64_t)D, 1, 2 * (cuuint64_t)g.BH * g.b2};
+    cuuint64_t sm3[2] = {(cuuint64_t)D * 2, (cuuint64_t)D * 2};
     if ((rc = make_map(&rmaps.q, q, dq, 4, dq4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.k, k, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.v, v, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.qt, w.qt, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.qm, w.qbar, dq, 3, dm3, sm3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
