@@ -13,53 +13,66 @@ namespace monarch {
 // ---------------------------------------------------------------------------
 // Mean query per (head, position) over all query tiles: the q~ of cached key
 // tiles in the first R step of a KV-cache call.  grid (b2, BH), block
-// kQbarThreads: thread (group, pair) sums column pair `pair` over the query
-// tiles group, group + groups, ... (a warp reads 32 consecutive pairs of one
-// token row), then the groups are added in shared memory.  Output: f32
-// [BH][b2][d] for f32 inputs; for bf16 / f16 inputs the tensor-core R step's
-// A operand, a high plane round(m) and a low plane round(m - high) of the
-// input type, [2][BH][b2][d] (the same bytes).
+// kQbarThreads.  The token offsets of the position's query tiles are computed
+// once into shared memory; then thread (group, quad) sums the four columns
+// `quad` over the query tiles group, group + groups, ... (a warp reads 32
+// consecutive 4-column pieces of one token row), and the groups are added in
+// shared memory.  Output: f32 [BH][b2][d] for f32 inputs; for bf16 / f16
+// inputs the tensor-core R step's A operand, a high plane round(m) and a low
+// plane round(m - high) of the input type, [2][BH][b2][d] (the same bytes).
 constexpr int kQbarThreads = 512;
+constexpr int kQbarMaxTiles = 4096;   // query tiles whose offsets fit the shared table
 
 template <typename T>
 __global__ void __launch_bounds__(kQbarThreads)
 qbar_kernel(const T* __restrict__ q, void* __restrict__ qbar, Geo g) {
-  __shared__ float2 part[kQbarThreads];
+  __shared__ float4 part[kQbarThreads];
+  __shared__ long long tok[kQbarMaxTiles];   // token offsets (elements) of this position's query tiles
   ptx::griddep_launch();
   ptx::griddep_wait();
   const int a2 = blockIdx.x, bh = blockIdx.y;
-  const int npair = g.d / 2, groups = kQbarThreads / npair;
-  const int pair = threadIdx.x % npair, grp = threadIdx.x / npair;
-  const T* qh = q + (long long)bh * g.Nq * g.d + 2 * pair;
-  float2 acc = make_float2(0.f, 0.f);
+  const int nquad = g.d / 4, groups = kQbarThreads / nquad;
+  const int quad = threadIdx.x % nquad, grp = threadIdx.x / nquad;
+  const T* qh = q + (long long)bh * g.Nq * g.d + 4 * quad;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int base = 0; base < g.b1q; base += kQbarMaxTiles) {
+    const int n = min(kQbarMaxTiles, g.b1q - base);
+    __syncthreads();   // the previous chunk's offsets are read
+    for (int i = threadIdx.x; i < n; i += kQbarThreads) tok[i] = token_of(g, base + i, a2) * g.d;
+    __syncthreads();
 #pragma unroll 4
-  for (int a1 = grp; a1 < g.b1q; a1 += groups) {
-    const T* p = qh + token_of(g, a1, a2) * g.d;
-    acc.x += to_f(p[0]);
-    acc.y += to_f(p[1]);
+    for (int i = grp; i < n; i += groups) {
+      const T* p = qh + tok[i];
+      if constexpr (sizeof(T) == 4) {
+        const float4 x = *reinterpret_cast<const float4*>(p);
+        acc.x += x.x; acc.y += x.y; acc.z += x.z; acc.w += x.w;
+      } else {
+        const uint2 x = *reinterpret_cast<const uint2*>(p);
+        const T* e = reinterpret_cast<const T*>(&x);
+        acc.x += to_f(e[0]); acc.y += to_f(e[1]); acc.z += to_f(e[2]); acc.w += to_f(e[3]);
+      }
+    }
   }
   part[threadIdx.x] = acc;
   __syncthreads();
   if (grp == 0) {
     for (int i = 1; i < groups; ++i) {
-      const float2 o = part[i * npair + pair];
-      acc.x += o.x;
-      acc.y += o.y;
+      const float4 o = part[i * nquad + quad];
+      acc.x += o.x; acc.y += o.y; acc.z += o.z; acc.w += o.w;
     }
     const float inv = 1.f / (float)g.b1q;
-    const long long o = ((long long)bh * g.b2 + a2) * g.d + 2 * pair;
-    const float m0 = acc.x * inv, m1 = acc.y * inv;
+    const long long o = ((long long)bh * g.b2 + a2) * g.d + 4 * quad;
+    const float m[4] = {acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv};
     if constexpr (sizeof(T) == 4) {
       float* dst = static_cast<float*>(qbar) + o;
-      dst[0] = m0;
-      dst[1] = m1;
+      for (int e = 0; e < 4; ++e) dst[e] = m[e];
     } else {
       T* hi = static_cast<T*>(qbar) + o;
       T* lo = hi + (long long)g.BH * g.b2 * g.d;
-      hi[0] = from_f<T>(m0);
-      hi[1] = from_f<T>(m1);
-      lo[0] = from_f<T>(m0 - to_f(hi[0]));
-      lo[1] = from_f<T>(m1 - to_f(hi[1]));
+      for (int e = 0; e < 4; ++e) {
+        hi[e] = from_f<T>(m[e]);
+        lo[e] = from_f<T>(m[e] - to_f(hi[e]));
+      }
     }
   }
 }
