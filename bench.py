@@ -409,7 +409,9 @@ def run_ours(args, rank, world, device):
     e2e_ms = max_over_ranks(statistics.median(e2e_times), world, device)
     del qh, kh, vh, oh
 
-    configs = extra_configs(m, args, device, stream, flush_buf, peaks, world) if not args.no_configs else {}
+    # the per-configuration timings are single-GPU figures: one run (N = 1) gives them
+    configs = extra_configs(m, args, device, stream, flush_buf, peaks, world) \
+        if (world == 1 and not args.no_configs) else {}
 
     es = q.element_size()
     rec = {
