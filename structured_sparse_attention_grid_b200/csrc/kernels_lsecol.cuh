@@ -15,7 +15,10 @@
 // acc += L^T_hi q + L^T_lo q, then q~ = acc / beta as hi / lo planes of the
 // input type.  Every query block and key tile is loaded once, by TMA, at the
 // start; the two passes share the operands (q is the A operand of phase A and
-// the B operand of phase B, both K-major and, for L^T q, MN-major).
+// the B operand of phase B, both K-major and, for L^T q, MN-major).  On the
+// stacked geometry of the smallest grids (several positions of a head in one
+// 128-row block) each row's window of keys, or each key row's window of
+// queries, is its own position's (row_keys, col_queries).
 //
 // TMEM (512 columns).  Phase A: S(query tile t, key block b) at 256 t + 128 b,
 // all four issued at once.  Phase B: key tile t at 256 t, S^T in [0, 128)
