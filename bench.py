@@ -42,9 +42,9 @@ L2_BYTES = 126 * 2**20
 # scaled to the workload's heads where the capture used fewer (profiles/);
 # a kernel without a capture of its current code reports null.
 NCU_TRAFFIC = {
-    ("chunk_4680_bf16", "r_step"): 47.77e6,     # mean of the call's two launches (30.44 and 65.10 MB)
-    ("chunk_4680_bf16", "l_lsecol"): 43.82e6,
-    ("chunk_4680_bf16", "l_out"): 75.62e6,
+    ("chunk_4680_bf16", "r_step"): 47.35e6,     # mean of the call's two launches (30.08 and 64.63 MB)
+    ("chunk_4680_bf16", "l_lsecol"): 43.84e6,
+    ("chunk_4680_bf16", "l_out"): 75.65e6,
     ("full_32760_bf16", "l_col"): 875.9e6,      # 291.96 MB at 8 heads x 3
     ("full_32760_bf16", "l_lse"): 418.1e6,      # 139.36 MB at 8 heads x 3
 }
@@ -277,6 +277,18 @@ def time_forward(m, w, qd, kd, vd, out, steps, warmup, stream, flush, world=1, c
     return [a.elapsed_time(b) for a, b in zip(starts, ends)], launches, step
 
 
+def keep_loaded(step, timed_ms, device, clocks, at_least_ms=1000.0):
+    """If the timed steps were short, keep the same calls running (untimed)
+    so that the clock sampler sees the GPU under that load for about a
+    second; the sampled window then ends here."""
+    if timed_ms < at_least_ms:
+        t_end = time.time() + (at_least_ms - timed_ms) / 1e3
+        while time.time() < t_end:
+            step()
+        torch.cuda.synchronize(device)
+        clocks.end()
+
+
 # Every configuration the headline metric covers (N = 4680 to 32760), timed in
 # the same run as the headline: the toy, the KV-cache step, the shape sweep, the
 # full sequence, and the one-step and chunk-causal training forms (the three
@@ -286,10 +298,11 @@ EXTRA_WORKLOADS = ["toy_256_f32", "kvcache_4680x32760_bf16", "sweep_2048_f16", "
                    "train_32760_bf16_causal"]
 
 
-def extra_configs(m, args, device, stream, flush_buf, peaks, world):
+def extra_configs(m, args, device, stream, flush_buf, peaks, world, clocks=None):
     """ms per call (median of CUDA-event-timed steps), effective TFLOP/s and
     the whole-call roofline fraction of every other configuration, with dense
-    SDPA on the same tensors as context."""
+    SDPA on the same tensors as context, and the SM clocks sampled while each
+    one ran (a 1000 W part settles lower under the long full-sequence calls)."""
     res = {}
     for name in EXTRA_WORKLOADS:
         if name == args.workload:
@@ -301,7 +314,9 @@ def extra_configs(m, args, device, stream, flush_buf, peaks, world):
         out = torch.empty(qd.shape, dtype=torch.float32, device=device)
         flush = flush_buf if model["io_bytes"] < 4 * L2_BYTES else None
         steps = max(5, min(args.steps, 20 if model["flops"] > 5e11 else 50))
-        times, _, _ = time_forward(m, w, qd, kd, vd, out, steps, args.warmup, stream, flush, world)
+        times, _, step = time_forward(m, w, qd, kd, vd, out, steps, args.warmup, stream, flush, world, clocks)
+        if clocks:
+            keep_loaded(step, sum(times), device, clocks)
         ms = max_over_ranks(statistics.median(times), world, device)
         rec = {"ms_per_call": ms, "mean_ms": statistics.fmean(times), "steps": steps,
                "value": world * model["flops"] / (ms * 1e-3) / 1e12, "unit": "TFLOP/s",
@@ -311,6 +326,8 @@ def extra_configs(m, args, device, stream, flush_buf, peaks, world):
                           "chunk_frames": w.chunk_frames},
                "call_roofline": call_roofline(w, model, peaks, ms),
                "l2": "flushed between steps" if flush is not None else "inputs larger than L2"}
+        if clocks:
+            rec["clocks"] = clocks.summary()
         rec["dense_context"] = dense_context(qd, kd, vd, model, flush, stream, ms)
         res[name] = rec
         del qd, kd, vd, out
@@ -338,14 +355,8 @@ def run_ours(args, rank, world, device):
     per_step, launches, step = time_forward(m, w, qd, kd, vd, out, args.steps, args.warmup, stream, flush,
                                             world, clocks)
     ms = statistics.median(per_step)
-    # If the timed steps were short, keep sampling clocks for a moment under load.
-    if sum(per_step) < 1000.0:
-        t_end = time.time() + 1.0
-        while time.time() < t_end:
-            step()
-        torch.cuda.synchronize(device)
-        clocks.end()
-    clocks.stop()
+    keep_loaded(step, sum(per_step), device, clocks)
+    head_clocks = clocks.summary()
 
     ms = max_over_ranks(ms, world, device)
     mean_ms = max_over_ranks(statistics.fmean(per_step), world, device)
@@ -410,8 +421,9 @@ def run_ours(args, rank, world, device):
     del qh, kh, vh, oh
 
     # the per-configuration timings are single-GPU figures: one run (N = 1) gives them
-    configs = extra_configs(m, args, device, stream, flush_buf, peaks, world) \
+    configs = extra_configs(m, args, device, stream, flush_buf, peaks, world, clocks) \
         if (world == 1 and not args.no_configs) else {}
+    clocks.stop()
 
     es = q.element_size()
     rec = {
@@ -444,7 +456,7 @@ def run_ours(args, rank, world, device):
                 "h2d_bytes_per_step": (q.numel() + k.numel() + v.numel()) * es,
                 "d2h_bytes_per_step": q.numel() * 4},
         "gpu_launches": launches,
-        "clocks": clocks.summary(),
+        "clocks": head_clocks,
         "dense_context": dense,
         "backward": backward,
         "configs": configs,
