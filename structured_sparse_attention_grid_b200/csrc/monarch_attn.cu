@@ -148,6 +148,11 @@ struct Plan {
   size_t off[kRegions];
   size_t counters;   // int [1 + BH]: the ticket and per-head R-item counts of onestep_tc
   size_t total;
+  // key tiles per R-step CTA; 0: chosen for this plan's geometry.  A call that
+  // runs its units in groups sets the whole call's choice: the stacking of
+  // key tiles sets the order of the MMAs' sums, so every group then computes
+  // the bits of the one-call forward.
+  int r_group = 0;
 };
 
 constexpr int kMaxB2 = 64;
@@ -475,7 +480,7 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   const int sm_count = sm_count_of_device();
   const long long col_items = (long long)g.BH * g.b2 * ((g.b1k + 2 * kTile - 1) / (2 * kTile));
   const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
-  const int r_group = r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
+  const int r_group = p.r_group ? p.r_group : r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   if (p.iters == 1 && onestep_fused()) {
     // one refinement step: the R step and the output pass in one kernel
@@ -951,7 +956,41 @@ int workspace_pool(cudaMemPool_t* out) {
 
 // Copy streams of the host-buffer entry point, one pair per device, created
 // on first use (non-blocking) and kept for the life of the process.
-constexpr int kHostGroups = 8;   // most groups one host-buffer call splits its units into
+constexpr int kHostGroups = 16;  // most groups one host-buffer call splits its units into
+
+// Unit counts of the groups of a host-buffer call.  Groups hold about 10 MB
+// of input each (at most 8 of them; one group below 10 MB).  With two or more,
+// the first and the last groups ramp (1, 2, 4, 8 units while smaller than the
+// others): the copy-out starts sooner, runs beside more of the copy-in, and
+// the forward and copy-out of the last group, which nothing overlaps, are
+// short.  Measured on B200 (full_32760, 24 heads): 1, 2, 3 x 6, 2, 1 took
+// 14.4 ms against 15.0 ms for 3 x 8; the 4680-token grid is bound by the host
+// link either way.
+int host_groups(long long U, long long in_bytes, long long* sizes) {
+  int ng = (int)std::max<long long>(1, std::min<long long>({in_bytes / (10LL << 20), U, 8LL}));
+  const long long gs = (U + ng - 1) / ng;
+  ng = (int)((U + gs - 1) / gs);
+  if (ng == 1) {
+    sizes[0] = U;
+    return 1;
+  }
+  long long ramp[4];
+  int nr = 0;
+  long long left = U;
+  for (long long r = 1; r < gs && nr < 4 && left >= 2 * r + gs; r *= 2) {
+    ramp[nr++] = r;
+    left -= 2 * r;
+  }
+  int n = 0;
+  for (int i = 0; i < nr; ++i) sizes[n++] = ramp[i];
+  while (left > 0) {
+    const long long t = std::min(gs, left);
+    sizes[n++] = t;
+    left -= t;
+  }
+  for (int i = nr - 1; i >= 0; --i) sizes[n++] = ramp[i];
+  return n;
+}
 
 struct HostStreams {
   cudaStream_t in = nullptr, out = nullptr;
@@ -1239,14 +1278,14 @@ int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void*
   const size_t es = elem_size(dtype), eo = elem_size(out_dtype);
   const size_t qu = (size_t)p.g.Nq * d * es, ku = (size_t)p.g.Nk * d * es, ou = (size_t)p.g.Nq * d * eo;
   const long long in_bytes = (long long)(U * (qu + 2 * ku));
-  // about 10 MB of input per group: smaller groups make the forward of a group
-  // latency-bound (measured best: 4 groups for 43 MB, 8 for 216 MB and 604 MB)
-  int ng = (int)std::max<long long>(1, std::min<long long>({in_bytes / (10LL << 20), U, (long long)kHostGroups}));
-  const long long gs = (U + ng - 1) / ng;
-  ng = (int)((U + gs - 1) / gs);
-  Plan pg;   // one group of gs units (B = 1, heads = gs); the last group may be smaller
+  long long sizes[kHostGroups], starts[kHostGroups];
+  const int ng = host_groups(U, in_bytes, sizes);
+  for (int i = 0; i < ng; ++i) starts[i] = i ? starts[i - 1] + sizes[i - 1] : 0;
+  const long long gs = *std::max_element(sizes, sizes + ng);
+  Plan pg;   // the largest group (B = 1, heads = gs): its workspace serves every group
   if ((rc = make_plan(1, (int)gs, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pg, chunk_frames)))
     return rc;
+  pg.r_group = r_step_group(p.g, sm_count_of_device());
   const size_t oq = 0, ok = align256(U * qu), ov = ok + align256(U * ku), oo = ov + align256(U * ku);
   const size_t ow = oo + align256(U * ou);
   char* buf = nullptr;
@@ -1263,7 +1302,7 @@ int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void*
     cudaEventRecord(ev_alloc, stream);
     cudaStreamWaitEvent(hs.in, ev_alloc, 0);
     for (int gi = 0; gi < ng && rc == MONARCH_OK; ++gi) {
-      const long long u0 = gi * gs, n = std::min<long long>(gs, U - u0);
+      const long long u0 = starts[gi], n = sizes[gi];
       const char* qh = static_cast<const char*>(q_host);
       const char* kh = static_cast<const char*>(k_host);
       const char* vh = static_cast<const char*>(v_host);
@@ -1274,11 +1313,12 @@ int monarch_attn_fwd_host_ex(const void* q_host, const void* k_host, const void*
       cudaEventRecord(ev[gi], hs.in);
     }
     for (int gi = 0; gi < ng && rc == MONARCH_OK; ++gi) {
-      const long long u0 = gi * gs, n = std::min<long long>(gs, U - u0);
+      const long long u0 = starts[gi], n = sizes[gi];
       Plan pn = pg;
       if (n != gs &&
           (rc = make_plan(1, (int)n, T, H, W, d, tile_h, tile_w, iters, kv_len, dtype, out_dtype, &pn, chunk_frames)))
         break;
+      pn.r_group = pg.r_group;
       cudaStreamWaitEvent(stream, ev[gi], 0);
       rc = dispatch(pn, buf + oq + u0 * qu, buf + ok + u0 * ku, buf + ov + u0 * ku, buf + oo + u0 * ou, buf + ow,
                     stream);

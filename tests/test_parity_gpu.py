@@ -197,9 +197,10 @@ def test_host_buffer_entry_point(cuda_lib):
 
 @pytest.mark.parametrize("name", ["chunk_4680_bf16", "kvcache_4680x32760_bf16"])
 def test_host_buffer_groups_match_the_device_call(name, cuda_lib):
-    """The host entry point pipelines groups of (batch, head) units (4 and 6
-    groups here, the last one shorter for the KV cache); every row is computed
-    by the same arithmetic as in one device call over all units."""
+    """The host entry point pipelines groups of (batch, head) units (1, 2, 3,
+    3, 2, 1 heads for chunk_4680 and 1, 2, 2, 2, 2, 2, 1 for the KV cache);
+    every row is computed by the same arithmetic, key tiles stacked the same
+    way, as in one device call over all units."""
     w = WORKLOADS[name]
     q, k, v = make_inputs(w)
     out = torch.empty(q.shape, dtype=torch.float32).pin_memory()
@@ -210,8 +211,8 @@ def test_host_buffer_groups_match_the_device_call(name, cuda_lib):
 
 
 def test_host_buffer_groups_with_the_chunk_mask(cuda_lib):
-    """The masked host entry point (6 groups of 2 heads) equals the masked
-    device call."""
+    """The masked host entry point (groups of 1, 2, 2, 2, 2, 2, 1 heads)
+    equals the masked device call."""
     w = _custom("bf16", 6, 30, 52, 128, 6, 4, 2, B=1, heads=12, C=2)
     q, k, v = make_inputs(w)
     out = torch.empty(q.shape, dtype=torch.float32).pin_memory()
