@@ -16,10 +16,12 @@
 //                                    memory, N = d)
 // R is zero outside the diagonal blocks, so these are the per-tile products.
 // The epilogue splits each row into hi / lo planes, stages them in shared
-// memory in the swizzled box layout and one thread stores them with per-tile
-// TMA boxes into [plane][BH][b2][b1k][d] (position-major), the layout the L
-// step reads.  In the first step the exact query rows, already in shared
-// memory, go out the same way as the block-major copy of q.
+// memory in the swizzled box layout, the G tiles' rows packed (tile g at rows
+// [g b2, (g + 1) b2)), and one thread stores each (plane, d half) with one
+// TMA box of all G tiles into [plane][BH][b2][b1k][d] (position-major), the
+// layout the L step reads: the store map walks positions before tiles, so
+// the box lands tile by tile.  In the first step the exact query rows go out
+// the same way as the block-major copy of q.
 //
 // Loads: keys, values and exact query rows come through the 4-D grid map
 // (d, W, H, frames) with one tile per box, so the grid -> block permutation is
@@ -50,8 +52,10 @@ struct RtcMaps {
   CUtensorMap qt;   // q~ planes  {d, b1k, 2*BH*b2},      box {64, 1, b2}
   CUtensorMap qm;   // mean-query planes (KV init) {d, 1, 2*BH*b2}, box {64, 1, b2}
   CUtensorMap qb;   // block-major q, f16 (store) {d, b1q, BH*b2},   box {64, 1, b2}
-  CUtensorMap kt;   // k~ planes, f16 (store)     {d, b1k, 2*BH*b2}, box {64, 1, b2}
-  CUtensorMap z;    // z planes, f16 (store) {d, b1k, 2*BH*b2},   box {64, 1, b2}
+  // stores of G tiles at once, positions before tiles (strides b1k d, d):
+  CUtensorMap qbg;  // block-major q, f16 {d, b2, b1q, BH},     box {64, b2, G, 1}
+  CUtensorMap kt;   // k~ planes, f16     {d, b2, b1k, 2*BH},   box {64, b2, G, 1}
+  CUtensorMap z;    // z planes, f16      {d, b2, b1k, 2*BH},   box {64, b2, G, 1}
 };
 
 // Planes written by the R step.
@@ -215,18 +219,6 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
         }
       }
       ok = ptx::mbar_wait(bar_ld, 0);
-      if (ok && mode != QT_BUFFER && !bf16) {
-        // first step, f16 input: the exact query rows just loaded are also the
-        // block-major copy of q that the L step reads
-        for (int gg = 0; gg < Gn; ++gg) {
-          const int c1 = c1_0 + gg;
-          if (!exact_q(c1)) continue;
-          for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(&maps.qb, sA + hf * kRBox + (uint32_t)(gg * rs) * 128, hf * 64, c1 - g.off,
-                              bh * g.b2);
-        }
-        ptx::bulk_commit();
-      }
       ptx::tc_fence_after();
       // S = A K^T: both operands K-major (d along the 128-byte rows)
       if (ok) {
@@ -243,6 +235,19 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
             if (use_lo) ptx::mma_f16_ss(tS, dA + ((NH * kRBox) >> 4) + off, dK + off, idS, 1);
           }
         ptx::mma_commit(bar_s);
+      }
+      if (ok && mode != QT_BUFFER && !bf16) {
+        // first step, f16 input: the exact query rows just loaded are also the
+        // block-major copy of q that the L step reads (the store, like S,
+        // only reads A, so it goes out after the score MMAs are issued)
+        for (int gg = 0; gg < Gn; ++gg) {
+          const int c1 = c1_0 + gg;
+          if (!exact_q(c1)) continue;
+          for (int hf = 0; hf < NH; ++hf)
+            ptx::tma_store_3d(&maps.qb, sA + hf * kRBox + (uint32_t)(gg * rs) * 128, hf * 64, c1 - g.off,
+                              bh * g.b2);
+        }
+        ptx::bulk_commit();
       }
       if (final_step) {
         // V lands in the A hi plane once the score MMAs and the q copy (its
@@ -292,6 +297,10 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
     const int gg = r / rs, a2 = r - gg * rs;
     const int c1 = c1_0 + gg;
     const bool valid = gg < Gn && a2 < g.b2;
+    // staging row of this TMEM lane: the G tiles packed at b2 rows, the
+    // shared-memory order of one store box of all of them
+    const bool staged = gg < G && a2 < g.b2;
+    const int srow = gg * g.b2 + a2;
     const uint32_t lane_off = (uint32_t)(32 * qw) << 16;
     constexpr int kSeg = NH * 4;                // 16-byte chunks of a row per half
     bool ok = true;
@@ -300,14 +309,19 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
     // First step, bf16 input: the L step reads q in f16 (exact for |q| <
     // 65504; larger finite magnitudes set kErrRange).  The loaded rows are
     // converted into the A lo plane and stored from there as the block-major
-    // copy of q.
+    // copy of q: without a KV cache in the packed staging order, one box of
+    // all G tiles per d half; with one per exact tile, as loaded (a group may
+    // also hold cached tiles, which have no copy).
+    const bool packed_q = mode == QT_IDENTITY;
     auto convert_and_store_q = [&]() {
       if (valid && exact_q(c1)) {
         bool over = false;
+        const int wrow = packed_q ? srow : r;   // row of the converted copy in the A lo plane
 #pragma unroll
         for (int k = 0; k < kSeg; ++k) {
           const int i = half * kSeg + k, hf = i >> 3, ch = i & 7;
           const uint32_t o = hf * kRBox + r * 128 + ((ch ^ (r & 7)) << 4);
+          const uint32_t ow = hf * kRBox + wrow * 128 + ((ch ^ (wrow & 7)) << 4);
           uint4 u = *reinterpret_cast<const uint4*>(sA + o);
           uint32_t* wv = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
@@ -318,7 +332,7 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
             const __half2 hv = __floats2half2_rn(__uint_as_float(wv[e] << 16), __uint_as_float(wv[e] & 0xFFFF0000u));
             wv[e] = *reinterpret_cast<const uint32_t*>(&hv);
           }
-          *reinterpret_cast<uint4*>(sA + NH * kRBox + o) = u;
+          *reinterpret_cast<uint4*>(sA + NH * kRBox + ow) = u;
         }
         if (over) atomicExch(&ptx::g_device_error, ptx::kErrRange);
       }
@@ -327,11 +341,16 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
       if (final_step && lane == 0) ptx::mbar_arrive(bar_q);
       ptx::named_bar(bar_row, kRtcRowThreads);
       if (tid == 0 && ok) {
-        for (int t = 0; t < Gn; ++t) {
-          if (!exact_q(c1_0 + t)) continue;
+        if (packed_q) {
           for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * rs) * 128, hf * 64,
-                              c1_0 + t - g.off, bh * g.b2);
+            ptx::tma_store_4d(&maps.qbg, sA + (NH + hf) * kRBox, hf * 64, 0, c1_0, bh);
+        } else {
+          for (int t = 0; t < Gn; ++t) {
+            if (!exact_q(c1_0 + t)) continue;
+            for (int hf = 0; hf < NH; ++hf)
+              ptx::tma_store_3d(&maps.qb, sA + (NH + hf) * kRBox + (uint32_t)(t * rs) * 128, hf * 64,
+                                c1_0 + t - g.off, bh * g.b2);
+          }
         }
         ptx::bulk_commit();
       }
@@ -456,23 +475,24 @@ __device__ __forceinline__ void r_step_item(const RtcMaps& maps, const TQ* __res
         for (int i = 0; i < 8; ++i)
           tc::split2<__half>(make_float2(__uint_as_float(a[k & 1][2 * i]), __uint_as_float(a[k & 1][2 * i + 1])),
                              hi[i], lo[i]);
+        if (staged) {
 #pragma unroll
-        for (int v = 0; v < 2; ++v) {
-          const int ch8 = (cc & 3) * 2 + v;
-          const uint32_t o = (cc >> 2) * kRBox + r * 128 + ((ch8 ^ (r & 7)) << 4);
-          *reinterpret_cast<uint4*>(shi + o) = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
-          *reinterpret_cast<uint4*>(slo + o) = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+          for (int v = 0; v < 2; ++v) {
+            const int ch8 = (cc & 3) * 2 + v;
+            const uint32_t o = (cc >> 2) * kRBox + srow * 128 + ((ch8 ^ (srow & 7)) << 4);
+            *reinterpret_cast<uint4*>(shi + o) = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
+            *reinterpret_cast<uint4*>(slo + o) = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
+          }
         }
       }
       ptx::fence_proxy_async();
     };
-    // one thread: a box of b2 rows per (tile, plane, d half)
+    // one thread: one box of all G tiles per (plane, d half); tiles past the
+    // end of the head fall outside the tensor and are not written
     auto store_tiles = [&](const CUtensorMap* map, const uint8_t* shi, const uint8_t* slo) {
-      for (int t = 0; t < Gn; ++t)
-        for (int p = 0; p < 2; ++p)
-          for (int hf = 0; hf < NH; ++hf)
-            ptx::tma_store_3d(map, (p ? slo : shi) + hf * kRBox + (uint32_t)(t * rs) * 128, hf * 64, c1_0 + t,
-                              (p * g.BH + bh) * g.b2);
+      for (int p = 0; p < 2; ++p)
+        for (int hf = 0; hf < NH; ++hf)
+          ptx::tma_store_4d(map, (p ? slo : shi) + hf * kRBox, hf * 64, 0, c1_0, p * g.BH + bh);
       ptx::bulk_commit();
     };
     ok = ok && ptx::mbar_wait(bar_acc, 0);

@@ -395,7 +395,7 @@ int tc_l_maps(const Geo& g, const Work& w, const __half* kt_hi, const __half* z_
 // forward and the backward's recompute).
 template <typename TQ, int D>
 int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& w, TcPlanes<TQ>& planes,
-               tc::Maps& maps, RtcMaps& rmaps) {
+               tc::Maps& maps, RtcMaps& rmaps, int G) {
   planes.kt_hi = reinterpret_cast<__half*>(w.kt);
   planes.z_hi = reinterpret_cast<__half*>(w.z);
   planes.plane = (long long)g.BH * g.b2 * g.b1k * D;
@@ -420,10 +420,22 @@ int tc_prepare(const Geo& g, const TQ* q, const TQ* k, const TQ* v, const Work& 
         (rc = make_map(&rmaps.k, k, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.v, v, dq, 4, dk4, s4, box4, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (rc = make_map(&rmaps.qt, w.qt, dq, 3, dt3, st3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&rmaps.qm, w.qbar, dq, 3, dm3, sm3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&rmaps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
+        (rc = make_map(&rmaps.qm, w.qbar, dq, 3, dm3, sm3, boxt, CU_TENSOR_MAP_SWIZZLE_128B)))
+      return rc;
+    // R-step stores of all G tiles of an item in one box per (plane, d half):
+    // dims (d, position, tile, plane*BH + head), the position stride above the
+    // tile stride, so the box's shared-memory rows are tile-major (tile g at
+    // rows [g b2, (g + 1) b2))
+    cuuint32_t boxg[4] = {64, (cuuint32_t)g.b2, (cuuint32_t)G, 1};
+    cuuint64_t dg4[4] = {(cuuint64_t)D, (cuuint64_t)g.b2, (cuuint64_t)g.b1k, 2 * (cuuint64_t)g.BH};
+    cuuint64_t sg4[3] = {(cuuint64_t)g.b1k * D * 2, (cuuint64_t)D * 2, (cuuint64_t)g.b2 * g.b1k * D * 2};
+    cuuint64_t dgq[4] = {(cuuint64_t)D, (cuuint64_t)g.b2, (cuuint64_t)g.b1q, (cuuint64_t)g.BH};
+    cuuint64_t sgq[3] = {(cuuint64_t)g.b1q * D * 2, (cuuint64_t)D * 2, (cuuint64_t)g.b2 * g.b1q * D * 2};
+    if ((rc = make_map(&rmaps.kt, planes.kt_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, dg4, sg4, boxg,
                        CU_TENSOR_MAP_SWIZZLE_128B)) ||
-        (rc = make_map(&rmaps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, dt3, st3, boxt,
+        (rc = make_map(&rmaps.z, planes.z_hi, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, dg4, sg4, boxg,
+                       CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (rc = make_map(&rmaps.qbg, w.qb, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4, dgq, sgq, boxg,
                        CU_TENSOR_MAP_SWIZZLE_128B)))
       return rc;
     cuuint64_t db3[3] = {(cuuint64_t)D, (cuuint64_t)g.b1q, (cuuint64_t)g.BH * g.b2};
@@ -450,7 +462,8 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   tc::Maps maps;
   RtcMaps rmaps;
   int rc;
-  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
+  const int r_group = p.r_group ? p.r_group : r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps, r_group))) return rc;
 
   constexpr size_t smem_lse = tc::lse_smem<D>();
   constexpr size_t smem_out = tc::row_smem<D, true>();
@@ -480,7 +493,6 @@ int run_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, TO* out, char* 
   const int sm_count = sm_count_of_device();
   const long long col_items = (long long)g.BH * g.b2 * ((g.b1k + 2 * kTile - 1) / (2 * kTile));
   const dim3 grid_k((unsigned)std::min<long long>(col_items, sm_count));
-  const int r_group = p.r_group ? p.r_group : r_step_group(g, sm_count_of_device());   // key tiles per R-step CTA
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   if (p.iters == 1 && onestep_fused()) {
     // one refinement step: the R step and the output pass in one kernel
@@ -751,7 +763,8 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
   tc::Maps maps;
   RtcMaps rmaps;
   int rc;
-  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
+  const int r_group = r_step_group(g, sm_count_of_device());
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps, r_group))) return rc;
   tcb::BwdMaps bmaps;
   {
     const cuuint64_t rows = (cuuint64_t)g.BH * g.b2;
@@ -788,7 +801,6 @@ int run_bwd_tc(const BwdPlan& bp, const TQ* q, const TQ* k, const TQ* v, const T
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
-  const int r_group = r_step_group(g, sm_count_of_device());
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   launch(MONARCH_PHASE_R_STEP, st, [&] {
     launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1,
@@ -846,7 +858,8 @@ int run_fwd_train_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, float
   tc::Maps maps;
   RtcMaps rmaps;
   int rc;
-  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps))) return rc;
+  const int r_group = r_step_group(g, sm_count_of_device());
+  if ((rc = tc_prepare<TQ, D>(g, q, k, v, w, planes, maps, rmaps, r_group))) return rc;
   constexpr size_t smem_out = tc::row_smem<D, true>();
   constexpr size_t smem_r = rtc_smem<D>();
   static std::atomic<bool> attrs_set[kMaxDevices];
@@ -861,7 +874,6 @@ int run_fwd_train_tc(const Plan& p, const TQ* q, const TQ* k, const TQ* v, float
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
   }
   const dim3 grid_q((g.b1q + 2 * kTile - 1) / (2 * kTile), g.b2, g.BH);
-  const int r_group = r_step_group(g, sm_count_of_device());
   const dim3 grid_r((g.b1k + r_group - 1) / r_group, g.BH);
   launch(MONARCH_PHASE_R_STEP, st, [&] {
     launch_pdl(r_step_tc5<TQ, D>, grid_r, dim3(kRtcThreads), smem_r, st, rmaps, q, w, planes, g, (int)QT_IDENTITY, 1,
