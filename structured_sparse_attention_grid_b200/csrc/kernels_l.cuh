@@ -406,23 +406,39 @@ __device__ __forceinline__ void l_row_item(TO* __restrict__ out, const Maps& map
         const int sp = a1 / g.pb1q;
         const long long tok = a1 < g.b1q ? token_of(g, a1 - sp * g.pb1q, a2 * g.pk + sp) : 0;
         TO* orow = out + ((long long)bh * g.Nq + tok) * D + hf * (D / 2);
+        // 32-byte stores when the caller's buffer allows them (every row
+        // offset is a multiple of 32 bytes; the ABI promises 16 for the base)
+        const bool wide = (reinterpret_cast<uintptr_t>(out) & 31) == 0;
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[16];
           ptx::tmem_ld16(tO(t) + lane_off + hf * (D / 2) + cc * 16, o);
           ptx::tmem_wait_ld();
           if (a1 < g.b1q && ok) {
+            if constexpr (sizeof(TO) == 4) {
 #pragma unroll
-            for (int i = 0; i < 16; i += 4) {
-              if constexpr (sizeof(TO) == 4) {
-                *reinterpret_cast<float4*>(orow + cc * 16 + i) =
-                    make_float4(__uint_as_float(o[i]) * inv, __uint_as_float(o[i + 1]) * inv,
-                                __uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+              for (int i = 0; i < 16; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * inv);
+              if (wide) {
+                ptx::st_global_v8(orow + cc * 16, *reinterpret_cast<const uint32_t(*)[8]>(o));
+                ptx::st_global_v8(orow + cc * 16 + 8, *reinterpret_cast<const uint32_t(*)[8]>(o + 8));
               } else {
-                TO v4[4];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) v4[e] = from_f<TO>(__uint_as_float(o[i + e]) * inv);
-                *reinterpret_cast<uint2*>(orow + cc * 16 + i) = *reinterpret_cast<uint2*>(v4);
+                for (int i = 0; i < 16; i += 4)
+                  *reinterpret_cast<uint4*>(orow + cc * 16 + i) = make_uint4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+              }
+            } else {
+              uint32_t pk[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                TO two[2] = {from_f<TO>(__uint_as_float(o[2 * e]) * inv), from_f<TO>(__uint_as_float(o[2 * e + 1]) * inv)};
+                pk[e] = *reinterpret_cast<const uint32_t*>(two);
+              }
+              if (wide) {
+                ptx::st_global_v8(orow + cc * 16, pk);
+              } else {
+#pragma unroll
+                for (int i = 0; i < 8; i += 4)
+                  *reinterpret_cast<uint4*>(orow + cc * 16 + 2 * i) = make_uint4(pk[i], pk[i + 1], pk[i + 2], pk[i + 3]);
               }
             }
           }
@@ -984,14 +1000,9 @@ l_col(const __grid_constant__ Maps maps, const float* __restrict__ hbuf, TQ* __r
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             split2<TQ>(mul2(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), inv2), hi[e], lo[e]);
-          if (c1 < g.b1k && ok) {
-            uint4* ph = reinterpret_cast<uint4*>(dst + cc * 16);
-            uint4* pl = reinterpret_cast<uint4*>(dst + plane + cc * 16);
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              ph[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
-              pl[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
-            }
+          if (c1 < g.b1k && ok) {   // 32 bytes a store (rows are D elements, planes 256-byte aligned)
+            ptx::st_global_v8(dst + cc * 16, hi);
+            ptx::st_global_v8(dst + plane + cc * 16, lo);
           }
         }
         // the accumulator is read: the next item may overwrite it

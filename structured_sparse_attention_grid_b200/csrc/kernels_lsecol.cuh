@@ -355,14 +355,9 @@ l_lsecol(const __grid_constant__ Maps maps, float* __restrict__ lse, TQ* __restr
 #pragma unroll
         for (int e = 0; e < 8; ++e)
           split2<TQ>(mul2(make_float2(__uint_as_float(o[2 * e]), __uint_as_float(o[2 * e + 1])), inv2), hi[e], lo[e]);
-        if (c1 < g.b1k && ok) {
-          uint4* ph = reinterpret_cast<uint4*>(dst + cc * 16);
-          uint4* pl = reinterpret_cast<uint4*>(dst + plane + cc * 16);
-#pragma unroll
-          for (int v = 0; v < 2; ++v) {
-            ph[v] = make_uint4(hi[4 * v], hi[4 * v + 1], hi[4 * v + 2], hi[4 * v + 3]);
-            pl[v] = make_uint4(lo[4 * v], lo[4 * v + 1], lo[4 * v + 2], lo[4 * v + 3]);
-          }
+        if (c1 < g.b1k && ok) {   // 32 bytes a store (rows are D elements, planes 256-byte aligned)
+          ptx::st_global_v8(dst + cc * 16, hi);
+          ptx::st_global_v8(dst + plane + cc * 16, lo);
         }
       }
     }

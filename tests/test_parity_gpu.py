@@ -186,6 +186,25 @@ def test_output_in_input_dtype_matches_the_oracle(name, cuda_lib):
     _compare(w, out, q, k, v, store_bits=STORE_BITS[w.dtype])
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16], ids=["f32", "bf16"])
+def test_output_buffer_with_16_byte_alignment(out_dtype, cuda_lib):
+    """The output pass stores 32 bytes at a time when the caller's buffer is
+    32-byte aligned and 16 bytes at a time otherwise (the ABI asks for 16);
+    both give the same bits."""
+    w = _custom("bf16", 5, 12, 20, 128, 4, 4, 2)
+    q, k, v = (t.cuda() for t in make_inputs(w))
+    n = q.numel()
+    a = torch.empty(q.shape, dtype=out_dtype, device=q.device)
+    shift = 16 // a.element_size()
+    b = torch.empty(n + shift, dtype=out_dtype, device=q.device)[shift:].view(q.shape)
+    assert a.data_ptr() % 32 == 0 and b.data_ptr() % 32 == 16
+    for o in (a, b):
+        m.monarch_attn_fwd(q, k, v, o, w.T, w.H, w.W, w.th, w.tw, w.iters)
+    torch.cuda.synchronize()
+    assert m.device_error() == 0
+    assert torch.equal(a, b)
+
+
 def test_host_buffer_entry_point(cuda_lib):
     w = WORKLOADS["toy_256_f32"]
     q, k, v = make_inputs(w)
