@@ -206,17 +206,21 @@ __device__ __forceinline__ void mma_accum(uint32_t tacc, uint32_t ta, int pa, ui
     ptx::mma_f16_ts(tacc, ta + kk * 16 + pa * 8, db + ((kk * 2048) >> 4), idA, !(first && kk == 0));
 }
 
-// Writes 16 accumulator columns of this thread's row, times `scale`, as f32.
+// Writes 16 accumulator columns of this thread's row, times `scale`, as f32
+// with two 32-byte stores (dst is a workspace row: 32-byte aligned).
 __device__ __forceinline__ void store_acc16(uint32_t taddr, float scale, float* dst, bool ok) {
   uint32_t o[16];
   ptx::tmem_ld16(taddr, o);
   ptx::tmem_wait_ld();
   if (!ok) return;
-  float4* p = reinterpret_cast<float4*>(dst);
+  uint32_t a[8], b[8];
 #pragma unroll
-  for (int v = 0; v < 4; ++v)
-    p[v] = make_float4(__uint_as_float(o[4 * v]) * scale, __uint_as_float(o[4 * v + 1]) * scale,
-                       __uint_as_float(o[4 * v + 2]) * scale, __uint_as_float(o[4 * v + 3]) * scale);
+  for (int i = 0; i < 8; ++i) {
+    a[i] = __float_as_uint(__uint_as_float(o[i]) * scale);
+    b[i] = __float_as_uint(__uint_as_float(o[8 + i]) * scale);
+  }
+  ptx::st_global_v8(dst, a);
+  ptx::st_global_v8(dst + 8, b);
 }
 
 // ===========================================================================
