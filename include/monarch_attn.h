@@ -170,13 +170,17 @@ size_t monarch_attn_bwd_workspace_bytes(int B, int heads, int T, int H, int W, i
 
 /* End-to-end variant on HOST buffers: copies q, k, v host->device, runs the
  * forward and copies out device->host, then synchronises `stream` before
- * returning (so `out` is ready).  The (batch, head) units are split into up
- * to 8 groups (about 10 MB of input each) whose copies overlap: copies in run on a library-owned stream,
- * each group's forward on `stream` after its inputs have landed, its copy
- * out on a second library-owned stream (one pair of non-blocking streams per
- * device, kept for the process).  Device buffers are allocated stream-ordered
- * and freed before return.  Pinned host memory gives asynchronous,
- * overlapping copies; pageable memory works but is slower. */
+ * returning (so `out` is ready).  The (batch, head) units are split into
+ * groups whose copies overlap: about 10 MB of input each (at most 8 such
+ * groups), the first and last ones smaller (1, 2, 4 ... units) so that the
+ * copy-out starts early and the last group's tail is short.  Copies in run
+ * on a library-owned stream, each group's forward on `stream` after its
+ * inputs have landed (with the R-step grouping of the one-call forward, so
+ * the result has the same bits), its copy out on a second library-owned
+ * stream (one pair of non-blocking streams per device, kept for the
+ * process).  Device buffers are allocated stream-ordered and freed before
+ * return.  Pinned host memory gives asynchronous, overlapping copies;
+ * pageable memory works but is slower. */
 int monarch_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                           void* out_host, int B, int heads, int T, int H, int W, int d,
                           int tile_h, int tile_w, int iters, long kv_len,
