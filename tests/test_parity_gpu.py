@@ -106,6 +106,11 @@ EDGE = [
     # largest supported tile (64 positions) and b1 exactly one 128-row block
     _custom("f16", 2, 32, 32, 64, 8, 8, 2),
     _custom("bf16", 8, 16, 16, 128, 4, 2, 2, B=1, heads=2),
+    # 64 positions with d = 128 (two tiles an R-step item): the fused L step,
+    # a KV cache, and 288 tiles a head (separate LSE and column passes)
+    _custom("bf16", 2, 16, 16, 128, 8, 8, 2),
+    _custom("bf16", 1, 16, 16, 128, 8, 8, 2, Tk=3),
+    _custom("bf16", 8, 48, 48, 128, 8, 8, 2, B=1, heads=1),
     # positions per tile not a multiple of 8 (padded rows inside each stacked
     # R-step tile), with and without a KV cache, both head sizes
     _custom("bf16", 2, 9, 10, 128, 3, 5, 2),
