@@ -43,10 +43,9 @@ L2_BYTES = 126 * 2**20
 # a kernel without a capture of its current code reports null.
 NCU_TRAFFIC = {
     ("chunk_4680_bf16", "r_step"): 48.13e6,     # mean of the call's two launches (30.15 and 66.11 MB)
-    ("chunk_4680_bf16", "l_lsecol"): 45.37e6,
+    ("chunk_4680_bf16", "l_lsecol"): 44.82e6,
     ("chunk_4680_bf16", "l_out"): 76.24e6,
     ("full_32760_bf16", "l_col"): 897.1e6,      # 299.03 MB (mean of two launches) at 8 heads x 3
-    ("full_32760_bf16", "l_lse"): 419.9e6,      # 139.98 MB at 8 heads x 3
     ("full_32760_bf16", "l_out"): 1341.4e6,     # 447.13 MB at 8 heads x 3
 }
 # FP32 FMA ceiling of the CUDA cores: 148 SMs x 128 lanes x 2 FLOP x 1.965 GHz

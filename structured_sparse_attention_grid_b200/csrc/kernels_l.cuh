@@ -501,7 +501,7 @@ l_row(TO* __restrict__ out, const __grid_constant__ Maps maps, float* __restrict
 // S = q k~_hi^T is one N = 128 MMA group per (tile, block); TMEM: tile t,
 // buffer b at column 256 t + 128 b, so block j + 1 is computed while the
 // softmax reads block j.  The two column halves of a row keep their own
-// running shift and sum and are merged at the end.  About 3/8 of the
+// running shift and sum and are merged at the end.  A quarter of the
 // exponentials run on the FMA pipe (ex2_fma2): with one plane the score MMA
 // has half the columns per exponential of the two-plane passes, so the MUFU
 // unit alone would be the bound.
@@ -698,8 +698,8 @@ l_lse(const __grid_constant__ Maps maps, float* __restrict__ lse, Geo g) {
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 d = add2(x[i], nm);
-            // three pairs in eight on the FMA pipe, the rest on the MUFU unit
-            const float2 e = ((i & 7) >= 5) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
+            // one pair in four on the FMA pipe, the rest on the MUFU unit
+            const float2 e = ((i & 3) == 3) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
             acc2 = add2(acc2, e);
           }
           l = fmaf(l, corr, acc2.x + acc2.y);

@@ -8,7 +8,7 @@
 //
 // Phase A is the arithmetic of l_lse: S = q k~_hi^T (f16, N = 128 keys per
 // MMA group), two column halves per row with their own running shift, merged
-// at the end, three exponential pairs in eight on the FMA pipe; the row LSE
+// at the end, one exponential pair in four on the FMA pipe; the row LSE
 // goes to shared memory (and to the workspace).  Phase B is the arithmetic of
 // l_col for the CTA's single item: S^T = k~_hi q^T + k~_lo q^T per 128-query
 // block, L^T = 2^(x - lse + 15) split into f16 hi / lo over S^T in TMEM,
@@ -249,8 +249,8 @@ l_lsecol(const __grid_constant__ Maps maps, float* __restrict__ lse, TQ* __restr
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
             const float2 d = add2(x[i], nm);
-            // three pairs in eight on the FMA pipe, the rest on the MUFU unit
-            const float2 e = ((i & 7) >= 5) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
+            // one pair in four on the FMA pipe, the rest on the MUFU unit
+            const float2 e = ((i & 3) == 3) ? ex2_fma2(d) : make_float2(ptx::ex2(d.x), ptx::ex2(d.y));
             acc2 = add2(acc2, e);
           }
           l = fmaf(l, corr, acc2.x + acc2.y);
